@@ -1,0 +1,279 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each pin takes a loaded oracle library and raises AssertionError when the
+oracle disagrees with what the page and the mathematics fix.  The sources of
+truth used here are independent of ``oracle/lca_oracle.c``:
+
+* torch float64 library routines (softmax, argmax, scaled_dot_product_attention,
+  matmul) applied to the condensed set built as the page describes it
+  ("Latent-Condensed Transformer for Efficient Long Context Modeling",
+  section 2, "O Algoritmo LCA", steps 1-3);
+* closed forms: zero query (uniform pooling, anchor = first token of each
+  group), groups of identical tokens (LCA = dense attention over one
+  representative per group, because no parameter or bias is added --
+  section 2, "Vantagens Teoricas"), g = 1 and w >= L (nothing condensed, so
+  LCA is dense MLA attention, section 1);
+* invariances: permuting tokens inside a group, a constant RoPE key;
+* constructed exact ties (lowest index wins);
+* brute force over every (g, w) on tiny L.
+
+The same pins are run against deliberately broken copies of the oracle
+(tests/test_oracle_mutants.py) to show that each plausible mistake is caught.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+from oracle import oracle as orc
+from workloads import bf16_bits_to_f32, f32_to_bf16_bits
+
+REL_TOL = 1e-10  # double vs double, different summation orders
+
+
+# ----------------------------------------------------------------------------- helpers
+def rand_inputs(rng, B, H, L, d_c, d_r, dtype="f32"):
+    s_q = 1.0 / math.sqrt(d_c + d_r)
+    q_c = (rng.standard_normal((B, H, d_c)) * s_q).astype(np.float32)
+    q_r = (rng.standard_normal((B, H, d_r)) * s_q).astype(np.float32)
+    c_kv = rng.standard_normal((B, L, d_c)).astype(np.float32)
+    k_r = rng.standard_normal((B, L, d_r)).astype(np.float32)
+    if dtype == "bf16":
+        return tuple(f32_to_bf16_bits(a) for a in (q_c, q_r, c_kv, k_r))
+    return q_c, q_r, c_kv, k_r
+
+
+def widen(a: np.ndarray) -> np.ndarray:
+    if a.dtype == np.uint16:
+        return bf16_bits_to_f32(a).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def partition(L: int, g: int, w: int):
+    """Groups and window by walking the sequence: the last w tokens are the
+    window; full groups of g are then taken from the front while they end
+    before the window; any leftover tokens join the window."""
+    win_start = max(0, L - w)
+    groups, t = [], 0
+    while t + g <= win_start:
+        groups.append(list(range(t, t + g)))
+        t += g
+    window = list(range(t, L))
+    return groups, window
+
+
+def rel_err(a: np.ndarray, b: np.ndarray) -> float:
+    """max over rows of ||a - b||_inf / ||b||_inf."""
+    a = a.reshape(-1, a.shape[-1]); b = b.reshape(-1, b.shape[-1])
+    num = np.abs(a - b).max(axis=1)
+    den = np.maximum(np.abs(b).max(axis=1), 1e-300)
+    return float((num / den).max())
+
+
+def torch_attention(q: np.ndarray, keys: np.ndarray, vals: np.ndarray) -> np.ndarray:
+    """Library softmax attention of one query per head over given rows, scale 1.
+    q [H, d], keys [H, n, d] or [n, d], vals [H, n, d_v] or [n, d_v]."""
+    H = q.shape[0]
+    qt = torch.from_numpy(q)[None, :, None, :]
+    kt = torch.from_numpy(keys)
+    vt = torch.from_numpy(vals)
+    if kt.dim() == 2:
+        kt = kt[None].expand(H, -1, -1)
+    if vt.dim() == 2:
+        vt = vt[None].expand(H, -1, -1)
+    o = F.scaled_dot_product_attention(qt, kt[None], vt[None], scale=1.0)
+    return o[0, :, 0, :].numpy()
+
+
+def torch_lca_seq(qc, qr, C, K, g, w):
+    """LCA for one sequence built from library routines, per the page's steps.
+    Returns (out [H, d_c], anchor [H, n_G])."""
+    H = qc.shape[0]
+    groups, window = partition(C.shape[0], g, w)
+    Ct, Kt = torch.from_numpy(C), torch.from_numpy(K)
+    outs, ancs = [], []
+    for h in range(H):
+        qch, qrh = torch.from_numpy(qc[h]), torch.from_numpy(qr[h])
+        s = Ct @ qch + Kt @ qrh                     # full MLA score of every token
+        keys, vals, anc = [], [], []
+        for G in groups:
+            idx = torch.tensor(G)
+            wts = torch.softmax(s[idx], dim=0)         # step 2: query-aware pooling weights
+            a = G[int(torch.argmax(s[idx]))]           # step 2: highest-scoring token (first max)
+            cbar = wts @ Ct[idx]
+            keys.append(torch.cat([cbar, Kt[a]]))
+            vals.append(cbar)
+            anc.append(a)
+        for t in window:                                # high-fidelity local window
+            keys.append(torch.cat([Ct[t], Kt[t]]))
+            vals.append(Ct[t])
+        keys_np = torch.stack(keys).numpy()
+        vals_np = torch.stack(vals).numpy()
+        q = np.concatenate([qc[h], qr[h]])[None]
+        outs.append(torch_attention(q, keys_np, vals_np)[0])   # step 3
+        ancs.append(anc)
+    return np.stack(outs), np.array(ancs, dtype=np.int32).reshape(H, len(groups))
+
+
+def torch_dense_seq(qc, qr, C, K):
+    q = np.concatenate([qc, qr], axis=1)
+    return torch_attention(q, np.concatenate([C, K], axis=1), C)
+
+
+# ----------------------------------------------------------------------------- pins
+def pin_segmentation(lib):
+    for g in (1, 2, 3, 4, 8, 16):
+        for k in (0, 1, 3):
+            for r in (0, 1, g - 1):
+                L = g * k + r + 5
+                for w in sorted({0, 1, max(g - 1, 0), L - 1, L, L + 5}):
+                    groups, _ = partition(L, g, w)
+                    assert orc.num_groups(L, g, w, lib) == len(groups), (L, g, w)
+
+
+def pin_dense_vs_torch(lib):
+    rng = np.random.default_rng(11)
+    for dtype in ("f32", "bf16"):
+        qc, qr, C, K = rand_inputs(rng, 2, 3, 37, 24, 8, dtype)
+        got = orc.mla(qc, qr, C, K, lib=lib)
+        for b in range(2):
+            ref = torch_dense_seq(widen(qc[b]), widen(qr[b]), widen(C[b]), widen(K[b]))
+            assert rel_err(got[b], ref) < REL_TOL
+
+
+def pin_g1_dense(lib):
+    rng = np.random.default_rng(12)
+    for dtype in ("f32", "bf16"):
+        qc, qr, C, K = rand_inputs(rng, 2, 3, 41, 24, 8, dtype)
+        for w in (0, 5, 40):
+            res = orc.lca(qc, qr, C, K, g=1, w=w, lib=lib)
+            nG = orc.num_groups(41, 1, w, lib)
+            for b in range(2):
+                ref = torch_dense_seq(widen(qc[b]), widen(qr[b]), widen(C[b]), widen(K[b]))
+                assert rel_err(res.out[b], ref) < REL_TOL
+                # with g = 1 the anchor of group j is token j itself
+                assert np.array_equal(res.anchor[b], np.tile(np.arange(nG, dtype=np.int32), (3, 1)))
+
+
+def pin_window_dense(lib):
+    rng = np.random.default_rng(13)
+    qc, qr, C, K = rand_inputs(rng, 1, 2, 33, 16, 8)
+    for g in (2, 4, 7):
+        for w in (33, 34, 100):
+            res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+            ref = torch_dense_seq(widen(qc[0]), widen(qr[0]), widen(C[0]), widen(K[0]))
+            assert res.anchor.shape[-1] == 0
+            assert rel_err(res.out[0], ref) < REL_TOL
+
+
+def pin_zero_query(lib):
+    rng = np.random.default_rng(14)
+    _, _, C, K = rand_inputs(rng, 1, 2, 53, 16, 8)
+    qc = np.zeros((1, 2, 16), np.float32); qr = np.zeros((1, 2, 8), np.float32)
+    for g, w in ((4, 5), (5, 0), (8, 13), (3, 52), (1, 7)):
+        res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+        groups, window = partition(53, g, w)
+        Cd = widen(C[0])
+        # all scores are 0: uniform pooling, every entry weighs the same
+        total = sum(Cd[G].mean(axis=0) for G in groups) + Cd[window].sum(axis=0)
+        ref = total / (len(groups) + len(window))
+        for h in range(2):
+            assert rel_err(res.out[0, h], ref) < REL_TOL
+            assert list(res.anchor[0, h]) == [G[0] for G in groups]
+
+
+def pin_constant_groups(lib):
+    rng = np.random.default_rng(15)
+    L, g, w, d_c, d_r, H = 30, 4, 6, 16, 8, 3
+    groups, window = partition(L, g, w)
+    qc, qr, C, K = rand_inputs(rng, 1, H, L, d_c, d_r)
+    reps = []
+    for G in groups:                       # every token of a group is the same token
+        C[0, G] = C[0, G[0]]
+        K[0, G] = K[0, G[0]]
+        reps.append(G[0])
+    res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+    keep = reps + window                   # one representative per group, then the window
+    ref = torch_dense_seq(widen(qc[0]), widen(qr[0]), widen(C[0][keep]), widen(K[0][keep]))
+    assert rel_err(res.out[0], ref) < REL_TOL
+    for h in range(H):                     # exact ties inside every group: lowest index
+        assert list(res.anchor[0, h]) == reps
+
+
+def pin_brute_force(lib):
+    rng = np.random.default_rng(16)
+    for dtype in ("f32", "bf16"):
+        for L in (1, 2, 5, 9, 16):
+            qc, qr, C, K = rand_inputs(rng, 1, 2, L, 8, 4, dtype)
+            for g in range(1, L + 2):
+                for w in range(0, L + 2):
+                    res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+                    ref, anc = torch_lca_seq(widen(qc[0]), widen(qr[0]), widen(C[0]), widen(K[0]), g, w)
+                    assert rel_err(res.out[0], ref) < REL_TOL, (dtype, L, g, w)
+                    assert np.array_equal(res.anchor[0], anc), (dtype, L, g, w)
+
+
+def pin_ties(lib):
+    rng = np.random.default_rng(17)
+    L, g, w, d_c, d_r = 40, 8, 8, 16, 8
+    qc, qr, C, K = rand_inputs(rng, 1, 1, L, d_c, d_r)
+    u = np.concatenate([widen(qc[0, 0]), widen(qr[0, 0])])
+    u /= np.linalg.norm(u)
+    row = (6.0 * u).astype(np.float32)         # scores far above the N(0,1) background
+    planted = {0: (2, 5), 1: (8, 9), 2: (17, 23), 3: (24, 25, 31)}
+    for j, ts in planted.items():
+        for t in ts:
+            C[0, t] = row[:d_c]; K[0, t] = row[d_c:]
+    res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+    for j, ts in planted.items():
+        assert res.anchor[0, 0, j] == min(ts)
+        assert res.tie_gap[0, 0, j] == 0.0
+
+
+def pin_formulations(lib):
+    rng = np.random.default_rng(18)
+    for dtype in ("f32", "bf16"):
+        for (L, g, w) in ((64, 8, 8), (67, 4, 5), (50, 16, 0), (20, 32, 3)):
+            qc, qr, C, K = rand_inputs(rng, 2, 3, L, 32, 8, dtype)
+            a = orc.lca(qc, qr, C, K, g=g, w=w, formulation=0, lib=lib)
+            b = orc.lca(qc, qr, C, K, g=g, w=w, formulation=1, lib=lib)
+            assert rel_err(b.out, a.out) < 1e-12
+            assert np.array_equal(a.anchor, b.anchor)
+
+
+def pin_permutation(lib):
+    rng = np.random.default_rng(19)
+    L, g, w = 45, 5, 7
+    qc, qr, C, K = rand_inputs(rng, 1, 2, L, 16, 8)
+    groups, _ = partition(L, g, w)
+    base = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+    perm = np.arange(L)
+    for G in groups:
+        perm[G] = rng.permutation(G)
+    C2, K2 = C[:, perm].copy(), K[:, perm].copy()   # new position t holds old token perm[t]
+    res = orc.lca(qc, qr, C2, K2, g=g, w=w, lib=lib)
+    assert rel_err(res.out, base.out) < REL_TOL
+    inv = np.argsort(perm)                           # old token -> new position
+    assert np.array_equal(res.anchor, inv[base.anchor])
+
+
+def pin_constant_rope(lib):
+    rng = np.random.default_rng(20)
+    L, g, w = 48, 4, 6
+    qc, qr, C, K = rand_inputs(rng, 1, 3, L, 16, 8)
+    k0 = rng.standard_normal(8).astype(np.float32)
+    Kc = np.broadcast_to(k0, K.shape).copy()
+    Kz = np.zeros_like(K)
+    a = orc.lca(qc, qr, C, Kc, g=g, w=w, lib=lib)
+    b = orc.lca(qc, qr, C, Kz, g=g, w=w, lib=lib)
+    # a constant positional key shifts every score by the same amount per head
+    assert rel_err(a.out, b.out) < REL_TOL
+    assert np.array_equal(a.anchor, b.anchor)
+
+
+ALL_PINS = [pin_segmentation, pin_dense_vs_torch, pin_g1_dense, pin_window_dense, pin_zero_query,
+            pin_constant_groups, pin_brute_force, pin_ties, pin_formulations, pin_permutation,
+            pin_constant_rope]

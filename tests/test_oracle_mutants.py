@@ -1,0 +1,83 @@
+"""Plant plausible mistakes in a copy of the oracle and check that a pin fails.
+
+Each mutant is a textual edit of ``oracle/lca_oracle.c`` compiled to a
+temporary library on the CPU.  A mutant that every pin accepts would mean the
+pins leave that part of the oracle unchecked.
+"""
+import os
+
+import pytest
+
+import oracle_pins as pins
+from oracle import oracle as orc
+
+MUTANTS = {
+    # anchor tie-break: highest index instead of lowest
+    "tie_break_highest": ("if (w->s[t] > m) { m = w->s[t]; a = t; }",
+                          "if (w->s[t] >= m) { m = w->s[t]; a = t; }"),
+    # pooling weights from the semantic score only (drops the RoPE part)
+    "pool_on_semantic_score": ("return exp(w->s[t] - w->gmax[j]) / w->gden[j];",
+                               "return exp(w->sc[t] - w->gmax[j]) / w->gden[j];"),
+    # fixed weights (not query-aware; 1/8 is the mean for g = 8)
+    "mean_pooling": ("return exp(w->s[t] - w->gmax[j]) / w->gden[j];",
+                     "return 0.125;"),
+    # pooling weights not normalised inside the group
+    "unnormalised_pooling": ("return exp(w->s[t] - w->gmax[j]) / w->gden[j];",
+                             "return exp(w->s[t] - w->gmax[j]);"),
+    # sign error in the pooling exponent
+    "pool_exponent_sign": ("return exp(w->s[t] - w->gmax[j]) / w->gden[j];",
+                           "return exp(w->gmax[j] - w->s[t]) / w->gden[j];"),
+    # condensed logit without the anchor's positional key
+    "no_anchor_key": ("l += dot_row(w->qr, k_r, w->ganc[j], d_r, dtype); /* anchor's K_R */", ""),
+    # anchor key taken from the first token of the group
+    "anchor_is_first_token": ("l += dot_row(w->qr, k_r, w->ganc[j], d_r, dtype); /* anchor's K_R */",
+                              "l += dot_row(w->qr, k_r, j * g, d_r, dtype);"),
+    # a +log(g) bias on condensed logits (the page adds no parameter)
+    "log_g_bias": ("w->ell[j] = l;", "w->ell[j] = l + log((double)g);"),
+    # a trailing partial group instead of leftovers joining the window
+    "ceil_group_count": ("return (L - (int64_t)w) / g;", "return (L - (int64_t)w + g - 1) / g;"),
+    # pooled latent reads the wrong token rows (index slip)
+    "pool_wrong_row": ("cbar[i] += wt * elem(c_kv, t * (int64_t)d_c + i, dtype);",
+                       "cbar[i] += wt * elem(c_kv, (t - j * g) * (int64_t)d_c + i, dtype);"),
+    # window drops the current (last) token
+    "window_drops_current": ("for (int64_t t = win0; t < L; ++t) {\n            double p = exp(",
+                             "for (int64_t t = win0; t < L - 1; ++t) {\n            double p = exp("),
+    # positional score uses the semantic query (transposed operand)
+    "rope_score_wrong_query": ("w->sr[t] = dot_row(w->qr, k_r, t, d_r, dtype);",
+                               "w->sr[t] = dot_row(w->qc, k_r, t, d_r, dtype);"),
+}
+
+
+@pytest.fixture(scope="module")
+def oracle_src():
+    with open(orc.SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, oracle_src, tmp_path):
+    old, new = MUTANTS[name]
+    assert oracle_src.count(old) >= 1, f"mutant anchor text not found: {name}"
+    src = tmp_path / "mutant.c"
+    src.write_text(oracle_src.replace(old, new, 1))
+    lib_path = str(tmp_path / "libmutant.so")
+    orc.build(str(src), lib_path)
+    lib = orc.load(lib_path)
+    failures = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            failures.append(pin.__name__)
+    assert failures, f"mutant {name} passed every pin"
+
+
+def test_unmutated_copy_passes(oracle_src, tmp_path):
+    src = tmp_path / "copy.c"
+    src.write_text(oracle_src)
+    lib_path = str(tmp_path / "libcopy.so")
+    orc.build(str(src), lib_path)
+    lib = orc.load(lib_path)
+    for pin in pins.ALL_PINS:
+        pin(lib)
+    assert os.path.exists(lib_path)
