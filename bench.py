@@ -1,0 +1,359 @@
+"""Benchmark of the LCA decode step (one step = one lca_decode over one batch).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload v2lite] [--no-cpu-baseline] [--no-e2e]
+
+Default workload: the DeepSeek-V2-Lite-shaped decode (B=8, H=16, d_c=512,
+d_r=64, L=32768, g=16, w=1024, bf16 latents, queries N(0,1)/sqrt(576)), with
+synthetic seeded inputs.  Metric: context tokens per second (B*L per step),
+whole job over all ranks.  Under torchrun every rank runs its own batch on
+its own GPU (sequences are independent: no collective on the data path) and
+the time is the max over ranks ("weak" scaling).
+
+Prints one JSON line on rank 0.  `--impl reference` times the CPU oracle on
+the host cores instead (rank 0 only), on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "LCA decode context tokens/s per GPU; HBM GB/s as % of B200 peak"
+UNIT = "context tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["kv_compression_b200/csrc/tc_kernel.cuh", "kv_compression_b200/csrc/ptx.cuh"]
+TRAFFIC_FILE = "profiles/lca_tc_kernel_v2lite_traffic.txt"
+
+
+def workload_desc(wl: workloads.Workload) -> str:
+    return (f"{wl.name}: B={wl.B} H={wl.H} d_c={wl.d_c} d_r={wl.d_r} L={wl.L} g={wl.g} w={wl.w} "
+            f"{wl.dtype} latents, q*{wl.q_scale:.4g}")
+
+
+def algorithmic_bytes(wl: workloads.Workload) -> int:
+    """Cache read once + queries + fp32 output + int32 anchors."""
+    es = wl.elem_bytes
+    cache = wl.B * wl.L * (wl.d_c + wl.d_r) * es
+    q = wl.B * wl.H * (wl.d_c + wl.d_r) * es
+    out = wl.B * wl.H * wl.d_c * 4
+    anc = wl.B * wl.H * wl.n_groups * 4
+    return cache + q + out + anc
+
+
+def measured_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic() -> int | None:
+    """DRAM bytes per launch of the main kernel from the committed ncu summary,
+    or None when absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("source_sha256") != kernel_source_sha():
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of one GPU while the benchmark runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.path = tempfile.mktemp(prefix="lca_clocks_", suffix=".csv")
+        self.proc = None
+        cmd = ["nvidia-smi", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if gpu_uuid:
+            cmd += ["-i", gpu_uuid]
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    sm.append(float(parts[2])); smax.append(float(parts[3])); power.append(float(parts[4]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[6:10]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": sorted(reasons), "samples": 0}
+        idle = min(power)
+        loaded = [s for s, p in zip(sm, power) if p > idle + 50.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+
+
+def to_device(a, torch):
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def run_cpu_oracle_steps(wl, x, steps: int, budget_s: float, nthreads: int):
+    """Time the oracle on bounded samples: one sequence per step, heads cut to fit the budget.
+    Returns (context tokens per second, description, threads)."""
+    from oracle import oracle
+    t0 = time.perf_counter()
+    oracle.lca(x.q_c[:, :1], x.q_r[:, :1], x.c_kv, x.k_r, g=wl.g, w=wl.w, rows=[0], nthreads=nthreads)
+    per_head = time.perf_counter() - t0
+    heads = int(max(1, min(wl.H, budget_s / max(steps, 1) / max(per_head, 1e-6))))
+    tok, secs = 0.0, 0.0
+    for k in range(steps):
+        b = k % wl.B
+        t0 = time.perf_counter()
+        oracle.lca(x.q_c[:, :heads], x.q_r[:, :heads], x.c_kv, x.k_r, g=wl.g, w=wl.w, rows=[b],
+                   nthreads=nthreads)
+        secs += time.perf_counter() - t0
+        tok += wl.L * heads / wl.H     # context tokens, counted at all H heads per token
+    desc = (f"{steps} step(s) of one sequence x {heads}/{wl.H} heads of {wl.name} "
+            f"(L={wl.L}, g={wl.g}, w={wl.w}), oracle formulation A, {nthreads} threads")
+    return tok / secs, desc, secs
+
+
+def reference_arm(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workloads.WORKLOADS[args.workload]
+    x = workloads.generate(wl)
+    from oracle import oracle
+    oracle.build()
+    nthreads = os.cpu_count() or 1
+    budget = float(os.environ.get("LCA_REFERENCE_BUDGET_S", "120"))
+    if args.warmup > 0:
+        run_cpu_oracle_steps(wl, x, min(args.warmup, 1), budget / 10, nthreads)
+    value, desc, secs = run_cpu_oracle_steps(wl, x, args.steps, budget, nthreads)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, workloads/)",
+        "config": {"workload": workload_desc(wl), "parallelism": "host threads (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def our_arm(args) -> None:
+    import torch
+    import kv_compression_b200 as kvc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    wl = workloads.WORKLOADS[args.workload].with_(seed=rank)   # each rank its own batch
+    x = workloads.generate(wl)
+    cache_bytes = x.c_kv.nbytes + x.k_r.nbytes
+    copies = 1 if cache_bytes >= 4 * L2_BYTES else 2   # rotate copies so no step starts L2-warm
+    dev = [(to_device(x.q_c, torch), to_device(x.q_r, torch), to_device(x.c_kv, torch),
+            to_device(x.k_r, torch)) for _ in range(copies)]
+    plan = kvc.Plan(wl.B, wl.H, wl.d_c, wl.d_r, wl.dtype, wl.L)
+    kernel = plan.kernel(wl.L, wl.g, wl.w)
+    nG = wl.n_groups
+    out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32, device="cuda")
+    anc = torch.empty(wl.B, wl.H, max(nG, 1), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(k: int) -> None:
+        q_c, q_r, c_kv, k_r = dev[k % copies]
+        plan.decode(q_c, q_r, c_kv, k_r, wl.L, wl.g, wl.w, out, anc if nG > 0 else None, stream)
+
+    sampler = ClockSampler(getattr(torch.cuda.get_device_properties(local), "uuid", None)
+                           and "GPU-" + str(torch.cuda.get_device_properties(local).uuid))
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    assert plan.device_error() == kvc.LCA_OK
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for e in ev_m:          # create the events so their handles exist
+        e.record(stream)
+    torch.cuda.synchronize()
+    e_begin = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_begin.record(stream)
+    for k in range(K):
+        ev_s[k].record(stream)
+        plan.set_timing_event(ev_m[k])
+        step(k)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    plan.set_timing_event(None)
+    t_total = e_begin.elapsed_time(e_end) * 1e-3
+    t_main = statistics.mean(ev_s[k].elapsed_time(ev_m[k]) for k in range(K)) * 1e-3
+    assert plan.device_error() == kvc.LCA_OK
+    if dist is not None:
+        t = torch.tensor([t_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_total = float(t.item())
+    clocks = sampler.stop()
+
+    tokens_per_step = world * wl.B * wl.L
+    value = tokens_per_step * K / t_total
+    peaks, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(wl)
+    achieved = alg / t_main / 1e9
+    traffic = profiled_traffic()
+
+    e2e = None
+    if not args.no_e2e:
+        def pinned(a):
+            t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+            return t.pin_memory()
+        hq_c, hq_r, hc, hk = pinned(x.q_c), pinned(x.q_r), pinned(x.c_kv), pinned(x.k_r)
+        h_out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32).pin_memory()
+        h_anc = torch.empty(wl.B, wl.H, max(nG, 1), dtype=torch.int32).pin_memory()
+        ke = max(1, min(K, 30))
+        plan.decode_host(hq_c, hq_r, hc, hk, wl.L, wl.g, wl.w, h_out, h_anc if nG > 0 else None, stream)
+        if dist is not None:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(ke):
+            plan.decode_host(hq_c, hq_r, hc, hk, wl.L, wl.g, wl.w, h_out,
+                             h_anc if nG > 0 else None, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = e0.elapsed_time(e1) * 1e-3
+        if dist is not None:
+            t = torch.tensor([te], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            te = float(t.item())
+        h2d = hq_c.numel() * hq_c.element_size() + hq_r.numel() * hq_r.element_size() + \
+            hc.numel() * hc.element_size() + hk.numel() * hk.element_size()
+        d2h = h_out.numel() * 4 + (wl.B * wl.H * nG * 4)
+        e2e = {"value": tokens_per_step * ke / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": ke,
+               "path": "lca_decode_host (pinned host buffers; copies inside the timed region)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle
+        nthreads = os.cpu_count() or 1
+        res = oracle.lca(x.q_c, x.q_r, x.c_kv, x.k_r, g=wl.g, w=wl.w, nthreads=nthreads)
+        cpu = {"value": wl.B * wl.L / res.seconds, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+               "sample": f"the whole batch ({wl.B} sequences x {wl.H} heads, L={wl.L}) once, "
+                         f"oracle formulation A, {res.seconds:.1f} s"}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": t_total / K * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded, workloads/)",
+        "config": {"workload": workload_desc(wl), "kernel": kernel, "parallelism": f"replicas x{world}",
+                   "l2": (f"inputs {cache_bytes / 1e6:.0f} MB per step > 126 MB L2; "
+                          f"{copies} copies rotated, no flush"),
+                   "hbm_gbs_whole_step": alg / (t_total / K) / 1e9,
+                   "hbm_frac_whole_step": alg / (t_total / K) / 1e9 / peaks["hbm_gbs"]},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": "lca_tc_kernel" if kernel == "tcgen05" else "lca_simt_kernel",
+                     "algorithmic_bytes_per_launch": alg, "launch_ms": t_main * 1e3,
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v2lite", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        our_arm(args)
+
+
+if __name__ == "__main__":
+    main()

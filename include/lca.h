@@ -1,0 +1,158 @@
+/*
+ * lca.h -- C ABI of liblca.so: the Latent-Condensed Attention (LCA) decode
+ * step and the dense multi-head latent attention (MLA) decode it condenses,
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one described in "Latent-Condensed Transformer for
+ * Efficient Long Context Modeling" (gist.science summary of arXiv
+ * 2604.12452), section 2 "Metodologia: Atencao Condensada Latente (LCA)",
+ * "O Algoritmo LCA", steps 1-3.  For one query token per sequence b and
+ * every head h, with scores s_t = q_c.c_t + q_r.k_t over the cached latents
+ * c_t (C_KV) and RoPE keys k_t (K_R), t in [0, L):
+ *
+ *   step 1  n_G = floor((L - w) / g) groups G_j = [j g, (j+1) g) from token 0
+ *           (0 when L <= w); the window W = [n_G g, L) -- the last w tokens
+ *           plus the (L - w) mod g leftovers -- stays uncompressed;
+ *   step 2  per group: pooling weights w_t = softmax_{t in G_j}(s_t) and the
+ *           anchor a_j = the lowest index t in G_j with the largest s_t;
+ *           the condensed entry is (c_bar_j = sum_t w_t c_t, k_{a_j});
+ *   step 3  out = softmax attention of the query over [condensed || window]
+ *           with value = latent:  logits S_j = q_c.c_bar_j + q_r.k_{a_j} and
+ *           s_t (t in W); out = sum_e softmax(logit)_e value_e.
+ *
+ * No parameter is added (section 2, "Vantagens Teoricas"): there is no bias
+ * and no internal scale; fold the softmax scale into q_c and q_r.  The
+ * condensation is per head.  Dense MLA decode (section 1, "O Problema") is
+ * out = sum_t softmax(s)_t c_t over all L tokens.
+ *
+ * All entry points are plain C: no exceptions cross them and none aborts.
+ * Device entry points are asynchronous on the given stream; argument errors
+ * are reported synchronously, before anything is launched or written.
+ */
+#ifndef LCA_H_
+#define LCA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LCA_OK = 0,
+    LCA_ERR_INVALID_ARG = 1,     /* null pointer, g < 1, w < 0, L < 1, L > max_L, bad option */
+    LCA_ERR_UNSUPPORTED = 2,     /* shape / dtype / group size with no kernel */
+    LCA_ERR_ALIGNMENT = 3,       /* a device pointer not 16-byte aligned */
+    LCA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+    LCA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait inside a kernel ran out (see lca_get_device_error) */
+    LCA_ERR_PLAN_MISMATCH = 6,   /* the plan was made for another shape / dtype / device */
+    LCA_ERR_NO_MEMORY = 7        /* device or host allocation failed */
+} lca_status;
+
+typedef enum { LCA_F32 = 0, LCA_BF16 = 1 } lca_dtype;
+
+/* Opaque plan: shapes, kernel choice, split schedule and device workspace. */
+typedef struct lca_plan lca_plan;
+
+/*
+ * Make a plan for batch B, H heads, latent width d_c, RoPE width d_r, element
+ * type dt, and contexts up to max_L tokens, on the current CUDA device.
+ * Allocates the plan's device workspace (split partials and the device
+ * error word) once; no later call allocates device memory, except the first
+ * lca_decode_host call (its staging buffers).
+ * Kernels: bf16 with (d_c, d_r) = (512, 64) and H a multiple of 16 runs the
+ * tcgen05/TMA kernel; every other shape with d_c <= 1024, d_r <= 256 and
+ * H <= 4096 runs the CUDA-core kernel (fp32 accumulation).
+ * Errors: LCA_ERR_INVALID_ARG (null out_plan, non-positive sizes),
+ * LCA_ERR_UNSUPPORTED, LCA_ERR_NO_MEMORY, LCA_ERR_CUDA.  *out_plan is
+ * written only on LCA_OK; the caller frees it with lca_plan_destroy.
+ */
+lca_status lca_plan_create(int B, int H, int d_c, int d_r, lca_dtype dt, int64_t max_L,
+                           lca_plan **out_plan);
+
+/* Free a plan and its workspace.  NULL is accepted.  Call it only after every
+ * launch that used the plan has finished. */
+lca_status lca_plan_destroy(lca_plan *plan);
+
+/* Plan options (lca_plan_set); values are int64. */
+typedef enum {
+    LCA_OPT_FORCE_SIMT = 1,        /* 1: use the CUDA-core kernel even where tcgen05 applies */
+    LCA_OPT_NUM_CTAS = 2,          /* >0: CTAs of the tcgen05 kernel (default: SM count); 0: default */
+    LCA_OPT_WAIT_TIMEOUT_NS = 3,   /* bound of every in-kernel wait (default 2e9 ns) */
+    LCA_OPT_DEBUG_SKIP_LOAD = 4    /* 1: the tcgen05 producer skips its first load, so the
+                                      consumer's bounded wait runs out (tests the timeout path) */
+} lca_option;
+
+lca_status lca_plan_set(lca_plan *plan, lca_option opt, int64_t value);
+
+/*
+ * LCA decode (steps 1-3 above) for all B sequences at context length L.
+ *   q_c        [B][H][d_c]  device, plan dtype, row-major, 16-byte aligned
+ *   q_r        [B][H][d_r]  device, plan dtype
+ *   c_kv       [B][L][d_c]  device, plan dtype (the cache holds exactly L rows
+ *                           per sequence: sequence b starts at b*L*d_c)
+ *   k_r        [B][L][d_r]  device, plan dtype
+ *   L          context length, 1 <= L <= max_L, the same for every sequence;
+ *              the current token is the last cached row
+ *   g, w       group size (>= 1) and window (>= 0); the tcgen05 kernel takes
+ *              g in {1, 2, 4, ..., 128}, the CUDA-core kernel g <= 1024
+ *   out        [B][H][d_c]  device float32, written
+ *   anchor_idx [B][H][n_G]  device int32, absolute token positions in [0, L);
+ *              may be NULL only when n_G == lca_num_groups(L, g, w) == 0
+ *   stream     a cudaStream_t (NULL = legacy default stream)
+ * The caller owns every buffer; nothing is retained after the call.  One
+ * plan must not be used by two streams at once (the workspace is shared).
+ */
+lca_status lca_decode(lca_plan *plan, const void *q_c, const void *q_r, const void *c_kv,
+                      const void *k_r, int64_t L, int g, int w, float *out, int32_t *anchor_idx,
+                      void *stream);
+
+/*
+ * Dense MLA decode: out[b][h] = sum_t softmax_t(q_c.c_t + q_r.k_t) c_t over all
+ * L tokens (section 1 of the page: the cost LCA condenses).  Same layouts,
+ * ownership and errors as lca_decode; no anchors.
+ */
+lca_status mla_decode(lca_plan *plan, const void *q_c, const void *q_r, const void *c_kv,
+                      const void *k_r, int64_t L, float *out, void *stream);
+
+/*
+ * lca_decode with HOST buffers (same shapes): copies the inputs host->device
+ * into plan-owned staging (allocated on the first call), runs lca_decode on
+ * `stream`, copies out/anchor_idx back and synchronises the stream before
+ * returning.  Pinned host memory gives full copy bandwidth.
+ */
+lca_status lca_decode_host(lca_plan *plan, const void *h_q_c, const void *h_q_r,
+                           const void *h_c_kv, const void *h_k_r, int64_t L, int g, int w,
+                           float *h_out, int32_t *h_anchor_idx, void *stream);
+
+/* n_G for (L, g, w): floor((L - w) / g) when L > w, else 0; -1 if g < 1, w < 0 or L < 1. */
+int64_t lca_num_groups(int64_t L, int g, int w);
+
+/* Static text for a status code (never NULL). */
+const char *lca_status_string(lca_status status);
+
+/*
+ * Synchronise `stream`, read and clear the plan's device error word.
+ * Returns LCA_OK, LCA_ERR_DEVICE_TIMEOUT when an in-kernel wait ran out (the
+ * kernel then skipped its remaining work and left outputs undefined), or
+ * LCA_ERR_CUDA when the synchronisation itself failed.
+ */
+lca_status lca_get_device_error(lca_plan *plan, void *stream);
+
+/*
+ * Instrumentation for measuring the main kernel on its own: when `event` (a
+ * cudaEvent_t) is non-NULL, each later lca_decode / mla_decode call records it
+ * on the call's stream right after launching the main kernel and before
+ * launching the split-combine kernel.  NULL turns it off.  The caller owns the
+ * event.  Returns LCA_ERR_INVALID_ARG for a NULL plan.
+ */
+lca_status lca_plan_set_timing_event(lca_plan *plan, void *event);
+
+/* Which kernel a plan runs for (L, g, w): 0 = none (invalid), 1 = CUDA-core, 2 = tcgen05. */
+int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCA_H_ */

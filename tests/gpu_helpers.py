@@ -1,0 +1,93 @@
+"""Shared helpers of the GPU tests: upload seeded inputs, run the library,
+run the oracle on the same inputs, compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import kv_compression_b200 as kvc
+import workloads
+from oracle import oracle as orc
+
+BF16_TOL = 2e-2      # bf16 latents, fp32 accumulation
+F32_TOL = 1e-5       # fp32 latents
+ANCHOR_GAP = 1e-3    # bf16 anchors are gated where the oracle's top-2 gap > 1e-3 * max|s|
+
+
+def to_device(a: np.ndarray) -> torch.Tensor:
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+class DeviceInputs:
+    def __init__(self, x: workloads.Inputs):
+        self.x = x
+        self.q_c, self.q_r = to_device(x.q_c), to_device(x.q_r)
+        self.c_kv, self.k_r = to_device(x.c_kv), to_device(x.k_r)
+
+
+def make_plan(wl: workloads.Workload, opts: dict | None = None) -> kvc.Plan:
+    plan = kvc.Plan(wl.B, wl.H, wl.d_c, wl.d_r, wl.dtype, wl.L)
+    for k, v in (opts or {}).items():
+        plan.set(k, v)
+    return plan
+
+
+def run_lca(plan: kvc.Plan, d: DeviceInputs, g: int, w: int):
+    wl = d.x.wl
+    nG = kvc.num_groups(wl.L, g, w)
+    out = torch.full((wl.B, wl.H, wl.d_c), float("nan"), dtype=torch.float32, device="cuda")
+    anc = torch.full((wl.B, wl.H, max(nG, 1)), -7, dtype=torch.int32, device="cuda")
+    plan.decode(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, g, w, out, anc if nG > 0 else None)
+    torch.cuda.synchronize()
+    assert plan.device_error() == kvc.LCA_OK
+    return out.cpu().numpy().astype(np.float64), anc.cpu().numpy()[:, :, :nG]
+
+
+def run_dense(plan: kvc.Plan, d: DeviceInputs):
+    wl = d.x.wl
+    out = torch.full((wl.B, wl.H, wl.d_c), float("nan"), dtype=torch.float32, device="cuda")
+    plan.dense(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64)
+
+
+def oracle_lca(x: workloads.Inputs, g: int, w: int, rows=None, heads=None):
+    qc, qr = x.q_c, x.q_r
+    if heads is not None:
+        qc, qr = qc[:, heads], qr[:, heads]
+    return orc.lca(qc, qr, x.c_kv, x.k_r, g=g, w=w, rows=rows)
+
+
+def oracle_dense(x: workloads.Inputs, rows=None, heads=None):
+    qc, qr = x.q_c, x.q_r
+    if heads is not None:
+        qc, qr = qc[:, heads], qr[:, heads]
+    return orc.mla(qc, qr, x.c_kv, x.k_r, rows=rows)
+
+
+def rel_err(got: np.ndarray, ref: np.ndarray) -> float:
+    """max over (b, h) of ||got - ref||_inf / ||ref||_inf."""
+    g = got.reshape(-1, got.shape[-1]); r = ref.reshape(-1, ref.shape[-1])
+    return float((np.abs(g - r).max(1) / np.maximum(np.abs(r).max(1), 1e-30)).max())
+
+
+def compare(got_out, got_anc, ref, tol: float, exact_anchors: bool):
+    """Check outputs and anchors; returns (rel_err, gated anchor agreement, gated count)."""
+    assert np.all(np.isfinite(got_out))
+    err = rel_err(got_out, ref.out)
+    assert err <= tol, f"max relative error {err:.3e} > {tol:.1e}"
+    if ref.anchor.size == 0:
+        return err, 1.0, 0
+    assert got_anc.shape == ref.anchor.shape
+    assert np.all((got_anc >= 0)), "anchor not written"
+    if exact_anchors:
+        thr = 1e-6 * ref.max_abs_s[..., None]
+        assert np.all(ref.tie_gap > thr), "near-tie in an exact-anchor case"
+        assert np.array_equal(got_anc, ref.anchor)
+        return err, 1.0, ref.anchor.size
+    gate = ref.tie_gap > ANCHOR_GAP * ref.max_abs_s[..., None]
+    agree = got_anc[gate] == ref.anchor[gate]
+    assert agree.all(), f"{(~agree).sum()} gated anchors differ"
+    return err, float(agree.mean()) if agree.size else 1.0, int(gate.sum())
