@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblca.so")
 
 LCA_OK = 0
+LCA_ERR_DEVICE_TIMEOUT = 5
 STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED", 3: "LCA_ERR_ALIGNMENT",
           4: "LCA_ERR_CUDA", 5: "LCA_ERR_DEVICE_TIMEOUT", 6: "LCA_ERR_PLAN_MISMATCH",
           7: "LCA_ERR_NO_MEMORY"}

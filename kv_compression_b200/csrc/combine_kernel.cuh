@@ -10,6 +10,7 @@
 namespace lca {
 
 constexpr int kCombineThreads = 128;
+constexpr int kCombineMaxParts = 1024;   // per (sequence, head); the plan keeps far fewer
 
 struct CombineParams {
   const float* part_o;   // [slots][H][d_c]
@@ -33,8 +34,10 @@ __device__ __forceinline__ int64_t range_owner(int64_t u, int64_t U, int64_t G) 
 }
 
 __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const CombineParams p) {
+  __shared__ float scale[kCombineMaxParts];
+  __shared__ float red[kCombineThreads / 32];
   if (p.wait_prior) ptx::griddep_wait();
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   int64_t first, count;
   if (p.mode == 0) {
     first = (int64_t)b * p.n_split;
@@ -46,21 +49,45 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     first = b + c0;
     count = c1 - c0 + 1;
   }
-  float M = -INFINITY;
-  for (int64_t i = 0; i < count; ++i) M = fmaxf(M, p.part_mz[((first + i) * p.H + h) * 2]);
-  float Z = 0.f;
-  for (int64_t i = 0; i < count; ++i) {
+  if (count > kCombineMaxParts) count = kCombineMaxParts;  // the host never plans more
+  // M = max_i M_i
+  float m = -INFINITY;
+  for (int64_t i = tid; i < count; i += kCombineThreads)
+    m = fmaxf(m, p.part_mz[((first + i) * p.H + h) * 2]);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((tid & 31) == 0) red[tid >> 5] = m;
+  __syncthreads();
+  float M = red[0];
+  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+  // per-partial factors e^{M_i - M} and Z
+  float z = 0.f;
+  for (int64_t i = tid; i < count; i += kCombineThreads) {
     const float* mz = p.part_mz + ((first + i) * p.H + h) * 2;
-    Z += expf(mz[0] - M) * mz[1];
+    const float f = expf(mz[0] - M);
+    scale[i] = f;
+    z = fmaf(f, mz[1], z);
   }
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if ((tid & 31) == 0) red[tid >> 5] = z;
+  __syncthreads();
+  float Z = 0.f;
+  for (int w = 0; w < kCombineThreads / 32; ++w) Z += red[w];
   const float invZ = 1.f / Z;
-  for (int d = threadIdx.x; d < p.d_c; d += kCombineThreads) {
-    float acc = 0.f;
-    for (int64_t i = 0; i < count; ++i) {
-      const float sc = expf(p.part_mz[((first + i) * p.H + h) * 2] - M);
-      acc = fmaf(sc, p.part_o[((first + i) * p.H + h) * p.d_c + d], acc);
+  // out[d] = sum_i f_i O_i[d] / Z; four independent accumulators per thread
+  const float* po = p.part_o + (first * p.H + h) * (int64_t)p.d_c;
+  const int64_t stride = (int64_t)p.H * p.d_c;
+  for (int d = tid; d < p.d_c; d += kCombineThreads) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int64_t i = 0;
+    for (; i + 4 <= count; i += 4) {
+      a0 = fmaf(scale[i], po[i * stride + d], a0);
+      a1 = fmaf(scale[i + 1], po[(i + 1) * stride + d], a1);
+      a2 = fmaf(scale[i + 2], po[(i + 2) * stride + d], a2);
+      a3 = fmaf(scale[i + 3], po[(i + 3) * stride + d], a3);
     }
-    p.out[((int64_t)b * p.H + h) * p.d_c + d] = acc * invZ;
+    for (; i < count; ++i) a0 = fmaf(scale[i], po[i * stride + d], a0);
+    p.out[((int64_t)b * p.H + h) * p.d_c + d] = ((a0 + a1) + (a2 + a3)) * invZ;
   }
 }
 

@@ -144,16 +144,38 @@ lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c
   return launch_combine(p, cp, stream, false);
 }
 
+template <int LOG2G>
+cudaError_t launch_tc(const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream, int device) {
+  static int configured_device = -1;
+  if (configured_device != device) {
+    cudaError_t e = cudaFuncSetAttribute(lca::tc::lca_tc_kernel<LOG2G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         lca::tc::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    configured_device = device;
+  }
+  lca::tc::lca_tc_kernel<LOG2G><<<grid, lca::tc::kThreads, lca::tc::kSmemAlloc, stream>>>(tp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_g(int g, const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream,
+                        int device) {
+  switch (g) {
+    case 1: return launch_tc<0>(tp, grid, stream, device);
+    case 2: return launch_tc<1>(tp, grid, stream, device);
+    case 4: return launch_tc<2>(tp, grid, stream, device);
+    case 8: return launch_tc<3>(tp, grid, stream, device);
+    case 16: return launch_tc<4>(tp, grid, stream, device);
+    case 32: return launch_tc<5>(tp, grid, stream, device);
+    case 64: return launch_tc<6>(tp, grid, stream, device);
+    case 128: return launch_tc<7>(tp, grid, stream, device);
+  }
+  return cudaErrorInvalidValue;
+}
+
 lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                   const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
                   cudaStream_t stream) {
-  static int smem_set_device = -1;
-  if (smem_set_device != p->device) {
-    if (cudaFuncSetAttribute(lca::tc::lca_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             lca::tc::kSmemAlloc) != cudaSuccess)
-      return LCA_ERR_CUDA;
-    smem_set_device = p->device;
-  }
   lca::tc::TcParams tp;
   std::memset(&tp, 0, sizeof(tp));
   const uint64_t rows = (uint64_t)p->B * (uint64_t)L;
@@ -167,13 +189,12 @@ lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_k
   const int ctas = p->num_ctas > 0 ? p->num_ctas : p->num_sms;
   const int64_t G = std::max<int64_t>(1, std::min<int64_t>(ctas / n_hb, U));
   if ((int64_t)p->B + G - 1 > p->ws_slots) return LCA_ERR_UNSUPPORTED;
-  tp.B = p->B; tp.H = p->H; tp.L = L; tp.g = nG > 0 ? g : 1; tp.nG = nG;
+  tp.B = p->B; tp.H = p->H; tp.L = L; tp.nG = nG;
   tp.tiles_per_seq = tps; tp.U = U; tp.G = G; tp.n_hb = n_hb;
   tp.anchor = anchor; tp.part_o = p->part_o; tp.part_mz = p->part_mz; tp.err = p->err;
   tp.timeout_ns = p->timeout_ns; tp.debug_skip_load = p->debug_skip_load;
   const unsigned grid = (unsigned)(G * n_hb);
-  lca::tc::lca_tc_kernel<<<grid, lca::tc::kThreads, lca::tc::kSmemAlloc, stream>>>(tp);
-  if (cudaGetLastError() != cudaSuccess) return LCA_ERR_CUDA;
+  if (launch_tc_g(nG > 0 ? g : 1, tp, grid, stream, p->device) != cudaSuccess) return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
   lca::CombineParams cp = {};
   cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;

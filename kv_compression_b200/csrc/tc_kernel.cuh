@@ -5,17 +5,20 @@
 // Context Modeling", section 2, "O Algoritmo LCA", steps 1-3) for 16 heads of
 // one sequence over a contiguous range of 128-token tiles:
 //   scores     S^T[128 tokens x 16 heads] = [C_KV | K_R]_tile . [q_c | q_r]^T,
-//              kept as two TMEM accumulators, sc (K = 512) and sr (K = 64),
-//              because the condensed logit needs the semantic part alone;
-//   condense   each thread owns one token row (the TMEM lane): group max and
-//              lowest-index argmax (the anchor), group-local softmax weights
-//              w_t and the condensed logit S_j = sum_t w_t sc_t + sr_{a_j}
-//              (= q_c.c_bar_j + q_r.k_{a_j}; c_bar_j is never formed), by warp
-//              shuffles for g <= 32 and a shared-memory exchange for g = 64, 128;
-//   attend     online softmax over [condensed || window]: P_t = e^{S_j - M} w_t
-//              for a grouped token, e^{s_t - M} for a window token, written as
-//              bf16 to shared memory; O^T[512 x 16] += C_KV_tile^T . P^T is one
-//              more MMA per tile (group weight x in-group weight folded into P).
+//              two TMEM accumulators, sc (K = 512) and sr (K = 64), because the
+//              condensed logit needs the semantic part on its own;
+//   condense   (step 2) one thread per (group, head) runs over the g tokens of
+//              its group: max and lowest-index argmax (the anchor a_j), the
+//              group-local softmax sums den_j = sum e^{s_t - m_j} and
+//              num_j = sum e^{s_t - m_j} sc_t, and the condensed logit
+//              S_j = num_j / den_j + sr_{a_j}  (= q_c.c_bar_j + q_r.k_{a_j};
+//              c_bar_j is never formed);
+//   attend     (step 3) online softmax over [condensed || window].  A grouped
+//              token's weight p_j w_t = e^{S_j - M} e^{s_t - m_j} / den_j is
+//              written e^{s_t + k_j - M} with k_j = S_j - m_j - ln den_j, a window
+//              token's e^{s_t - M}: one exponential per (token, head).  The
+//              weights go to shared memory as bf16 and O^T[512 x 16] +=
+//              C_KV_tile^T . P^T is one more MMA per tile.
 // The range's partial (M, Z, O) goes to the workspace; the combine kernel
 // merges the ranges of a sequence.
 //
@@ -23,7 +26,8 @@
 // and its lane 0 issues MMAs; warps 2-5 (128 threads, one per TMEM lane) do
 // the softmax work.  Shared memory: a ring of five 32 KB slots for C_KV
 // column pairs ([128 tokens][2 x 64 dims], 128-byte swizzle), two 16 KB K_R
-// slots, the query block (9 x [16 heads][64 dims]) and two P buffers.
+// slots (each reused to stage its tile's scores once the score MMA is done),
+// the query block (9 x [16 heads][64 dims]) and two P buffers.
 // Every mbarrier wait is bounded; when a bound runs out the CTA records the
 // error, stops issuing work, waits for its own copies and MMAs in flight,
 // frees TMEM and exits.
@@ -51,16 +55,19 @@ constexpr int kPBytes = kT * kHC * 2;      // P^T tile, bf16
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
 constexpr int kSoftmaxBar = 1;             // named barrier of the 4 softmax warps
+constexpr int kMaxGroupsPerTile = 64;      // g >= 2 (g = 1 takes the per-token path)
+constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffPair = 0;
 constexpr int kOffKr = kOffPair + kNPair * kPairBytes;
 constexpr int kOffQ = kOffKr + kNKr * kChunk;
 constexpr int kOffP = kOffQ + kQBytes;
-constexpr int kOffRed = kOffP + 2 * kPBytes;           // float [2][4][16] tile maxima
-constexpr int kOffZred = kOffRed + 2 * 4 * kHC * 4;     // float [4][16]
-constexpr int kOffGrp = kOffZred + 4 * kHC * 4;         // float [2][4][16][5] group partials
-constexpr int kOffBar = kOffGrp + 2 * 4 * kHC * 5 * 4;
+constexpr int kOffK = kOffP + 2 * kPBytes;                  // float [64 groups][16 heads]: k_j
+constexpr int kOffGmax = kOffK + kMaxGroupsPerTile * kHC * 4;  // float [16]: max_j S_j of the tile
+constexpr int kOffWmax = kOffGmax + kHC * 4;                // float [4][16]: max window score
+constexpr int kOffZred = kOffWmax + 4 * kHC * 4;            // float [4][16]
+constexpr int kOffBar = kOffZred + 4 * kHC * 4;
 constexpr int kNumBars = 2 * kNPair + 2 * kNKr + 2 + 5 * 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
@@ -81,8 +88,7 @@ struct TcParams {
   CUtensorMap tm_qr;   // q_r   as [B*H rows][64],  box [16 rows][64],  128B swizzle
   int B, H;
   int64_t L;
-  int g;               // power of two <= 128 (1 when n_G == 0)
-  int64_t nG;
+  int64_t nG;          // condensed groups (0: dense attention)
   int64_t tiles_per_seq;
   int64_t U;           // B * tiles_per_seq
   int64_t G;           // number of tile ranges (CTA groups); G <= U
@@ -99,7 +105,7 @@ struct Bars {
   uint64_t* full_c;   // [kNPair]
   uint64_t* empty_c;  // [kNPair]
   uint64_t* full_k;   // [kNKr]
-  uint64_t* empty_k;  // [kNKr]
+  uint64_t* empty_k;  // [kNKr]  released by the softmax warps (they stage scores there)
   uint64_t* q_full;
   uint64_t* q_empty;
   uint64_t* s_full;   // [2]
@@ -140,6 +146,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Score staging in a K_R slot: [128 rows][32 floats] (sc of 16 heads, then sr),
+// float4 columns XOR-swizzled by (row ^ group-of-row) so that the group phase
+// (threads on different groups, same step) reads distinct banks.
+template <int LOG2G>
+__device__ __forceinline__ int stage_idx(int row, int col) {
+  const int sw = ((row ^ (row >> LOG2G)) & 7) << 2;
+  return row * 32 + (col ^ sw);
+}
+
 // Fold the O^T tile in TMEM buffer `ob` (its use `okb`) into the register
 // accumulator: O = O * al + O_tile.  Thread = latent row of each 128-row block.
 __device__ __forceinline__ void fold_o(float (&O)[4][kHC], const float (&al)[kHC], int ob, int okb,
@@ -160,7 +181,10 @@ __device__ __forceinline__ void fold_o(float (&O)[4][kHC], const float (&al)[kHC
   if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&bb.o_empty[ob]);
 }
 
+template <int LOG2G>
 __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr int g = 1 << LOG2G;
+  static_assert(g <= kT, "a group must fit in one tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -188,11 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   const int h0 = hb * kHC;
   const int64_t u0 = c * p.U / p.G;
   const int64_t u1 = (c + 1) * p.U / p.G;
-  const int64_t win0 = p.nG * p.g;
+  const int64_t win0 = p.nG * g;
 
   if (tid == 0) {
     for (int i = 0; i < kNPair; ++i) { ptx::mbar_init(&bb.full_c[i], 1); ptx::mbar_init(&bb.empty_c[i], 1); }
-    for (int i = 0; i < kNKr; ++i) { ptx::mbar_init(&bb.full_k[i], 1); ptx::mbar_init(&bb.empty_k[i], 1); }
+    for (int i = 0; i < kNKr; ++i) { ptx::mbar_init(&bb.full_k[i], 1); ptx::mbar_init(&bb.empty_k[i], 4); }
     ptx::mbar_init(bb.q_full, 1);
     ptx::mbar_init(bb.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
@@ -314,7 +338,6 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
           const uint64_t bq = ptx::smem_desc(s_q + 8 * kQChunk + 32 * k, 16, 1024, ptx::kSwizzle128B);
           ptx::mma_bf16_ss(d_sr, a, bq, kIdescS, k > 0);
         }
-        ptx::mma_commit(&bb.empty_k[ks]);
         ++nk;
       }
       // ---- sc = C_KV tile . q_c^T, one column pair (128 dims) per ring slot
@@ -339,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         ++nc;
       }
       if (!ok) break;
-      ptx::mma_commit(&bb.s_full[buf]);
+      ptx::mma_commit(&bb.s_full[buf]);   // also tells the softmax warps the K_R slot is read
       if (last_in_seg) ptx::mma_commit(bb.q_empty);
       // ---- O^T tile = C_KV tile^T . P^T, four 128-dim blocks
       ok = bounded_wait(&bb.p_full[buf], kb & 1, abort_flag, p, 0x204, true);
@@ -372,13 +395,19 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     // is ever left waiting at a named barrier.
     const int q4 = warp & 3;             // TMEM lane quarter this warp may access
     const int row = q4 * 32 + lane;      // token row of the tile owned by this thread
+    const int st = tid - 64;             // 0..127 among the softmax threads
     const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
-    float* red = reinterpret_cast<float*>(smem + kOffRed);     // [2][4][16]
-    float* zred = reinterpret_cast<float*>(smem + kOffZred);   // [4][16]
-    float* grp = reinterpret_cast<float*>(smem + kOffGrp);     // [2][4][16][5]
+    float* ks_tab = reinterpret_cast<float*>(smem + kOffK);      // [64][16] k_j
+    float* gmax_s = reinterpret_cast<float*>(smem + kOffGmax);   // [16]
+    float* wmax_s = reinterpret_cast<float*>(smem + kOffWmax);   // [4][16]
+    float* zred = reinterpret_cast<float*>(smem + kOffZred);     // [4][16]
     uint8_t* pbase = smem + kOffP;
-    const int g = p.g;
-    const int seg_g = g < 32 ? g : 32;   // lanes of one group inside this warp
+    // group phase: threads per head (consecutive), groups per thread
+    constexpr int kGt = kT / g;                          // groups per tile
+    constexpr int kTpH = kGt < 8 ? kGt : 8;
+    constexpr int kGpt = kGt / kTpH;
+    constexpr int kActive = kHC * kTpH;
+    constexpr int kUnroll = g < 16 ? g : 16;             // full unroll would spill for g >= 64
 
     float O[4][kHC];
     float Zt[kHC], Mh[kHC], apend[kHC];
@@ -397,6 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       const bool last_in_seg = (u + 1 == u1) || ((u + 1) / p.tiles_per_seq != b);
       const int buf = (int)(i & 1);
       const int kb = (int)(i >> 1);
+      const int ks = (int)(i % kNKr);
+      float* stage = reinterpret_cast<float*>(smem + kOffKr + ks * kChunk);
       warp_wait(&bb.s_full[buf], kb & 1, abort_flag, p, 0x300);
       ptx::tc_fence_after();
       float sc[kHC], sr[kHC];
@@ -411,91 +442,114 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       const int64_t t = tok0 + row;
       const bool valid = t < p.L;
       const bool grouped = t < win0;
-
-      // ---- step 2: group max, lowest-index anchor, group-local softmax, condensed logit
-      float s[kHC], ent[kHC], wgt[kHC];
-      int anc[kHC];
+      // tile-uniform flags
+      const bool tile_groups = (g > 1) && (tok0 < win0);
+      const bool tile_tokens = (g == 1) || (tok0 + kT > win0);   // per-token entries present
+      float s[kHC];
 #pragma unroll
-      for (int h = 0; h < kHC; ++h) {
-        s[h] = sc[h] + sr[h];
-        float m = s[h];
-        int idx = row;
-        for (int off = 1; off < seg_g; off <<= 1) {
-          const float om = __shfl_xor_sync(0xffffffffu, m, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
-          if (om > m || (om == m && oi < idx)) { m = om; idx = oi; }
-        }
-        const float e = __expf(s[h] - m);
-        float den = e, num = e * sc[h];
-        for (int off = 1; off < seg_g; off <<= 1) {
-          den += __shfl_xor_sync(0xffffffffu, den, off);
-          num += __shfl_xor_sync(0xffffffffu, num, off);
-        }
-        const float sra = __shfl_sync(0xffffffffu, sr[h], idx & 31);  // K_R score of the anchor
-        if (g <= 32) {
-          ent[h] = num / den + sra;          // S_j = sum_t w_t sc_t + sr_{a_j}
-          wgt[h] = e / den;                  // w_t
-          anc[h] = idx;
-        } else if (lane == 0) {
-          float* gp = grp + ((buf * 4 + q4) * kHC + h) * 5;
-          gp[0] = m; gp[1] = __int_as_float(idx); gp[2] = den; gp[3] = num; gp[4] = sra;
+      for (int h = 0; h < kHC; ++h) s[h] = sc[h] + sr[h];
+
+      if (tile_groups) {
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 v = c4 < 4 ? make_float4(sc[4 * c4], sc[4 * c4 + 1], sc[4 * c4 + 2], sc[4 * c4 + 3])
+                                  : make_float4(sr[4 * c4 - 16], sr[4 * c4 - 15], sr[4 * c4 - 14],
+                                                sr[4 * c4 - 13]);
+          *reinterpret_cast<float4*>(stage + stage_idx<LOG2G>(row, 4 * c4)) = v;
         }
       }
-      if (g > 32) {
-        // a group spans g/32 warps: merge their (max, argmax, sums) parts
-        ptx::named_bar_sync(kSoftmaxBar, 128);
-        const int wpg = g / 32;
-        const int q_first = q4 & ~(wpg - 1);
+      ptx::named_bar_sync(kSoftmaxBar, 128);                     // B1: staged scores visible
+
+      if (tile_groups && st < kActive) {
+        // ---- step 2, one thread per (group, head)
+        const int h = st / kTpH;
+        const int j0 = st % kTpH;
+        float gm = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kGpt; ++r) {
+          const int j = j0 + kTpH * r;                 // group within the tile
+          const int64_t jg = tok0 / g + j;             // group within the sequence
+          if (jg < p.nG) {
+            const int r0 = j * g;
+            float m = -INFINITY;
+            int a = 0;
+#pragma unroll kUnroll
+            for (int v = 0; v < g; ++v) {
+              const float x = stage[stage_idx<LOG2G>(r0 + v, h)] + stage[stage_idx<LOG2G>(r0 + v, 16 + h)];
+              if (x > m) { m = x; a = v; }             // strict: the lowest index keeps a tie
+            }
+            float den = 0.f, num = 0.f;
+            const float mb = m * kLog2e;
+#pragma unroll kUnroll
+            for (int v = 0; v < g; ++v) {
+              const float scv = stage[stage_idx<LOG2G>(r0 + v, h)];
+              const float x = scv + stage[stage_idx<LOG2G>(r0 + v, 16 + h)];
+              const float e = ex2(fmaf(x, kLog2e, -mb));
+              den += e;
+              num = fmaf(e, scv, num);
+            }
+            const float sra = stage[stage_idx<LOG2G>(r0 + a, 16 + h)];   // K_R score of the anchor
+            const float S = __fdividef(num, den) + sra;                 // condensed logit
+            ks_tab[j * kHC + h] = S - m - __logf(den);                  // k_j
+            gm = fmaxf(gm, S);
+            p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + jg] = (int32_t)(tok0 + r0 + a);
+          }
+        }
+#pragma unroll
+        for (int off = 1; off < kTpH; off <<= 1)
+          gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, off));
+        if (j0 == 0) gmax_s[h] = gm;
+      }
+      if (tile_tokens) {
+        // window tokens (and g = 1, where every grouped token is its own entry)
+        const bool own = valid && (!grouped || g == 1);
+        if (g == 1 && grouped) {
+#pragma unroll
+          for (int h = 0; h < kHC; ++h)
+            p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + t] = (int32_t)t;
+        }
 #pragma unroll
         for (int h = 0; h < kHC; ++h) {
-          float M = -INFINITY, sra = 0.f;
-          int idx = 0x7fffffff;
-          for (int k = 0; k < wpg; ++k) {
-            const float* gp = grp + ((buf * 4 + q_first + k) * kHC + h) * 5;
-            const float mk = gp[0];
-            const int ik = __float_as_int(gp[1]);
-            if (mk > M || (mk == M && ik < idx)) { M = mk; idx = ik; sra = gp[4]; }
-          }
-          float den = 0.f, num = 0.f;
-          for (int k = 0; k < wpg; ++k) {
-            const float* gp = grp + ((buf * 4 + q_first + k) * kHC + h) * 5;
-            const float f = __expf(gp[0] - M);
-            den = fmaf(gp[2], f, den);
-            num = fmaf(gp[3], f, num);
-          }
-          ent[h] = num / den + sra;
-          wgt[h] = __expf(s[h] - M) / den;
-          anc[h] = idx;
+          float v = own ? s[h] : -INFINITY;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+          if (lane == 0) wmax_s[q4 * kHC + h] = v;
         }
       }
-      if (grouped && (row % g) == 0) {   // first row of a group writes the group's anchors
-        const int64_t j = t / g;
-#pragma unroll
-        for (int h = 0; h < kHC; ++h)
-          p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + j] = (int32_t)(tok0 + anc[h]);
-      }
-      // ---- step 3: entry logits -> tile max per head across the 4 warps
-      float* rb = red + buf * 4 * kHC;
-#pragma unroll
-      for (int h = 0; h < kHC; ++h) {
-        if (!grouped) ent[h] = valid ? s[h] : -INFINITY;  // a window token is its own entry
-        float v = ent[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-        if (lane == 0) rb[q4 * kHC + h] = v;
-      }
-      // checkpoint: the only place the softmax warps leave the loop early
-      if (ptx::named_bar_or(kSoftmaxBar, 128, *abort_flag != 0)) break;
+      // B2, checkpoint: the only place the softmax warps leave the loop early
+      const bool stop = ptx::named_bar_or(kSoftmaxBar, 128, *abort_flag != 0);
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bb.empty_k[ks]);   // staging in the K_R slot is done
+      if (stop) break;
 
-      float alpha[kHC], pv[kHC];
+      // ---- step 3: tile maximum over entries, per-token weights
+      float alpha[kHC], mb[kHC];
 #pragma unroll
       for (int h = 0; h < kHC; ++h) {
-        const float mt = fmaxf(fmaxf(rb[h], rb[kHC + h]), fmaxf(rb[2 * kHC + h], rb[3 * kHC + h]));
+        float mt = tile_groups ? gmax_s[h] : -INFINITY;
+        if (tile_tokens)
+          mt = fmaxf(mt, fmaxf(fmaxf(wmax_s[h], wmax_s[kHC + h]),
+                               fmaxf(wmax_s[2 * kHC + h], wmax_s[3 * kHC + h])));
         const float mn = fmaxf(Mh[h], mt);
-        alpha[h] = __expf(Mh[h] - mn);   // 0 on the first tile of a range
+        alpha[h] = ex2((Mh[h] - mn) * kLog2e);   // 0 on the first tile of a range
         Mh[h] = mn;
-        if (grouped) pv[h] = __expf(ent[h] - mn) * wgt[h];   // group weight x in-group weight
-        else pv[h] = valid ? __expf(ent[h] - mn) : 0.f;
+        mb[h] = mn * kLog2e;
+      }
+      float pv[kHC];
+      if (grouped && g > 1) {
+        const float* kr = ks_tab + (row / g) * kHC;
+#pragma unroll
+        for (int h4 = 0; h4 < 4; ++h4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kr + 4 * h4);
+          pv[4 * h4 + 0] = ex2(fmaf(s[4 * h4 + 0] + k4.x, kLog2e, -mb[4 * h4 + 0]));
+          pv[4 * h4 + 1] = ex2(fmaf(s[4 * h4 + 1] + k4.y, kLog2e, -mb[4 * h4 + 1]));
+          pv[4 * h4 + 2] = ex2(fmaf(s[4 * h4 + 2] + k4.z, kLog2e, -mb[4 * h4 + 2]));
+          pv[4 * h4 + 3] = ex2(fmaf(s[4 * h4 + 3] + k4.w, kLog2e, -mb[4 * h4 + 3]));
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < kHC; ++h) pv[h] = valid ? ex2(fmaf(s[h], kLog2e, -mb[h])) : 0.f;
       }
       // ---- P^T tile, bf16, MN-major core matrices: token row -> K, head -> N
       uint32_t pk[8];
