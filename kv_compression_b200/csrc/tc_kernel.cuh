@@ -7,27 +7,33 @@
 //   scores     S^T[128 tokens x 16 heads] = [C_KV | K_R]_tile . [q_c | q_r]^T,
 //              two TMEM accumulators, sc (K = 512) and sr (K = 64), because the
 //              condensed logit needs the semantic part on its own;
-//   condense   (step 2) one thread per (group, head) runs over the g tokens of
-//              its group: max and lowest-index argmax (the anchor a_j), the
-//              group-local softmax sums den_j = sum e^{s_t - m_j} and
-//              num_j = sum e^{s_t - m_j} sc_t, and the condensed logit
-//              S_j = num_j / den_j + sr_{a_j}  (= q_c.c_bar_j + q_r.k_{a_j};
-//              c_bar_j is never formed);
+//   condense   (step 2) per group and head: max and lowest-index argmax (the
+//              anchor a_j), the group-local softmax sums den_j = sum e^{s_t - m_j}
+//              and num_j = sum e^{s_t - m_j} sc_t, and the condensed logit
+//              S_j = num_j / den_j + sr_{a_j}  (= q_c.c_bar_j + q_r.k_{a_j}; c_bar_j
+//              is never formed).  Each thread scans an 8-token segment of one
+//              head; a group of g > 8 tokens merges its segments by shuffles;
 //   attend     (step 3) online softmax over [condensed || window].  A grouped
 //              token's weight p_j w_t = e^{S_j - M} e^{s_t - m_j} / den_j is
 //              written e^{s_t + k_j - M} with k_j = S_j - m_j - ln den_j, a window
 //              token's e^{s_t - M}: one exponential per (token, head).  The
 //              weights go to shared memory as bf16 and O^T[512 x 16] +=
-//              C_KV_tile^T . P^T is one more MMA per tile.
+//              C_KV_tile^T . P^T is one more MMA chain per tile.
 // The range's partial (M, Z, O) goes to the workspace; the combine kernel
 // merges the ranges of a sequence.
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 allocates TMEM
-// and its lane 0 issues MMAs; warps 2-5 (128 threads, one per TMEM lane) do
-// the softmax work.  Shared memory: a ring of five 32 KB slots for C_KV
-// column pairs ([128 tokens][2 x 64 dims], 128-byte swizzle), two 16 KB K_R
-// slots (each reused to stage its tile's scores once the score MMA is done),
-// the query block (9 x [16 heads][64 dims]) and two P buffers.
+// Roles (320 threads): warp 0 lane 0 issues TMA loads and L2 prefetches two
+// tiles ahead; warp 1 allocates TMEM and its lane 0 issues MMAs; warps 2-9
+// (256 threads) do the softmax work, two warps per TMEM lane quarter, each
+// owning 8 of the 16 heads.  C_KV is read twice per tile: once for the scores
+// (kept in L2 with an evict-last hint) and once more, from L2, for O = C^T P^T
+// after the softmax.  MMA order: scores(i), then O(i-1); each column pair
+// leaves shared memory as soon as its MMAs are done, so the softmax of tile i
+// overlaps the tensor work of tiles i-1 and i+1 and the loads keep streaming.
+// Shared memory: a ring of five 32 KB slots for C_KV column pairs ([128
+// tokens][2 x 64 dims], 128-byte swizzle), two 16 KB K_R slots (each reused to
+// stage its tile's scores once the score MMA is done), the query block
+// (9 x [16 heads][64 dims]) and two P buffers.
 // Every mbarrier wait is bounded; when a bound runs out the CTA records the
 // error, stops issuing work, waits for its own copies and MMAs in flight,
 // frees TMEM and exits.
@@ -52,11 +58,16 @@ constexpr int kNKr = 2;                    // K_R slots
 constexpr int kQChunk = kHC * 128;         // [16 heads][64 bf16] = 2 KB
 constexpr int kQBytes = 9 * kQChunk;       // 8 chunks of q_c, 1 of q_r
 constexpr int kPBytes = kT * kHC * 2;      // P^T tile, bf16
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kHH = kHC / 2;               // heads per softmax thread
 constexpr int kTmemCols = 256;
-constexpr int kSoftmaxBar = 1;             // named barrier of the 4 softmax warps
+constexpr int kSoftmaxBar = 1;             // named barrier of the softmax warps
 constexpr int kMaxGroupsPerTile = 64;      // g >= 2 (g = 1 takes the per-token path)
+constexpr int kPrefetchAhead = 2;          // tiles brought into L2 ahead of their loads
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffPair = 0;
@@ -152,33 +163,67 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Score staging in a K_R slot: [128 rows][32 floats] (sc of 16 heads, then sr),
-// float4 columns XOR-swizzled by (row ^ group-of-row) so that the group phase
-// (threads on different groups, same step) reads distinct banks.
-template <int LOG2G>
+// float4 columns XOR-swizzled by row so that threads reading the same step of
+// different segments hit different banks.
 __device__ __forceinline__ int stage_idx(int row, int col) {
-  const int sw = ((row ^ (row >> LOG2G)) & 7) << 2;
+  const int sw = ((row ^ (row >> 3)) & 7) << 2;
   return row * 32 + (col ^ sw);
 }
 
 // Fold the O^T tile in TMEM buffer `ob` (its use `okb`) into the register
-// accumulator: O = O * al + O_tile.  Thread = latent row of each 128-row block.
-__device__ __forceinline__ void fold_o(float (&O)[4][kHC], const float (&al)[kHC], int ob, int okb,
-                                       uint32_t t_lane, const Bars& bb, volatile int* abort_flag,
+// accumulator: O = O * al + O_tile, for this thread's latent rows and 8 heads.
+__device__ __forceinline__ void fold_o(float (&O)[4][kHH], const float (&al)[kHH], int ob, int okb,
+                                       uint32_t t_cols, const Bars& bb, volatile int* abort_flag,
                                        const TcParams& p) {
   warp_wait(&bb.o_full[ob], okb & 1, abort_flag, p, 0x303);
   ptx::tc_fence_after();
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    float ot[kHC];
-    ptx::tmem_ld16(t_lane + kColO + 64 * ob + 16 * m, ot);
+    float ot[kHH];
+    ptx::tmem_ld8(t_cols + kColO + 64 * ob + 16 * m, ot);
     ptx::tmem_wait_ld();
 #pragma unroll
-    for (int h = 0; h < kHC; ++h) O[m][h] = fmaf(O[m][h], al[h], ot[h]);
+    for (int h = 0; h < kHH; ++h) O[m][h] = fmaf(O[m][h], al[h], ot[h]);
   }
   ptx::tc_fence_before();
   __syncwarp();
   if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&bb.o_empty[ob]);
+}
+
+// Group statistics over v in [v0, v0 + n) of a thread's 8-token segment.
+struct GroupStat {
+  float m;    // max score
+  int a;      // tile row of the first maximum
+  float den;  // sum e^{s - m}
+  float num;  // sum e^{s - m} sc
+};
+
+template <int N>
+__device__ __forceinline__ GroupStat scan_group(const float (&x)[8], const float (&c)[8], int v0,
+                                                int row0) {
+  GroupStat r;
+  r.m = x[v0];
+  r.a = row0 + v0;
+#pragma unroll
+  for (int v = 1; v < N; ++v)
+    if (x[v0 + v] > r.m) { r.m = x[v0 + v]; r.a = row0 + v0 + v; }   // strict: lowest index keeps a tie
+  const float mb = r.m * kLog2e;
+  r.den = 0.f;
+  r.num = 0.f;
+#pragma unroll
+  for (int v = 0; v < N; ++v) {
+    const float e = ex2(fmaf(x[v0 + v], kLog2e, -mb));
+    r.den += e;
+    r.num = fmaf(e, c[v0 + v], r.num);
+  }
+  return r;
 }
 
 template <int LOG2G>
@@ -216,15 +261,18 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 
   if (tid == 0) {
     for (int i = 0; i < kNPair; ++i) { ptx::mbar_init(&bb.full_c[i], 1); ptx::mbar_init(&bb.empty_c[i], 1); }
-    for (int i = 0; i < kNKr; ++i) { ptx::mbar_init(&bb.full_k[i], 1); ptx::mbar_init(&bb.empty_k[i], 4); }
+    for (int i = 0; i < kNKr; ++i) {
+      ptx::mbar_init(&bb.full_k[i], 1);
+      ptx::mbar_init(&bb.empty_k[i], kSoftmaxWarps);
+    }
     ptx::mbar_init(bb.q_full, 1);
     ptx::mbar_init(bb.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bb.s_full[i], 1);
-      ptx::mbar_init(&bb.s_empty[i], 4);
-      ptx::mbar_init(&bb.p_full[i], 4);
+      ptx::mbar_init(&bb.s_empty[i], kSoftmaxWarps);
+      ptx::mbar_init(&bb.p_full[i], kSoftmaxWarps);
       ptx::mbar_init(&bb.o_full[i], 1);
-      ptx::mbar_init(&bb.o_empty[i], 4);
+      ptx::mbar_init(&bb.o_empty[i], kSoftmaxWarps);
     }
     ptx::mbar_init(bb.drain, 1);
     *abort_flag = 0;
@@ -241,20 +289,56 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ===================================================== TMA producer
+    // Load order = MMA consumption order: for tile i, K_R(i) and the four
+    // column pairs of C_KV(i) for the scores, then the four pairs of tile i-1
+    // again for O(i-1) (read back from L2), and after the last tile the pairs
+    // of that tile.  Each pair slot is freed as soon as its MMAs are done, so
+    // shared memory never has to hold a whole tile across the softmax.
     ptx::prefetch_tmap(&p.tm_c);
     ptx::prefetch_tmap(&p.tm_k);
     ptx::prefetch_tmap(&p.tm_qc);
     ptx::prefetch_tmap(&p.tm_qr);
+    const uint64_t keep = ptx::l2_policy_evict_last();    // first read: keep for the second
+    const uint64_t drop = ptx::l2_policy_evict_first();   // second read: last use
+    auto tile_row = [&](int64_t u) -> int32_t {
+      return (int32_t)((u / p.tiles_per_seq) * p.L + (u % p.tiles_per_seq) * kT);
+    };
+    auto prefetch_tile = [&](int64_t u) {
+      const int32_t row = tile_row(u);
+      ptx::tma_prefetch_l2_2d(&p.tm_k, 0, row);
+      for (int ch = 0; ch < 8; ++ch) ptx::tma_prefetch_l2_2d(&p.tm_c, 64 * ch, row);
+    };
+    for (int64_t u = u0 + 1; u < u0 + kPrefetchAhead && u < u1; ++u) prefetch_tile(u);
     int issued_c[kNPair], issued_k[kNKr];
+#pragma unroll
     for (int i = 0; i < kNPair; ++i) issued_c[i] = -1;
+#pragma unroll
     for (int i = 0; i < kNKr; ++i) issued_k[i] = -1;
     int issued_q = -1;
     int64_t nc = 0, nk = 0;
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
+    // the four pairs of the tile at `row` into the next ring slots
+    auto load_pairs = [&](int32_t row, uint64_t policy) -> bool {
+      for (int pr = 0; pr < 4; ++pr) {
+        const int cs = (int)(nc % kNPair);
+        const int ck = (int)(nc / kNPair);
+        if (ck >= 1 && !bounded_wait(&bb.empty_c[cs], (ck - 1) & 1, abort_flag, p, 0x102, true))
+          return false;
+        ptx::mbar_arrive_expect_tx(&bb.full_c[cs], kPairBytes);
+        uint8_t* dst = smem + kOffPair + cs * kPairBytes;
+        ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, &bb.full_c[cs], policy);
+        ptx::tma_load_2d_hint(dst + kChunk, &p.tm_c, 128 * pr + 64, row, &bb.full_c[cs], policy);
+#pragma unroll
+        for (int q = 0; q < kNPair; ++q) if (q == cs) issued_c[q] = ck;
+        ++nc;
+      }
+      return true;
+    };
     for (int64_t u = u0; u < u1 && ok; ++u) {
-      const int64_t b = u / p.tiles_per_seq, tile = u % p.tiles_per_seq;
+      const int64_t b = u / p.tiles_per_seq;
+      if (u + kPrefetchAhead < u1) prefetch_tile(u + kPrefetchAhead);
       if (b != cur_b) {
         cur_b = b;
         ++seg;
@@ -267,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         ptx::tma_load_2d(smem + kOffQ + 8 * kQChunk, &p.tm_qr, 0, qrow, bb.q_full);
         issued_q = seg;
       }
-      const int32_t row = (int32_t)(b * p.L + tile * kT);
+      const int32_t row = tile_row(u);
       {
         const int ks = (int)(nk % kNKr);
         const int kk = (int)(nk / kNKr);
@@ -276,26 +360,20 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         if (!(p.debug_skip_load && nk == 0)) {
           ptx::mbar_arrive_expect_tx(&bb.full_k[ks], kChunk);
           ptx::tma_load_2d(smem + kOffKr + ks * kChunk, &p.tm_k, 0, row, &bb.full_k[ks]);
-          issued_k[ks] = kk;
+#pragma unroll
+          for (int q = 0; q < kNKr; ++q) if (q == ks) issued_k[q] = kk;
         }
         ++nk;
       }
-      for (int pr = 0; pr < 4 && ok; ++pr) {
-        const int cs = (int)(nc % kNPair);
-        const int ck = (int)(nc / kNPair);
-        if (ck >= 1) ok = bounded_wait(&bb.empty_c[cs], (ck - 1) & 1, abort_flag, p, 0x102, true);
-        if (!ok) break;
-        ptx::mbar_arrive_expect_tx(&bb.full_c[cs], kPairBytes);
-        uint8_t* dst = smem + kOffPair + cs * kPairBytes;
-        ptx::tma_load_2d(dst, &p.tm_c, 128 * pr, row, &bb.full_c[cs]);
-        ptx::tma_load_2d(dst + kChunk, &p.tm_c, 128 * pr + 64, row, &bb.full_c[cs]);
-        issued_c[cs] = ck;
-        ++nc;
-      }
+      ok = load_pairs(row, keep);                       // scores(u)
+      if (ok && u > u0) ok = load_pairs(tile_row(u - 1), drop);   // O(u-1)
     }
+    if (ok && u1 > u0) load_pairs(tile_row(u1 - 1), drop);        // O(last)
     // Let every copy this thread started land before the CTA can exit.
+#pragma unroll
     for (int i = 0; i < kNPair; ++i)
       if (issued_c[i] >= 0) bounded_wait(&bb.full_c[i], issued_c[i] & 1, abort_flag, p, 0x1F0, false);
+#pragma unroll
     for (int i = 0; i < kNKr; ++i)
       if (issued_k[i] >= 0) bounded_wait(&bb.full_k[i], issued_k[i] & 1, abort_flag, p, 0x1F1, false);
     if (issued_q >= 0) bounded_wait(bb.q_full, issued_q & 1, abort_flag, p, 0x1F2, false);
@@ -303,14 +381,65 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     // ===================================================== MMA issuer
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kT, kHC, 0, 0);   // K-major A and B
     constexpr uint32_t kIdescP = ptx::idesc_bf16_f32(128, kHC, 1, 1);  // MN-major A and B
-    const uint32_t s_pair = ptx::smem_u32(smem + kOffPair);
-    const uint32_t s_kr = ptx::smem_u32(smem + kOffKr);
-    const uint32_t s_q = ptx::smem_u32(smem + kOffQ);
-    const uint32_t s_p = ptx::smem_u32(smem + kOffP);
+    // Descriptor templates; a K step adds (bytes >> 4) to the start-address field.
+    const uint64_t d_pair = ptx::smem_desc(ptx::smem_u32(smem + kOffPair), 16, 1024, ptx::kSwizzle128B);
+    const uint64_t d_kr = ptx::smem_desc(ptx::smem_u32(smem + kOffKr), 16, 1024, ptx::kSwizzle128B);
+    const uint64_t d_q = ptx::smem_desc(ptx::smem_u32(smem + kOffQ), 16, 1024, ptx::kSwizzle128B);
+    // A = C^T, M = 128 latent dims (two 64-dim atoms 16 KB apart), K = 16 tokens
+    const uint64_t d_ct = ptx::smem_desc(ptx::smem_u32(smem + kOffPair), kChunk, 1024, ptx::kSwizzle128B);
+    // B = P^T, N = 16 heads (8-head core blocks 2 KB apart), K = 16 tokens
+    const uint64_t d_pt = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 128, 2048, ptx::kSwizzleNone);
     int64_t nc = 0, nk = 0, i = 0;
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
+
+    // O^T(j) = C_KV(j)^T . P^T(j): the next four ring entries hold tile j's pairs again
+    auto issue_pc = [&](int64_t j) -> bool {
+      const int buf = (int)(j & 1), kb = (int)(j >> 1);
+      if (!bounded_wait(&bb.p_full[buf], kb & 1, abort_flag, p, 0x204, true)) return false;
+      if (kb >= 1 && !bounded_wait(&bb.o_empty[buf], (kb - 1) & 1, abort_flag, p, 0x205, true))
+        return false;
+      const uint64_t bpt = d_pt + (uint64_t)((buf * kPBytes) >> 4);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int cs = (int)(nc % kNPair);
+        if (!bounded_wait(&bb.full_c[cs], (int)(nc / kNPair) & 1, abort_flag, p, 0x206, true))
+          return false;
+        ptx::tc_fence_after();
+        const uint32_t d_o = tmem + kColO + 64 * buf + 16 * m;
+        const uint64_t act = d_ct + (uint64_t)((cs * kPairBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_bf16_ss(d_o, act + (uint64_t)(kk * (2048 >> 4)), bpt + (uint64_t)(kk * (256 >> 4)),
+                           kIdescP, kk > 0);
+        ptx::mma_commit(&bb.empty_c[cs]);
+        ++nc;
+      }
+      ptx::mma_commit(&bb.o_full[buf]);
+      return true;
+    };
+    // scores(i) for column pair `pr` into sc of S buffer `buf`; frees the slot
+    auto issue_sc_pair = [&](int buf, int pr) -> bool {
+      const int cs = (int)(nc % kNPair);
+      if (!bounded_wait(&bb.full_c[cs], (int)(nc / kNPair) & 1, abort_flag, p, 0x203, true))
+        return false;
+      ptx::tc_fence_after();
+      const uint32_t d_sc = tmem + kColS + 32 * buf;
+      const uint64_t a0 = d_pair + (uint64_t)((cs * kPairBytes) >> 4);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ptx::mma_bf16_ss(d_sc, a0 + (uint64_t)((ch * kChunk + 32 * k) >> 4),
+                           d_q + (uint64_t)(((2 * pr + ch) * kQChunk + 32 * k) >> 4), kIdescS,
+                           (pr | ch | k) != 0);
+      }
+      ptx::mma_commit(&bb.empty_c[cs]);
+      ++nc;
+      return true;
+    };
+
     for (int64_t u = u0; u < u1 && ok; ++u, ++i) {
       const int64_t b = u / p.tiles_per_seq;
       const bool last_in_seg = (u + 1 == u1) || ((u + 1) / p.tiles_per_seq != b);
@@ -324,95 +453,56 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       const int kb = (int)(i >> 1);
       if (kb >= 1) ok = bounded_wait(&bb.s_empty[buf], (kb - 1) & 1, abort_flag, p, 0x201, true);
       if (!ok) break;
-      const uint32_t d_sc = tmem + kColS + 32 * buf;
-      const uint32_t d_sr = d_sc + 16;
-      // ---- sr = K_R tile . q_r^T
+      // ---- scores(i): sr = K_R . q_r^T, sc = C_KV . q_c^T
       {
         const int ks = (int)(nk % kNKr);
         ok = bounded_wait(&bb.full_k[ks], (int)(nk / kNKr) & 1, abort_flag, p, 0x202, true);
         if (!ok) break;
         ptx::tc_fence_after();
+        const uint32_t d_sr = tmem + kColS + 32 * buf + 16;
+        const uint64_t a0 = d_kr + (uint64_t)((ks * kChunk) >> 4);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t a = ptx::smem_desc(s_kr + ks * kChunk + 32 * k, 16, 1024, ptx::kSwizzle128B);
-          const uint64_t bq = ptx::smem_desc(s_q + 8 * kQChunk + 32 * k, 16, 1024, ptx::kSwizzle128B);
-          ptx::mma_bf16_ss(d_sr, a, bq, kIdescS, k > 0);
-        }
+        for (int k = 0; k < 4; ++k)
+          ptx::mma_bf16_ss(d_sr, a0 + (uint64_t)((32 * k) >> 4),
+                           d_q + (uint64_t)((8 * kQChunk + 32 * k) >> 4), kIdescS, k > 0);
         ++nk;
       }
-      // ---- sc = C_KV tile . q_c^T, one column pair (128 dims) per ring slot
-      int slotp[4];
-      for (int pr = 0; pr < 4; ++pr) {
-        const int cs = (int)(nc % kNPair);
-        ok = bounded_wait(&bb.full_c[cs], (int)(nc / kNPair) & 1, abort_flag, p, 0x203, true);
-        if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t a = ptx::smem_desc(s_pair + cs * kPairBytes + ch * kChunk + 32 * k, 16,
-                                              1024, ptx::kSwizzle128B);
-            const uint64_t bq = ptx::smem_desc(s_q + (2 * pr + ch) * kQChunk + 32 * k, 16, 1024,
-                                               ptx::kSwizzle128B);
-            ptx::mma_bf16_ss(d_sc, a, bq, kIdescS, (pr | ch | k) != 0);
-          }
-        }
-        slotp[pr] = cs;
-        ++nc;
-      }
+      ok = issue_sc_pair(buf, 0) && issue_sc_pair(buf, 1) && issue_sc_pair(buf, 2) &&
+           issue_sc_pair(buf, 3);
       if (!ok) break;
       ptx::mma_commit(&bb.s_full[buf]);   // also tells the softmax warps the K_R slot is read
       if (last_in_seg) ptx::mma_commit(bb.q_empty);
-      // ---- O^T tile = C_KV tile^T . P^T, four 128-dim blocks
-      ok = bounded_wait(&bb.p_full[buf], kb & 1, abort_flag, p, 0x204, true);
-      if (ok && kb >= 1) ok = bounded_wait(&bb.o_empty[buf], (kb - 1) & 1, abort_flag, p, 0x205, true);
-      if (!ok) break;
-      ptx::tc_fence_after();
-      for (int m = 0; m < 4; ++m) {
-        const uint32_t d_o = tmem + kColO + 64 * buf + 16 * m;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // A = C^T: M = 128 latent dims (two 64-dim atoms 16 KB apart), K = 16 tokens
-          const uint64_t a = ptx::smem_desc(s_pair + slotp[m] * kPairBytes + kk * 2048, kChunk,
-                                            1024, ptx::kSwizzle128B);
-          // B = P^T: N = 16 heads (8-head core blocks 2 KB apart), K = 16 tokens
-          const uint64_t bp = ptx::smem_desc(s_p + buf * kPBytes + kk * 256, 128, 2048,
-                                             ptx::kSwizzleNone);
-          ptx::mma_bf16_ss(d_o, a, bp, kIdescP, kk > 0);
-        }
-        ptx::mma_commit(&bb.empty_c[slotp[m]]);
-      }
-      ptx::mma_commit(&bb.o_full[buf]);
+      // ---- O(i-1), its softmax done while scores(i) ran
+      if (i > 0) ok = issue_pc(i - 1);
     }
+    if (ok && i > 0) issue_pc(i - 1);
     // Every MMA issued here must finish before TMEM is freed.
     ptx::mma_commit(bb.drain);
     bounded_wait(bb.drain, 0, abort_flag, p, 0x2F0, false);
   } else if (warp >= 2) {
     // ===================================================== softmax warps
-    // A failed wait only raises the abort flag; the four warps leave the tile
-    // loop together, at the one checkpoint barrier of each tile, so no warp
-    // is ever left waiting at a named barrier.
+    // A failed wait only raises the abort flag; the softmax warps leave the
+    // tile loop together, at the one checkpoint barrier of each tile, so no
+    // warp is ever left waiting at a named barrier.
     const int q4 = warp & 3;             // TMEM lane quarter this warp may access
+    const int hh = (warp - 2) >> 2;      // which 8 of the 16 heads
     const int row = q4 * 32 + lane;      // token row of the tile owned by this thread
-    const int st = tid - 64;             // 0..127 among the softmax threads
+    const int st = tid - 64;             // 0..255 among the softmax threads
     const uint32_t t_lane = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t t_cols = t_lane + kHH * hh;   // this thread's 8 head columns
     float* ks_tab = reinterpret_cast<float*>(smem + kOffK);      // [64][16] k_j
     float* gmax_s = reinterpret_cast<float*>(smem + kOffGmax);   // [16]
     float* wmax_s = reinterpret_cast<float*>(smem + kOffWmax);   // [4][16]
     float* zred = reinterpret_cast<float*>(smem + kOffZred);     // [4][16]
     uint8_t* pbase = smem + kOffP;
-    // group phase: threads per head (consecutive), groups per thread
-    constexpr int kGt = kT / g;                          // groups per tile
-    constexpr int kTpH = kGt < 8 ? kGt : 8;
-    constexpr int kGpt = kGt / kTpH;
-    constexpr int kActive = kHC * kTpH;
-    constexpr int kUnroll = g < 16 ? g : 16;             // full unroll would spill for g >= 64
+    // group phase: thread st scans tokens [8 sg, 8 sg + 8) of head gh
+    const int gh = st >> 4;
+    const int sg = st & 15;
 
-    float O[4][kHC];
-    float Zt[kHC], Mh[kHC], apend[kHC];
+    float O[4][kHH];
+    float Zt[kHH], Mh[kHH], apend[kHH];
 #pragma unroll
-    for (int h = 0; h < kHC; ++h) {
+    for (int h = 0; h < kHH; ++h) {
       Zt[h] = 0.f; Mh[h] = -INFINITY; apend[h] = 0.f;
 #pragma unroll
       for (int m = 0; m < 4; ++m) O[m][h] = 0.f;
@@ -430,9 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       float* stage = reinterpret_cast<float*>(smem + kOffKr + ks * kChunk);
       warp_wait(&bb.s_full[buf], kb & 1, abort_flag, p, 0x300);
       ptx::tc_fence_after();
-      float sc[kHC], sr[kHC];
-      ptx::tmem_ld16(t_lane + kColS + 32 * buf, sc);
-      ptx::tmem_ld16(t_lane + kColS + 32 * buf + 16, sr);
+      float sc[kHH], sr[kHH];
+      ptx::tmem_ld8(t_cols + kColS + 32 * buf, sc);
+      ptx::tmem_ld8(t_cols + kColS + 32 * buf + 16, sr);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
@@ -445,161 +535,174 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       // tile-uniform flags
       const bool tile_groups = (g > 1) && (tok0 < win0);
       const bool tile_tokens = (g == 1) || (tok0 + kT > win0);   // per-token entries present
-      float s[kHC];
+      float s[kHH];
 #pragma unroll
-      for (int h = 0; h < kHC; ++h) s[h] = sc[h] + sr[h];
+      for (int h = 0; h < kHH; ++h) s[h] = sc[h] + sr[h];
 
       if (tile_groups) {
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 v = c4 < 4 ? make_float4(sc[4 * c4], sc[4 * c4 + 1], sc[4 * c4 + 2], sc[4 * c4 + 3])
-                                  : make_float4(sr[4 * c4 - 16], sr[4 * c4 - 15], sr[4 * c4 - 14],
-                                                sr[4 * c4 - 13]);
-          *reinterpret_cast<float4*>(stage + stage_idx<LOG2G>(row, 4 * c4)) = v;
-        }
+        *reinterpret_cast<float4*>(stage + stage_idx(row, kHH * hh)) =
+            make_float4(sc[0], sc[1], sc[2], sc[3]);
+        *reinterpret_cast<float4*>(stage + stage_idx(row, kHH * hh + 4)) =
+            make_float4(sc[4], sc[5], sc[6], sc[7]);
+        *reinterpret_cast<float4*>(stage + stage_idx(row, 16 + kHH * hh)) =
+            make_float4(sr[0], sr[1], sr[2], sr[3]);
+        *reinterpret_cast<float4*>(stage + stage_idx(row, 16 + kHH * hh + 4)) =
+            make_float4(sr[4], sr[5], sr[6], sr[7]);
       }
-      ptx::named_bar_sync(kSoftmaxBar, 128);                     // B1: staged scores visible
+      ptx::named_bar_sync(kSoftmaxBar, kSoftmaxThreads);          // B1: staged scores visible
 
-      if (tile_groups && st < kActive) {
-        // ---- step 2, one thread per (group, head)
-        const int h = st / kTpH;
-        const int j0 = st % kTpH;
-        float gm = -INFINITY;
+      if (tile_groups) {
+        // ---- step 2: this thread's 8-token segment of head gh
+        const int row0 = 8 * sg;
+        float x[8], cv[8];
 #pragma unroll
-        for (int r = 0; r < kGpt; ++r) {
-          const int j = j0 + kTpH * r;                 // group within the tile
-          const int64_t jg = tok0 / g + j;             // group within the sequence
+        for (int v = 0; v < 8; ++v) {
+          cv[v] = stage[stage_idx(row0 + v, gh)];
+          x[v] = cv[v] + stage[stage_idx(row0 + v, 16 + gh)];   // the same fp32 sum as s above
+        }
+        float gm = -INFINITY;
+        if (g >= 8) {
+          GroupStat r = scan_group<8>(x, cv, 0, row0);
+          // merge the g/8 segments of a group (consecutive lanes)
+#pragma unroll
+          for (int off = 1; off < (g >= 8 ? g / 8 : 1); off <<= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, r.m, off);
+            const int oa = __shfl_xor_sync(0xffffffffu, r.a, off);
+            const float od = __shfl_xor_sync(0xffffffffu, r.den, off);
+            const float on = __shfl_xor_sync(0xffffffffu, r.num, off);
+            const float mm = fmaxf(r.m, om);
+            const float f1 = ex2((r.m - mm) * kLog2e), f2 = ex2((om - mm) * kLog2e);
+            r.den = r.den * f1 + od * f2;
+            r.num = r.num * f1 + on * f2;
+            if (om > r.m || (om == r.m && oa < r.a)) r.a = oa;
+            r.m = mm;
+          }
+          const int j = row0 / g;                    // group within the tile
+          const int64_t jg = tok0 / g + j;            // group within the sequence
           if (jg < p.nG) {
-            const int r0 = j * g;
-            float m = -INFINITY;
-            int a = 0;
-#pragma unroll kUnroll
-            for (int v = 0; v < g; ++v) {
-              const float x = stage[stage_idx<LOG2G>(r0 + v, h)] + stage[stage_idx<LOG2G>(r0 + v, 16 + h)];
-              if (x > m) { m = x; a = v; }             // strict: the lowest index keeps a tie
+            const float S = __fdividef(r.num, r.den) + stage[stage_idx(r.a, 16 + gh)];
+            gm = S;
+            if ((sg & (g / 8 - 1)) == 0) {
+              ks_tab[j * kHC + gh] = S - r.m - lg2(r.den) * kLn2;
+              p.anchor[((int64_t)b * p.H + h0 + gh) * p.nG + jg] = (int32_t)(tok0 + r.a);
             }
-            float den = 0.f, num = 0.f;
-            const float mb = m * kLog2e;
-#pragma unroll kUnroll
-            for (int v = 0; v < g; ++v) {
-              const float scv = stage[stage_idx<LOG2G>(r0 + v, h)];
-              const float x = scv + stage[stage_idx<LOG2G>(r0 + v, 16 + h)];
-              const float e = ex2(fmaf(x, kLog2e, -mb));
-              den += e;
-              num = fmaf(e, scv, num);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8 / g; ++q) {
+            const GroupStat r = scan_group<(g < 8 ? g : 1)>(x, cv, q * g, row0);
+            const int j = row0 / g + q;
+            const int64_t jg = tok0 / g + j;
+            if (jg < p.nG) {
+              const float S = __fdividef(r.num, r.den) + stage[stage_idx(r.a, 16 + gh)];
+              gm = fmaxf(gm, S);
+              ks_tab[j * kHC + gh] = S - r.m - lg2(r.den) * kLn2;
+              p.anchor[((int64_t)b * p.H + h0 + gh) * p.nG + jg] = (int32_t)(tok0 + r.a);
             }
-            const float sra = stage[stage_idx<LOG2G>(r0 + a, 16 + h)];   // K_R score of the anchor
-            const float S = __fdividef(num, den) + sra;                 // condensed logit
-            ks_tab[j * kHC + h] = S - m - __logf(den);                  // k_j
-            gm = fmaxf(gm, S);
-            p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + jg] = (int32_t)(tok0 + r0 + a);
           }
         }
+        // max over the head's 16 segments (lanes 16*(gh&1) .. +15)
 #pragma unroll
-        for (int off = 1; off < kTpH; off <<= 1)
-          gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, off));
-        if (j0 == 0) gmax_s[h] = gm;
+        for (int off = 1; off < 16; off <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, off));
+        if (sg == 0) gmax_s[gh] = gm;
       }
       if (tile_tokens) {
         // window tokens (and g = 1, where every grouped token is its own entry)
         const bool own = valid && (!grouped || g == 1);
         if (g == 1 && grouped) {
 #pragma unroll
-          for (int h = 0; h < kHC; ++h)
-            p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + t] = (int32_t)t;
+          for (int h = 0; h < kHH; ++h)
+            p.anchor[((int64_t)b * p.H + h0 + kHH * hh + h) * p.nG + t] = (int32_t)t;
         }
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) {
+        for (int h = 0; h < kHH; ++h) {
           float v = own ? s[h] : -INFINITY;
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-          if (lane == 0) wmax_s[q4 * kHC + h] = v;
+          if (lane == 0) wmax_s[q4 * kHC + kHH * hh + h] = v;
         }
       }
       // B2, checkpoint: the only place the softmax warps leave the loop early
-      const bool stop = ptx::named_bar_or(kSoftmaxBar, 128, *abort_flag != 0);
+      const bool stop = ptx::named_bar_or(kSoftmaxBar, kSoftmaxThreads, *abort_flag != 0);
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bb.empty_k[ks]);   // staging in the K_R slot is done
       if (stop) break;
 
       // ---- step 3: tile maximum over entries, per-token weights
-      float alpha[kHC], mb[kHC];
+      float alpha[kHH], mb[kHH], kt[kHH];
 #pragma unroll
-      for (int h = 0; h < kHC; ++h) {
-        float mt = tile_groups ? gmax_s[h] : -INFINITY;
+      for (int h = 0; h < kHH; ++h) {
+        const int hg = kHH * hh + h;
+        float mt = tile_groups ? gmax_s[hg] : -INFINITY;
         if (tile_tokens)
-          mt = fmaxf(mt, fmaxf(fmaxf(wmax_s[h], wmax_s[kHC + h]),
-                               fmaxf(wmax_s[2 * kHC + h], wmax_s[3 * kHC + h])));
+          mt = fmaxf(mt, fmaxf(fmaxf(wmax_s[hg], wmax_s[kHC + hg]),
+                               fmaxf(wmax_s[2 * kHC + hg], wmax_s[3 * kHC + hg])));
         const float mn = fmaxf(Mh[h], mt);
         alpha[h] = ex2((Mh[h] - mn) * kLog2e);   // 0 on the first tile of a range
         Mh[h] = mn;
         mb[h] = mn * kLog2e;
+        kt[h] = 0.f;
       }
-      float pv[kHC];
       if (grouped && g > 1) {
-        const float* kr = ks_tab + (row / g) * kHC;
-#pragma unroll
-        for (int h4 = 0; h4 < 4; ++h4) {
-          const float4 k4 = *reinterpret_cast<const float4*>(kr + 4 * h4);
-          pv[4 * h4 + 0] = ex2(fmaf(s[4 * h4 + 0] + k4.x, kLog2e, -mb[4 * h4 + 0]));
-          pv[4 * h4 + 1] = ex2(fmaf(s[4 * h4 + 1] + k4.y, kLog2e, -mb[4 * h4 + 1]));
-          pv[4 * h4 + 2] = ex2(fmaf(s[4 * h4 + 2] + k4.z, kLog2e, -mb[4 * h4 + 2]));
-          pv[4 * h4 + 3] = ex2(fmaf(s[4 * h4 + 3] + k4.w, kLog2e, -mb[4 * h4 + 3]));
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < kHC; ++h) pv[h] = valid ? ex2(fmaf(s[h], kLog2e, -mb[h])) : 0.f;
+        const float* kr = ks_tab + (row / g) * kHC + kHH * hh;
+        const float4 k0 = *reinterpret_cast<const float4*>(kr);
+        const float4 k1 = *reinterpret_cast<const float4*>(kr + 4);
+        kt[0] = k0.x; kt[1] = k0.y; kt[2] = k0.z; kt[3] = k0.w;
+        kt[4] = k1.x; kt[5] = k1.y; kt[6] = k1.z; kt[7] = k1.w;
       }
-      // ---- P^T tile, bf16, MN-major core matrices: token row -> K, head -> N
-      uint32_t pk[8];
+      float pv[kHH];
 #pragma unroll
-      for (int h2 = 0; h2 < 8; ++h2) {
+      for (int h = 0; h < kHH; ++h) pv[h] = valid ? ex2(fmaf(s[h] + kt[h], kLog2e, -mb[h])) : 0.f;
+      // ---- P^T tile, bf16, MN-major core matrices: token row -> K, head -> N
+      uint32_t pk[4];
+#pragma unroll
+      for (int h2 = 0; h2 < 4; ++h2) {
         pk[h2] = pack_bf16x2(pv[2 * h2], pv[2 * h2 + 1]);
         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pk[h2]);
         Zt[2 * h2] = fmaf(Zt[2 * h2], alpha[2 * h2], __low2float(v));   // Z from the rounded P
         Zt[2 * h2 + 1] = fmaf(Zt[2 * h2 + 1], alpha[2 * h2 + 1], __high2float(v));
       }
-      uint8_t* prow = pbase + buf * kPBytes + (row >> 3) * 128 + (row & 7) * 16;
+      uint8_t* prow = pbase + buf * kPBytes + (row >> 3) * 128 + (row & 7) * 16 + hh * 2048;
       *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(prow + 2048) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bb.p_full[buf]);
 
       // ---- fold the previous tile's O^T; at a range end also this tile's, then write
-      if (pending) fold_o(O, apend, pbuf, pkb, t_lane, bb, abort_flag, p);
+      if (pending) fold_o(O, apend, pbuf, pkb, t_cols, bb, abort_flag, p);
 #pragma unroll
-      for (int h = 0; h < kHC; ++h) apend[h] = alpha[h];
+      for (int h = 0; h < kHH; ++h) apend[h] = alpha[h];
       pending = true;
       pbuf = buf;
       pkb = kb;
       if (last_in_seg) {
-        fold_o(O, alpha, buf, kb, t_lane, bb, abort_flag, p);
+        fold_o(O, alpha, buf, kb, t_cols, bb, abort_flag, p);
         pending = false;
         const int64_t slot = b + c;
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) {
-          float* po = p.part_o + (slot * p.H + h0 + h) * kDC;
+        for (int h = 0; h < kHH; ++h) {
+          float* po = p.part_o + (slot * p.H + h0 + kHH * hh + h) * kDC;
 #pragma unroll
           for (int m = 0; m < 4; ++m) po[128 * m + row] = O[m][h];
           float z = Zt[h];
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-          if (lane == 0) zred[q4 * kHC + h] = z;
+          if (lane == 0) zred[q4 * kHC + kHH * hh + h] = z;
         }
-        ptx::named_bar_sync(kSoftmaxBar, 128);
-        if (warp == 2 && lane < kHC) {
+        ptx::named_bar_sync(kSoftmaxBar, kSoftmaxThreads);
+        if (q4 == 0 && lane < kHH) {
           float Mv = 0.f;
 #pragma unroll
-          for (int h = 0; h < kHC; ++h) if (h == lane) Mv = Mh[h];
-          const float z = zred[lane] + zred[kHC + lane] + zred[2 * kHC + lane] + zred[3 * kHC + lane];
-          p.part_mz[(slot * p.H + h0 + lane) * 2 + 0] = Mv;
-          p.part_mz[(slot * p.H + h0 + lane) * 2 + 1] = z;
+          for (int h = 0; h < kHH; ++h) if (h == lane) Mv = Mh[h];
+          const int hg = kHH * hh + lane;
+          const float z = zred[hg] + zred[kHC + hg] + zred[2 * kHC + hg] + zred[3 * kHC + hg];
+          p.part_mz[(slot * p.H + h0 + hg) * 2 + 0] = Mv;
+          p.part_mz[(slot * p.H + h0 + hg) * 2 + 1] = z;
         }
-        ptx::named_bar_sync(kSoftmaxBar, 128);
+        ptx::named_bar_sync(kSoftmaxBar, kSoftmaxThreads);
 #pragma unroll
-        for (int h = 0; h < kHC; ++h) {
+        for (int h = 0; h < kHH; ++h) {
           Zt[h] = 0.f; Mh[h] = -INFINITY;
 #pragma unroll
           for (int m = 0; m < 4; ++m) O[m][h] = 0.f;
