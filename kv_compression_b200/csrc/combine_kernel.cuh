@@ -33,6 +33,7 @@ __device__ __forceinline__ int64_t range_owner(int64_t u, int64_t U, int64_t G) 
   return ((u + 1) * G - 1) / U;  // largest c with floor(c*U/G) <= u
 }
 
+// Grid: (H, B, d_c / kCombineThreads); one thread per latent dimension.
 __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const CombineParams p) {
   __shared__ float scale[kCombineMaxParts];
   __shared__ float red[kCombineThreads / 32];
@@ -50,17 +51,19 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     count = c1 - c0 + 1;
   }
   if (count > kCombineMaxParts) count = kCombineMaxParts;  // the host never plans more
-  // M = max_i M_i
+  // M = max_i M_i (partials read in parallel)
   float m = -INFINITY;
   for (int64_t i = tid; i < count; i += kCombineThreads)
     m = fmaxf(m, p.part_mz[((first + i) * p.H + h) * 2]);
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((tid & 31) == 0) red[tid >> 5] = m;
   __syncthreads();
   float M = red[0];
+#pragma unroll
   for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, red[w]);
   __syncthreads();
-  // per-partial factors e^{M_i - M} and Z
+  // factors e^{M_i - M} and Z = sum_i e^{M_i - M} Z_i
   float z = 0.f;
   for (int64_t i = tid; i < count; i += kCombineThreads) {
     const float* mz = p.part_mz + ((first + i) * p.H + h) * 2;
@@ -68,27 +71,31 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     scale[i] = f;
     z = fmaf(f, mz[1], z);
   }
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   if ((tid & 31) == 0) red[tid >> 5] = z;
   __syncthreads();
   float Z = 0.f;
+#pragma unroll
   for (int w = 0; w < kCombineThreads / 32; ++w) Z += red[w];
   const float invZ = 1.f / Z;
-  // out[d] = sum_i f_i O_i[d] / Z; four independent accumulators per thread
-  const float* po = p.part_o + (first * p.H + h) * (int64_t)p.d_c;
+  // out[d] = sum_i f_i O_i[d] / Z with eight loads in flight
+  const int d = blockIdx.z * kCombineThreads + tid;
+  if (d >= p.d_c) return;
   const int64_t stride = (int64_t)p.H * p.d_c;
-  for (int d = tid; d < p.d_c; d += kCombineThreads) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int64_t i = 0;
-    for (; i + 4 <= count; i += 4) {
-      a0 = fmaf(scale[i], po[i * stride + d], a0);
-      a1 = fmaf(scale[i + 1], po[(i + 1) * stride + d], a1);
-      a2 = fmaf(scale[i + 2], po[(i + 2) * stride + d], a2);
-      a3 = fmaf(scale[i + 3], po[(i + 3) * stride + d], a3);
-    }
-    for (; i < count; ++i) a0 = fmaf(scale[i], po[i * stride + d], a0);
-    p.out[((int64_t)b * p.H + h) * p.d_c + d] = ((a0 + a1) + (a2 + a3)) * invZ;
+  const float* po = p.part_o + (first * p.H + h) * (int64_t)p.d_c + d;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int64_t i = 0;
+  for (; i + 8 <= count; i += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = po[(i + k) * stride];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(scale[i + k], v[k], acc[k]);
   }
+  for (; i < count; ++i) acc[0] = fmaf(scale[i], po[i * stride], acc[0]);
+  const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  p.out[((int64_t)b * p.H + h) * p.d_c + d] = sum * invZ;
 }
 
 }  // namespace lca

@@ -102,7 +102,8 @@ Kernel choose(const lca_plan* p, int64_t nG, int g) {
 lca_status launch_combine(const lca_plan* p, const lca::CombineParams& cp, cudaStream_t stream,
                           bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p->H, (unsigned)p->B, 1);
+  cfg.gridDim = dim3((unsigned)p->H, (unsigned)p->B,
+                     (unsigned)((p->d_c + lca::kCombineThreads - 1) / lca::kCombineThreads));
   cfg.blockDim = dim3(lca::kCombineThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
