@@ -151,6 +151,32 @@ lca_status lca_plan_set_timing_event(lca_plan *plan, void *event);
 /* Which kernel a plan runs for (L, g, w): 0 = none (invalid), 1 = CUDA-core, 2 = tcgen05. */
 int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
 
+/*
+ * lca_decode without a plan and without any allocation.  The page has no
+ * counterpart: this is a deployment variant of lca_decode for callers that may
+ * not allocate device memory when they decode (a server whose memory is all
+ * reserved up front by its own pool, where a cudaMalloc would fail or
+ * fragment it, and which cannot keep a plan per shape).
+ * Arguments: B, H, d_c, d_r and dt as for lca_plan_create; the rest, their
+ * layouts and ownership as for lca_decode (L has no max_L bound).  Same
+ * kernels and results as lca_decode.
+ * Scratch: the split partials live in one fixed file-scope device array of
+ * 16 MiB (plus 64 KiB), so the tile ranges are capped to what fits; shapes
+ * with B * H * d_c > 4 Mi floats return LCA_ERR_UNSUPPORTED.  The device error
+ * word in that array is cleared on `stream` at the start of every call; a
+ * bounded in-kernel wait that runs out leaves outputs undefined and is not
+ * reported by this call.
+ * The first call on a device looks up the scratch's address there and sets
+ * the kernels' shared-memory limit; make that first call before any stream
+ * capture.  Every call on a device shares the one scratch: calls that overlap
+ * in time (two streams, or two host threads) race and corrupt each other's
+ * results.  Errors: LCA_ERR_INVALID_ARG, LCA_ERR_UNSUPPORTED,
+ * LCA_ERR_ALIGNMENT, LCA_ERR_CUDA.
+ */
+lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, const void *q_c,
+                              const void *q_r, const void *c_kv, const void *k_r, int64_t L, int g,
+                              int w, float *out, int32_t *anchor_idx, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

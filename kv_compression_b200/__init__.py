@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblca.so")
 
 LCA_OK = 0
+LCA_ERR_UNSUPPORTED = 2
 LCA_ERR_DEVICE_TIMEOUT = 5
 STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED", 3: "LCA_ERR_ALIGNMENT",
           4: "LCA_ERR_CUDA", 5: "LCA_ERR_DEVICE_TIMEOUT", 6: "LCA_ERR_PLAN_MISMATCH",
@@ -25,7 +26,7 @@ KERNEL_NAMES = {0: "none", 1: "simt", 2: "tcgen05"}
 
 EXPORTS = ["lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
            "lca_decode_host", "lca_num_groups", "lca_status_string", "lca_get_device_error",
-           "lca_plan_kernel", "lca_plan_set_timing_event"]
+           "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc"]
 
 
 class LcaError(RuntimeError):
@@ -59,9 +60,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lca_get_device_error.argtypes = [vp, vp]
     lib.lca_plan_kernel.argtypes = [vp, i64, i32, i32]
     lib.lca_plan_set_timing_event.argtypes = [vp, vp]
+    lib.lca_decode_noalloc.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i32, i32, vp,
+                                       vp, vp]
     for name in ("lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
                  "lca_decode_host", "lca_get_device_error", "lca_plan_kernel",
-                 "lca_plan_set_timing_event"):
+                 "lca_plan_set_timing_event", "lca_decode_noalloc"):
         getattr(lib, name).restype = i32
     if path == LIB_PATH:
         _lib = lib

@@ -40,6 +40,15 @@ struct lca_plan {
   int32_t* st_anc;
 };
 
+// Fixed device scratch of lca_decode_noalloc (zero at module load): split
+// partials [slots][H][d_c] and [slots][H][2] floats, then the device error
+// word (2 ints).  Only lca_decode_noalloc uses it, through the address that
+// cudaGetSymbolAddress gives for the current device.
+constexpr size_t kNoAllocOFloats = (size_t)4 << 20;              // 16 MiB of partial outputs
+constexpr size_t kNoAllocMzFloats = kNoAllocOFloats / 256;       // (M, Z) pairs of the same slots
+constexpr size_t kNoAllocErrOffset = kNoAllocOFloats + kNoAllocMzFloats;
+static __device__ __align__(256) float lca_noalloc_scratch[kNoAllocErrOffset + 64];
+
 namespace {
 
 constexpr int64_t kDefaultTimeoutNs = 2000000000LL;  // 2 s bound on any in-kernel wait
@@ -400,6 +409,61 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
     return LCA_ERR_CUDA;
   if (host[0] != 0 && cudaMemset(p->err, 0, sizeof(host)) != cudaSuccess) return LCA_ERR_CUDA;
   return host[0] != 0 ? LCA_ERR_DEVICE_TIMEOUT : LCA_OK;
+}
+
+// For callers that may not allocate device memory when they decode -- a
+// server whose memory is all reserved up front by its own pool (a cudaMalloc
+// here would fail or fragment it) and that cannot keep a plan per shape --
+// this entry point runs the same kernels as lca_decode with the fixed
+// file-scope scratch above in place of a plan's workspace, and allocates
+// nothing.  The first call on a device looks up the scratch's address there
+// (cudaGetSymbolAddress) and sets the kernels' shared-memory limit.
+lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, const void* q_c,
+                              const void* q_r, const void* c_kv, const void* k_r, int64_t L, int g,
+                              int w, float* out, int32_t* anchor, void* stream) {
+  constexpr int kMaxDevices = 64;
+  static float* scratch[kMaxDevices] = {};   // the scratch's address, per device
+  static int sms[kMaxDevices] = {};
+  if (B < 1 || H < 1 || d_c < 1 || d_r < 1 || L < 1 || g < 1 || w < 0) return LCA_ERR_INVALID_ARG;
+  if (!q_c || !q_r || !c_kv || !k_r || !out) return LCA_ERR_INVALID_ARG;
+  if (dt != LCA_F32 && dt != LCA_BF16) return LCA_ERR_INVALID_ARG;
+  if (d_c > lca::kSimtMaxDc || d_r > 256 || H > 4096 || (d_c % 8) != 0 || (d_r % 8) != 0)
+    return LCA_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LCA_ERR_UNSUPPORTED;
+  if (!scratch[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, lca_noalloc_scratch) != cudaSuccess) return LCA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return LCA_ERR_CUDA;
+    scratch[dev] = static_cast<float*>(ptr);
+  }
+  // Split slots that fit the scratch; fewer than B is a size beyond its limit.
+  const int64_t cap = (int64_t)(kNoAllocOFloats / ((size_t)H * (size_t)d_c));
+  if (cap < B) return LCA_ERR_UNSUPPORTED;
+  lca_plan plan;
+  std::memset(&plan, 0, sizeof(plan));
+  plan.B = B; plan.H = H; plan.d_c = d_c; plan.d_r = d_r; plan.dt = dt; plan.max_L = L;
+  plan.device = dev;
+  plan.num_sms = sms[dev];
+  plan.tc_shape = dt == LCA_BF16 && d_c == lca::tc::kDC && d_r == lca::tc::kDR &&
+                  (H % lca::tc::kHC) == 0;
+  plan.ws_slots = cap;
+  plan.part_o = scratch[dev];
+  plan.part_mz = scratch[dev] + kNoAllocOFloats;
+  plan.err = reinterpret_cast<int*>(scratch[dev] + kNoAllocErrOffset);
+  plan.timeout_ns = kDefaultTimeoutNs;
+  if (plan.tc_shape) {   // as many tile ranges as the scratch holds partials for
+    const int64_t n_hb = H / lca::tc::kHC;
+    plan.num_ctas = (int)std::min<int64_t>(plan.num_sms, n_hb * (cap - B + 1));
+    if (plan.num_ctas < n_hb) plan.num_ctas = (int)n_hb;
+  }
+  // The kernels only OR into the error word, so it must start each call at zero.
+  if (cudaMemsetAsync(plan.err, 0, 2 * sizeof(int), static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return LCA_ERR_CUDA;
+  return decode_impl(&plan, q_c, q_r, c_kv, k_r, L, g, w, out, anchor, stream, false);
 }
 
 }  // extern "C"
