@@ -153,11 +153,15 @@ __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.  The
+// warp reconverges here even when the caller ignores the verdict, so the
+// other lanes wait at this barrier rather than at the next aligned tcgen05
+// instruction.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const TcParams& p, int where) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, abort, p, where, true);
+  __syncwarp();
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -674,6 +678,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   }
 
   // ===================================================== teardown
+  // Lanes that skipped a one-lane role wait for their lane 0 first.
+  __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
