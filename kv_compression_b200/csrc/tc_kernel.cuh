@@ -58,7 +58,9 @@ constexpr int kDR = 64;                    // RoPE key width
 constexpr int kChunk = kT * 128;           // [128 rows][64 bf16] = 16 KB
 constexpr int kPairBytes = 2 * kChunk;     // two 64-dim chunks = 128 latent dims
 constexpr int kPairsPerTile = kDC / 128;
-constexpr int kNPair = 5;                  // C_KV pair slots: one tile plus one pair
+constexpr int kNPair = 5;                  // C_KV pair slots: ring A (2) then ring B (3)
+constexpr int kNA = 2;                     // ring A: column pairs 0-1, streamed
+constexpr int kNB = kNPair - kNA;          // ring B: column pairs 2-3, held until O
 constexpr int kNKr = 2;                    // K_R slots
 constexpr int kQChunk = kHC * 128;         // [16 heads][64 bf16] = 2 KB
 constexpr int kQBytes = 9 * kQChunk;       // 8 chunks of q_c, 1 of q_r
@@ -69,7 +71,6 @@ constexpr int kOWarp = 2 + kSoftmaxWarps;   // issues O^T += C^T P^T
 constexpr int kThreads = 32 * (kOWarp + 1);
 constexpr int kTmemCols = 128;
 constexpr int kSoftmaxBar = 1;             // named barrier of the softmax warps
-constexpr int kPrefetchAhead = 2;          // tiles brought into L2 ahead of their loads
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.f;        // M rises once an entry exceeds it by 2^8
@@ -84,7 +85,7 @@ constexpr int kOffGanc = kOffGpart + 4 * kHC * 16;      // int [4][16]: row of t
 constexpr int kOffWmax = kOffGanc + 4 * kHC * 4;        // float [4][16]: max entry per quarter
 constexpr int kOffZred = kOffWmax + 4 * kHC * 4;        // float [4][16]
 constexpr int kOffBar = kOffZred + 4 * kHC * 4;
-constexpr int kNumBars = 2 * kNPair + 2 * kNKr + 2 + 4 * 2 + 2;
+constexpr int kNumBars = 2 * kNPair + 2 * kNA + 2 * kNKr + 2 + 4 * 2 + 2;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;          // alignment slack
@@ -118,8 +119,15 @@ struct TcParams {
 };
 
 struct Bars {
-  uint64_t* full_c;   // [kNPair]
-  uint64_t* empty_c;  // [kNPair]  released after O += C^T P^T of the slot's tile
+  // Ring A slot s holds column pair s, loaded alternately for the scores and
+  // (again) for O; each use has its own full/empty pair, so that every barrier
+  // is waited on by one thread, phase after phase.
+  uint64_t* full_as;  // [kNA]  scores load landed
+  uint64_t* full_ar;  // [kNA]  reload for O landed
+  uint64_t* empty_as; // [kNA]  released after the score MMAs
+  uint64_t* empty_ar; // [kNA]  released after O += C^T P^T
+  uint64_t* full_b;   // [kNB]  ring B
+  uint64_t* empty_b;  // [kNB]  released after O += C^T P^T of the slot's tile
   uint64_t* full_k;   // [kNKr]
   uint64_t* empty_k;  // [kNKr]
   uint64_t* q_full;
@@ -231,9 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   Bars bb;
-  bb.full_c = bars;
-  bb.empty_c = bb.full_c + kNPair;
-  bb.full_k = bb.empty_c + kNPair;
+  bb.full_as = bars;
+  bb.full_ar = bb.full_as + kNA;
+  bb.empty_as = bb.full_ar + kNA;
+  bb.empty_ar = bb.empty_as + kNA;
+  bb.full_b = bb.empty_ar + kNA;
+  bb.empty_b = bb.full_b + kNB;
+  bb.full_k = bb.empty_b + kNB;
   bb.empty_k = bb.full_k + kNKr;
   bb.q_full = bb.empty_k + kNKr;
   bb.q_empty = bb.q_full + 1;
@@ -262,7 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   };
 
   if (tid == 0) {
-    for (int i = 0; i < kNPair; ++i) { ptx::mbar_init(&bb.full_c[i], 1); ptx::mbar_init(&bb.empty_c[i], 1); }
+    for (int i = 0; i < kNA; ++i) {
+      ptx::mbar_init(&bb.full_as[i], 1); ptx::mbar_init(&bb.full_ar[i], 1);
+      ptx::mbar_init(&bb.empty_as[i], 1); ptx::mbar_init(&bb.empty_ar[i], 1);
+    }
+    for (int i = 0; i < kNB; ++i) { ptx::mbar_init(&bb.full_b[i], 1); ptx::mbar_init(&bb.empty_b[i], 1); }
     for (int i = 0; i < kNKr; ++i) { ptx::mbar_init(&bb.full_k[i], 1); ptx::mbar_init(&bb.empty_k[i], 1); }
     ptx::mbar_init(bb.q_full, 1);
     ptx::mbar_init(bb.q_empty, 1);
@@ -288,35 +304,84 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ===================================================== TMA producer
-    // Per tile: K_R, then the four column pairs of C_KV into the next ring
-    // slots.  A slot is reused once O += C^T P^T of its previous tile is done.
+    // Two rings of 32 KB column-pair slots.  Ring B (3 slots) holds pairs 2-3
+    // of a tile from their load until O += C^T P^T of that tile.  Ring A (2
+    // slots) streams pairs 0-1: once for the scores (kept in L2 with an
+    // evict-last hint) and once more, read back from L2, for O.  So during the
+    // softmax of tile i, the scores of tile i+1 run on its pairs 0-2 and the
+    // pairs 0-1 of tile i come back for O(i); pair 3 of tile i+1 follows as
+    // soon as O(i) frees a ring B slot.  Per tile the load order is
+    //   K_R(i), A: i.p0, i.p1,  B: i.p2,  A: (i-1).p0', (i-1).p1',  B: i.p3
+    // and the last tile's reloads come after the loop; each load waits only on
+    // MMAs that need no later load of this order.
     ptx::prefetch_tmap(&p.tm_c);
     ptx::prefetch_tmap(&p.tm_k);
     ptx::prefetch_tmap(&p.tm_qc);
     ptx::prefetch_tmap(&p.tm_qr);
-    const uint64_t once = ptx::l2_policy_evict_first();   // every byte is read once
+    const uint64_t keep = ptx::l2_policy_evict_last();    // pairs 0-1: read again from L2
+    const uint64_t once = ptx::l2_policy_evict_first();   // read once
     auto tile_row = [&](int64_t u) -> int32_t {
       return (int32_t)((u / p.tiles_per_seq) * p.L + (u % p.tiles_per_seq) * kT);
     };
-    auto prefetch_tile = [&](int64_t u) {
-      const int32_t row = tile_row(u);
-      ptx::tma_prefetch_l2_2d(&p.tm_k, 0, row);
-      for (int ch = 0; ch < 8; ++ch) ptx::tma_prefetch_l2_2d(&p.tm_c, 64 * ch, row);
-    };
-    for (int64_t u = u0 + 1; u < u0 + kPrefetchAhead && u < u1; ++u) prefetch_tile(u);
-    int issued_c[kNPair], issued_k[kNKr];
+    // last phase issued on each full barrier (-1: none), so that every copy can
+    // be waited for before the CTA exits
+    int issued_as[kNA], issued_ar[kNA], issued_b[kNB], issued_k[kNKr];
 #pragma unroll
-    for (int i = 0; i < kNPair; ++i) issued_c[i] = -1;
+    for (int i = 0; i < kNA; ++i) { issued_as[i] = -1; issued_ar[i] = -1; }
+#pragma unroll
+    for (int i = 0; i < kNB; ++i) issued_b[i] = -1;
 #pragma unroll
     for (int i = 0; i < kNKr; ++i) issued_k[i] = -1;
     int issued_q = -1;
-    int64_t nc = 0, nk = 0;
+    int64_t nb = 0, nk = 0;
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
+    const int64_t T = n_tiles;
+    auto issue = [&](uint64_t* full, int slot, int32_t row, int pr, uint64_t policy) {
+      ptx::mbar_arrive_expect_tx(full, kPairBytes);
+      uint8_t* dst = smem + kOffPair + slot * kPairBytes;
+      ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, full, policy);
+      ptx::tma_load_2d_hint(dst + kChunk, &p.tm_c, 128 * pr + 64, row, full, policy);
+    };
+    // ring A, pair pr of tile i for its scores.  The slot's previous content:
+    // nothing (i = 0), the scores load of tile 0 (i = 1), else the reload of i-2.
+    auto load_scores_a = [&](int64_t i, int32_t row, int pr) -> bool {
+      if (i == 1 && !bounded_wait(&bb.empty_as[pr], 0, abort_flag, p, 0x102, true)) return false;
+      if (i >= 2 && !bounded_wait(&bb.empty_ar[pr], (uint32_t)(i - 2) & 1, abort_flag, p, 0x102, true))
+        return false;
+      issue(&bb.full_as[pr], pr, row, pr, keep);
+#pragma unroll
+      for (int q = 0; q < kNA; ++q) if (q == pr) issued_as[q] = (int)i;
+      return true;
+    };
+    // ring A, pair pr of tile j again for O.  The slot's previous content: the
+    // scores load of tile j+1, or for the last tile the reload of j-1 (the
+    // scores load of tile 0 when it is the only tile).
+    auto load_reload_a = [&](int64_t j, int32_t row, int pr) -> bool {
+      bool w;
+      if (j + 1 < T) w = bounded_wait(&bb.empty_as[pr], (uint32_t)(j + 1) & 1, abort_flag, p, 0x103, true);
+      else if (j >= 1) w = bounded_wait(&bb.empty_ar[pr], (uint32_t)(j - 1) & 1, abort_flag, p, 0x103, true);
+      else w = bounded_wait(&bb.empty_as[pr], 0, abort_flag, p, 0x103, true);
+      if (!w) return false;
+      issue(&bb.full_ar[pr], pr, row, pr, once);
+#pragma unroll
+      for (int q = 0; q < kNA; ++q) if (q == pr) issued_ar[q] = (int)j;
+      return true;
+    };
+    // ring B: the next slot, after O of the tile that held it
+    auto load_b = [&](int32_t row, int pr) -> bool {
+      const int cs = (int)(nb % kNB);
+      const int ck = (int)(nb / kNB);
+      if (ck >= 1 && !bounded_wait(&bb.empty_b[cs], (ck - 1) & 1, abort_flag, p, 0x104, true)) return false;
+      issue(&bb.full_b[cs], kNA + cs, row, pr, once);
+#pragma unroll
+      for (int q = 0; q < kNB; ++q) if (q == cs) issued_b[q] = ck;
+      ++nb;
+      return true;
+    };
     for (int64_t u = u0; u < u1 && ok; ++u) {
       const int64_t b = u / p.tiles_per_seq;
-      if (u + kPrefetchAhead < u1) prefetch_tile(u + kPrefetchAhead);
       if (b != cur_b) {
         cur_b = b;
         ++seg;
@@ -343,39 +408,42 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         }
         ++nk;
       }
-      for (int pr = 0; pr < kPairsPerTile && ok; ++pr) {
-        const int cs = (int)(nc % kNPair);
-        const int ck = (int)(nc / kNPair);
-        if (ck >= 1) ok = bounded_wait(&bb.empty_c[cs], (ck - 1) & 1, abort_flag, p, 0x102, true);
-        if (!ok) break;
-        ptx::mbar_arrive_expect_tx(&bb.full_c[cs], kPairBytes);
-        uint8_t* dst = smem + kOffPair + cs * kPairBytes;
-        ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, &bb.full_c[cs], once);
-        ptx::tma_load_2d_hint(dst + kChunk, &p.tm_c, 128 * pr + 64, row, &bb.full_c[cs], once);
-#pragma unroll
-        for (int q = 0; q < kNPair; ++q) if (q == cs) issued_c[q] = ck;
-        ++nc;
+      const int64_t i = u - u0;
+      ok = load_scores_a(i, row, 0) && load_scores_a(i, row, 1) && load_b(row, 2);
+      if (ok && i >= 1) {
+        const int32_t prev = tile_row(u - 1);
+        ok = load_reload_a(i - 1, prev, 0) && load_reload_a(i - 1, prev, 1);
       }
+      if (ok) ok = load_b(row, 3);
+    }
+    if (ok && T > 0) {
+      const int32_t last = tile_row(u1 - 1);
+      if (load_reload_a(T - 1, last, 0)) load_reload_a(T - 1, last, 1);
     }
     // Let every copy this thread started land before the CTA can exit.
 #pragma unroll
-    for (int i = 0; i < kNPair; ++i)
-      if (issued_c[i] >= 0) bounded_wait(&bb.full_c[i], issued_c[i] & 1, abort_flag, p, 0x1F0, false);
+    for (int i = 0; i < kNA; ++i) {
+      if (issued_as[i] >= 0) bounded_wait(&bb.full_as[i], issued_as[i] & 1, abort_flag, p, 0x1F0, false);
+      if (issued_ar[i] >= 0) bounded_wait(&bb.full_ar[i], issued_ar[i] & 1, abort_flag, p, 0x1F0, false);
+    }
+#pragma unroll
+    for (int i = 0; i < kNB; ++i)
+      if (issued_b[i] >= 0) bounded_wait(&bb.full_b[i], issued_b[i] & 1, abort_flag, p, 0x1F0, false);
 #pragma unroll
     for (int i = 0; i < kNKr; ++i)
       if (issued_k[i] >= 0) bounded_wait(&bb.full_k[i], issued_k[i] & 1, abort_flag, p, 0x1F1, false);
     if (issued_q >= 0) bounded_wait(bb.q_full, issued_q & 1, abort_flag, p, 0x1F2, false);
   } else if (warp == 1 && lane == 0) {
     // ===================================================== score MMA issuer
-    // Pair n (tile n / 4, column pair n % 4) once it has landed; the first pair
-    // of a tile also waits for that tile's K_R (sr goes first), for its S buffer
-    // to be released and, for a new sequence part, for the query block.
+    // Tile t: K_R (sr first), then column pairs 0-1 from ring A (each slot
+    // released after its MMAs) and 2-3 from ring B (held for O), each once it
+    // has landed; also waits for the S buffer to be released and, for a new
+    // sequence part, for the query block.
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kT, kHC, 0, 0);   // K-major A and B
     // Descriptor templates; a K step adds (bytes >> 4) to the start-address field.
     const uint64_t d_pair = ptx::smem_desc(ptx::smem_u32(smem + kOffPair), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_kr = ptx::smem_desc(ptx::smem_u32(smem + kOffKr), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_q = ptx::smem_desc(ptx::smem_u32(smem + kOffQ), 16, 1024, ptx::kSwizzle128B);
-    int64_t nc = 0;
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
@@ -403,12 +471,15 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
                            d_q + (uint64_t)((8 * kQChunk + 32 * k) >> 4), kIdescS, k > 0);
         ptx::mma_commit(&bb.empty_k[t % kNKr]);
       }
-      for (int pr = 0; pr < kPairsPerTile; ++pr, ++nc) {   // sc += C_KV[:, pair] . q_c[pair]^T
-        ok = bounded_wait(&bb.full_c[nc % kNPair], (uint32_t)(nc / kNPair) & 1, abort_flag, p, 0x203, true);
+      for (int pr = 0; pr < kPairsPerTile; ++pr) {   // sc += C_KV[:, pair] . q_c[pair]^T
+        const int64_t n = 2 * t + (pr - 2);           // ring B index of pairs 2-3
+        const int cs = pr < 2 ? pr : kNA + (int)(n % kNB);   // shared-memory slot
+        ok = pr < 2 ? bounded_wait(&bb.full_as[pr], (uint32_t)t & 1, abort_flag, p, 0x203, true)
+                    : bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x203, true);
         if (!ok) break;
         ptx::tc_fence_after();
         const uint32_t d_sc = tmem + kColS + 32 * buf;
-        const uint64_t a0 = d_pair + (uint64_t)(((nc % kNPair) * kPairBytes) >> 4);
+        const uint64_t a0 = d_pair + (uint64_t)((cs * kPairBytes) >> 4);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
@@ -417,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
                              d_q + (uint64_t)(((2 * pr + ch) * kQChunk + 32 * k) >> 4), kIdescS,
                              (pr | ch | k) != 0);
         }
+        if (pr < 2) ptx::mma_commit(&bb.empty_as[pr]);   // ring A: read again later from L2
       }
       if (!ok) break;
       ptx::mma_commit(&bb.s_full[buf]);
@@ -427,9 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     bounded_wait(&bb.drain[0], 0, abort_flag, p, 0x2F0, false);
   } else if (warp == kOWarp && lane == 0) {
     // ===================================================== O MMA issuer
-    // Tile j once its P is written: O^T += C^T P^T over its four pairs (still in
-    // their ring slots), releasing each slot after; a sequence part starts the
-    // accumulator afresh.
+    // Tile j once its P is written: O^T += C^T P^T over pairs 2-3 (held in ring
+    // B) and pairs 0-1 (loaded again into ring A), releasing each slot after;
+    // a sequence part starts the accumulator afresh.
     constexpr uint32_t kIdescP = ptx::idesc_bf16_f32(128, kHC, 1, 1);  // MN-major A and B
     // A = C^T, M = 128 latent dims (two 64-dim atoms 16 KB apart), K = 16 tokens
     const uint64_t d_ct = ptx::smem_desc(ptx::smem_u32(smem + kOffPair), kChunk, 1024, ptx::kSwizzle128B);
@@ -442,16 +514,22 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       const int64_t uj = u0 + j;
       const uint32_t acc0 = uj > seg_start(uj) ? 1u : 0u;
       const uint64_t bpt = d_pt + (uint64_t)((buf * kPBytes) >> 4);
-#pragma unroll
-      for (int m = 0; m < kPairsPerTile; ++m) {
-        const int cs = (int)((j * kPairsPerTile + m) % kNPair);
+#pragma unroll 1
+      for (int mm = 0; mm < kPairsPerTile; ++mm) {
+        const int m = (mm + 2) & 3;                 // pairs 2, 3 (ring B) first, then 0, 1
+        const int64_t n = 2 * j + (m - 2);            // ring B index of pairs 2-3
+        const int cs = m >= 2 ? kNA + (int)(n % kNB) : m;    // shared-memory slot
+        const bool okw = m >= 2 ? bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x206, true)
+                                : bounded_wait(&bb.full_ar[m], (uint32_t)j & 1, abort_flag, p, 0x206, true);
+        if (!okw) break;
+        ptx::tc_fence_after();
         const uint32_t d_o = tmem + kColO + 16 * m;
         const uint64_t act = d_ct + (uint64_t)((cs * kPairBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           ptx::mma_bf16_ss(d_o, act + (uint64_t)(kk * (2048 >> 4)),
                            bpt + (uint64_t)(kk * (256 >> 4)), kIdescP, kk > 0 ? 1u : acc0);
-        ptx::mma_commit(&bb.empty_c[cs]);
+        ptx::mma_commit(m >= 2 ? &bb.empty_b[cs - kNA] : &bb.empty_ar[m]);
       }
       ptx::mma_commit(&bb.o_full[buf]);
     }
