@@ -25,18 +25,20 @@
 // The range's partial (M, Z, O) goes to the workspace; the combine kernel
 // merges the ranges of a sequence.
 //
-// Each C_KV tile is read from HBM once: its four 128-dim column pairs stay in
-// a ring of five 32 KB shared-memory slots from their load until O^T += C^T P^T
-// has used them.  Two threads issue MMAs, so that the scores of tile i+1 (as
-// their pairs land) and O of tile i (once its P is written) overlap.
+// Each C_KV byte is read from HBM once.  Of a tile's four 128-dim column
+// pairs, pair 3 stays in shared memory from its load until O^T += C^T P^T has
+// used it; pairs 0-2 are loaded for the scores and loaded again, from L2, for
+// O.  So the scores of tile i+1 complete while the softmax of tile i runs.
+// Two threads issue MMAs: the scores of a tile as its pairs land, O of a tile
+// once its P is written.
 //
-// Roles (352 threads): warp 0 lane 0 issues TMA loads and L2 prefetches; warp
-// 1 allocates TMEM and its lane 0 issues the score MMAs; warps 2-9 (256
-// threads) do the softmax, two warps per TMEM lane quarter, each owning 8 of
-// the 16 heads; warp 10 lane 0 issues the O MMAs.
-// Shared memory: the pair ring ([128 tokens][2 x 64 dims] per slot, 128-byte
-// swizzle), two K_R slots, the query block (9 x [16 heads][64 dims]) and two
-// P buffers.
+// Roles (352 threads): warp 0 lane 0 issues TMA loads; warp 1 allocates TMEM
+// and its lane 0 issues the score MMAs; warps 2-9 (256 threads) do the
+// softmax, two warps per TMEM lane quarter, each owning 8 of the 16 heads;
+// warp 10 lane 0 issues the O MMAs.
+// Shared memory: five column-pair slots ([128 tokens][2 x 64 dims] each,
+// 128-byte swizzle), two K_R slots, the query block (9 x [16 heads][64 dims])
+// and two P buffers.
 // Every mbarrier wait is bounded; when a bound runs out the CTA records the
 // error, stops issuing work, waits for its own copies and MMAs in flight,
 // frees TMEM and exits.
@@ -58,9 +60,11 @@ constexpr int kDR = 64;                    // RoPE key width
 constexpr int kChunk = kT * 128;           // [128 rows][64 bf16] = 16 KB
 constexpr int kPairBytes = 2 * kChunk;     // two 64-dim chunks = 128 latent dims
 constexpr int kPairsPerTile = kDC / 128;
-constexpr int kNPair = 5;                  // C_KV pair slots: ring A (2) then ring B (3)
-constexpr int kNA = 2;                     // ring A: column pairs 0-1, streamed
-constexpr int kNB = kNPair - kNA;          // ring B: column pairs 2-3, held until O
+constexpr int kNPair = 5;                  // C_KV pair slots: ring A then ring B
+constexpr int kNA = 3;                     // ring A: column pairs 0-2 (one slot each), streamed
+constexpr int kHeld = kPairsPerTile - kNA; // pairs per tile held in ring B until O
+constexpr int kNB = kNPair - kNA;          // ring B slots: the held pairs of two tiles
+static_assert(kNB == 2 * kHeld, "ring B holds the held pairs of two tiles");
 constexpr int kNKr = 2;                    // K_R slots
 constexpr int kQChunk = kHC * 128;         // [16 heads][64 bf16] = 2 KB
 constexpr int kQBytes = 9 * kQChunk;       // 8 chunks of q_c, 1 of q_r
@@ -264,13 +268,12 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   const int64_t u1 = (c + 1) * p.U / p.G;
   const int64_t n_tiles = u1 - u0;
   const int64_t win0 = p.nG * g;
-  // first tile of the part of tile u's sequence that lies in this CTA's range
-  auto seg_start = [&](int64_t u) -> int64_t {
-    const int64_t s0 = (u / p.tiles_per_seq) * p.tiles_per_seq;
-    return s0 > u0 ? s0 : u0;
-  };
-  auto last_in_seg = [&](int64_t u) -> bool {
-    return (u + 1 == u1) || ((u + 1) / p.tiles_per_seq != u / p.tiles_per_seq);
+  // (sequence, tile within it) of the range's first tile; each role then steps
+  // its own copy once per tile rather than dividing
+  const int64_t seq0 = u0 / p.tiles_per_seq;
+  const int64_t tile0 = u0 - seq0 * p.tiles_per_seq;
+  auto step = [&](int64_t& seq, int64_t& tile) {
+    if (++tile == p.tiles_per_seq) { tile = 0; ++seq; }
   };
 
   if (tid == 0) {
@@ -304,14 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ===================================================== TMA producer
-    // Two rings of 32 KB column-pair slots.  Ring B (3 slots) holds pairs 2-3
-    // of a tile from their load until O += C^T P^T of that tile.  Ring A (2
-    // slots) streams pairs 0-1: once for the scores (kept in L2 with an
-    // evict-last hint) and once more, read back from L2, for O.  So during the
-    // softmax of tile i, the scores of tile i+1 run on its pairs 0-2 and the
-    // pairs 0-1 of tile i come back for O(i); pair 3 of tile i+1 follows as
-    // soon as O(i) frees a ring B slot.  Per tile the load order is
-    //   K_R(i), A: i.p0, i.p1,  B: i.p2,  A: (i-1).p0', (i-1).p1',  B: i.p3
+    // Two rings of 32 KB column-pair slots.  Ring B (two slots) holds pair 3 of
+    // a tile from its load until O += C^T P^T of that tile, for two tiles at a
+    // time.  Ring A (one slot per pair 0-2) streams each of those pairs twice:
+    // once for the scores (kept in L2 with an evict-last hint) and once more,
+    // read back from L2, for O.  So the scores of tile i+1 complete while the
+    // softmax of tile i runs, and the softmaxes follow each other directly.
+    // Per tile the load order is
+    //   K_R(i), A: i.p0, i.p1, i.p2,  B: i.p3,  A: (i-1).p0', p1', p2'
     // and the last tile's reloads come after the loop; each load waits only on
     // MMAs that need no later load of this order.
     ptx::prefetch_tmap(&p.tm_c);
@@ -320,9 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     ptx::prefetch_tmap(&p.tm_qr);
     const uint64_t keep = ptx::l2_policy_evict_last();    // pairs 0-1: read again from L2
     const uint64_t once = ptx::l2_policy_evict_first();   // read once
-    auto tile_row = [&](int64_t u) -> int32_t {
-      return (int32_t)((u / p.tiles_per_seq) * p.L + (u % p.tiles_per_seq) * kT);
-    };
     // last phase issued on each full barrier (-1: none), so that every copy can
     // be waited for before the CTA exits
     int issued_as[kNA], issued_ar[kNA], issued_b[kNB], issued_k[kNKr];
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, full, policy);
       ptx::tma_load_2d_hint(dst + kChunk, &p.tm_c, 128 * pr + 64, row, full, policy);
     };
-    // ring A, pair pr of tile i for its scores.  The slot's previous content:
+    // ring A, pair pr (slot pr) of tile i for its scores.  The slot's previous content:
     // nothing (i = 0), the scores load of tile 0 (i = 1), else the reload of i-2.
     auto load_scores_a = [&](int64_t i, int32_t row, int pr) -> bool {
       if (i == 1 && !bounded_wait(&bb.empty_as[pr], 0, abort_flag, p, 0x102, true)) return false;
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       for (int q = 0; q < kNA; ++q) if (q == pr) issued_ar[q] = (int)j;
       return true;
     };
-    // ring B: the next slot, after O of the tile that held it
+    // ring B: the next slot, after O of the tile two back that held it
     auto load_b = [&](int32_t row, int pr) -> bool {
       const int cs = (int)(nb % kNB);
       const int ck = (int)(nb / kNB);
@@ -380,8 +380,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       ++nb;
       return true;
     };
-    for (int64_t u = u0; u < u1 && ok; ++u) {
-      const int64_t b = u / p.tiles_per_seq;
+    int64_t pseq = seq0, ptile = tile0;
+    int32_t prev_row = 0;             // first row of the previous tile
+    for (int64_t u = u0; u < u1 && ok; ++u, step(pseq, ptile)) {
+      const int64_t b = pseq;
       if (b != cur_b) {
         cur_b = b;
         ++seg;
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         ptx::tma_load_2d(smem + kOffQ + 8 * kQChunk, &p.tm_qr, 0, qrow, bb.q_full);
         issued_q = seg;
       }
-      const int32_t row = tile_row(u);
+      const int32_t row = (int32_t)(b * p.L + ptile * kT);
       {
         const int ks = (int)(nk % kNKr);
         const int kk = (int)(nk / kNKr);
@@ -409,17 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         ++nk;
       }
       const int64_t i = u - u0;
-      ok = load_scores_a(i, row, 0) && load_scores_a(i, row, 1) && load_b(row, 2);
-      if (ok && i >= 1) {
-        const int32_t prev = tile_row(u - 1);
-        ok = load_reload_a(i - 1, prev, 0) && load_reload_a(i - 1, prev, 1);
-      }
-      if (ok) ok = load_b(row, 3);
+      for (int pr = 0; pr < kNA && ok; ++pr) ok = load_scores_a(i, row, pr);
+      for (int pr = kNA; pr < kPairsPerTile && ok; ++pr) ok = load_b(row, pr);
+      for (int pr = 0; pr < kNA && ok && i >= 1; ++pr) ok = load_reload_a(i - 1, prev_row, pr);
+      prev_row = row;
     }
-    if (ok && T > 0) {
-      const int32_t last = tile_row(u1 - 1);
-      if (load_reload_a(T - 1, last, 0)) load_reload_a(T - 1, last, 1);
-    }
+    for (int pr = 0; pr < kNA && ok && T > 0; ++pr) ok = load_reload_a(T - 1, prev_row, pr);   // the last tile
     // Let every copy this thread started land before the CTA can exit.
 #pragma unroll
     for (int i = 0; i < kNA; ++i) {
@@ -435,9 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     if (issued_q >= 0) bounded_wait(bb.q_full, issued_q & 1, abort_flag, p, 0x1F2, false);
   } else if (warp == 1 && lane == 0) {
     // ===================================================== score MMA issuer
-    // Tile t: K_R (sr first), then column pairs 0-1 from ring A (each slot
-    // released after its MMAs) and 2-3 from ring B (held for O), each once it
-    // has landed; also waits for the S buffer to be released and, for a new
+    // Tile t: K_R (sr first), then column pairs 0-2 from ring A (each slot
+    // released after its MMAs) and pair 3 from ring B (held for O), each once
+    // it has landed; also waits for the S buffer to be released and, for a new
     // sequence part, for the query block.
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kT, kHC, 0, 0);   // K-major A and B
     // Descriptor templates; a K step adds (bytes >> 4) to the start-address field.
@@ -447,9 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
-    for (int64_t t = 0; t < n_tiles && ok; ++t) {
-      const int64_t u = u0 + t;
-      const int64_t b = u / p.tiles_per_seq;
+    int64_t sseq = seq0, stile = tile0;
+    for (int64_t t = 0; t < n_tiles && ok; ++t, step(sseq, stile)) {
+      const int64_t b = sseq;
+      const bool last_in_seg = t + 1 == n_tiles || stile + 1 == p.tiles_per_seq;
       const int buf = (int)(t & 1);
       if (b != cur_b) {
         cur_b = b;
@@ -472,10 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         ptx::mma_commit(&bb.empty_k[t % kNKr]);
       }
       for (int pr = 0; pr < kPairsPerTile; ++pr) {   // sc += C_KV[:, pair] . q_c[pair]^T
-        const int64_t n = 2 * t + (pr - 2);           // ring B index of pairs 2-3
-        const int cs = pr < 2 ? pr : kNA + (int)(n % kNB);   // shared-memory slot
-        ok = pr < 2 ? bounded_wait(&bb.full_as[pr], (uint32_t)t & 1, abort_flag, p, 0x203, true)
-                    : bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x203, true);
+        const int64_t n = kHeld * t + (pr - kNA);     // ring B index of a held pair
+        const int cs = pr < kNA ? pr : kNA + (int)(n % kNB);   // shared-memory slot
+        ok = pr < kNA ? bounded_wait(&bb.full_as[pr], (uint32_t)t & 1, abort_flag, p, 0x203, true)
+                      : bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x203, true);
         if (!ok) break;
         ptx::tc_fence_after();
         const uint32_t d_sc = tmem + kColS + 32 * buf;
@@ -488,39 +486,39 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
                              d_q + (uint64_t)(((2 * pr + ch) * kQChunk + 32 * k) >> 4), kIdescS,
                              (pr | ch | k) != 0);
         }
-        if (pr < 2) ptx::mma_commit(&bb.empty_as[pr]);   // ring A: read again later from L2
+        if (pr < kNA) ptx::mma_commit(&bb.empty_as[pr]);   // ring A: read again later from L2
       }
       if (!ok) break;
       ptx::mma_commit(&bb.s_full[buf]);
-      if (last_in_seg(u)) ptx::mma_commit(bb.q_empty);
+      if (last_in_seg) ptx::mma_commit(bb.q_empty);
     }
     // Every MMA issued here must finish before TMEM is freed.
     ptx::mma_commit(&bb.drain[0]);
     bounded_wait(&bb.drain[0], 0, abort_flag, p, 0x2F0, false);
   } else if (warp == kOWarp && lane == 0) {
     // ===================================================== O MMA issuer
-    // Tile j once its P is written: O^T += C^T P^T over pairs 2-3 (held in ring
-    // B) and pairs 0-1 (loaded again into ring A), releasing each slot after;
-    // a sequence part starts the accumulator afresh.
+    // Tile j once its P is written: O^T += C^T P^T over pair 3 (held in ring B)
+    // and pairs 0-2 (loaded again into ring A), releasing each slot after; a
+    // sequence part starts the accumulator afresh.
     constexpr uint32_t kIdescP = ptx::idesc_bf16_f32(128, kHC, 1, 1);  // MN-major A and B
     // A = C^T, M = 128 latent dims (two 64-dim atoms 16 KB apart), K = 16 tokens
     const uint64_t d_ct = ptx::smem_desc(ptx::smem_u32(smem + kOffPair), kChunk, 1024, ptx::kSwizzle128B);
     // B = P^T, N = 16 heads (8-head core blocks 2 KB apart), K = 16 tokens
     const uint64_t d_pt = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 128, 2048, ptx::kSwizzleNone);
-    for (int64_t j = 0; j < n_tiles; ++j) {
+    int64_t oseq = seq0, otile = tile0;
+    for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile)) {
       const int buf = (int)(j & 1);
       if (!bounded_wait(&bb.p_full[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x204, true)) break;
       ptx::tc_fence_after();
-      const int64_t uj = u0 + j;
-      const uint32_t acc0 = uj > seg_start(uj) ? 1u : 0u;
+      const uint32_t acc0 = (j > 0 && otile > 0) ? 1u : 0u;   // a sequence part starts afresh
       const uint64_t bpt = d_pt + (uint64_t)((buf * kPBytes) >> 4);
 #pragma unroll 1
       for (int mm = 0; mm < kPairsPerTile; ++mm) {
-        const int m = (mm + 2) & 3;                 // pairs 2, 3 (ring B) first, then 0, 1
-        const int64_t n = 2 * j + (m - 2);            // ring B index of pairs 2-3
-        const int cs = m >= 2 ? kNA + (int)(n % kNB) : m;    // shared-memory slot
-        const bool okw = m >= 2 ? bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x206, true)
-                                : bounded_wait(&bb.full_ar[m], (uint32_t)j & 1, abort_flag, p, 0x206, true);
+        const int m = (mm + kNA) % kPairsPerTile;   // held pairs (ring B) first, then the reloads
+        const int64_t n = kHeld * j + (m - kNA);      // ring B index of a held pair
+        const int cs = m >= kNA ? kNA + (int)(n % kNB) : m;  // shared-memory slot
+        const bool okw = m >= kNA ? bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x206, true)
+                                  : bounded_wait(&bb.full_ar[m], (uint32_t)j & 1, abort_flag, p, 0x206, true);
         if (!okw) break;
         ptx::tc_fence_after();
         const uint32_t d_o = tmem + kColO + 16 * m;
@@ -529,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         for (int kk = 0; kk < 8; ++kk)
           ptx::mma_bf16_ss(d_o, act + (uint64_t)(kk * (2048 >> 4)),
                            bpt + (uint64_t)(kk * (256 >> 4)), kIdescP, kk > 0 ? 1u : acc0);
-        ptx::mma_commit(m >= 2 ? &bb.empty_b[cs - kNA] : &bb.empty_ar[m]);
+        ptx::mma_commit(m >= kNA ? &bb.empty_b[cs - kNA] : &bb.empty_ar[m]);
       }
       ptx::mma_commit(&bb.o_full[buf]);
     }
@@ -554,9 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 #pragma unroll
     for (int h = 0; h < kHH; ++h) { Zt[h] = 0.f; Mh[h] = -INFINITY; }
 
-    for (int64_t i = 0; i < n_tiles; ++i) {
-      const int64_t u = u0 + i;
-      const int64_t b = u / p.tiles_per_seq, tile = u % p.tiles_per_seq;
+    int64_t cseq = seq0, ctile = tile0;
+    for (int64_t i = 0; i < n_tiles; ++i, step(cseq, ctile)) {
+      const int64_t b = cseq, tile = ctile;
+      const bool last_in_seg = i + 1 == n_tiles || tile + 1 == p.tiles_per_seq;
       const int buf = (int)(i & 1);
       const int kb = (int)(i >> 1);
       warp_wait(&bb.s_full[buf], kb & 1, abort_flag, p, 0x300);
@@ -642,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       // to the tile's largest entry; later it rises only when an entry exceeds
       // it by more than 2^8, and then Z and O^T are rescaled.  The checkpoint
       // barrier ORs "abort, or take this slow path" over the softmax threads.
-      const bool first = u == seg_start(u);
+      const bool first = i == 0 || tile == 0;
       bool need = first;
 #pragma unroll
       for (int h = 0; h < kHH; ++h) need = need || (ent[h] - Mh[h]) * kLog2e > kRescaleLog2;
@@ -716,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bb.p_full[buf]);
 
-      if (last_in_seg(u)) {
+      if (last_in_seg) {
         // the partial of the range's part of sequence b
         const int64_t slot = b + c;
         warp_wait(&bb.o_full[buf], (uint32_t)kb & 1, abort_flag, p, 0x304);
