@@ -10,7 +10,6 @@
 namespace lca {
 
 constexpr int kCombineThreads = 128;
-constexpr int kCombineMaxParts = 1024;   // per (sequence, head); the plan keeps far fewer
 
 struct CombineParams {
   const float* part_o;   // [slots][H][d_c]
@@ -33,12 +32,18 @@ __device__ __forceinline__ int64_t range_owner(int64_t u, int64_t U, int64_t G) 
   return ((u + 1) * G - 1) / U;  // largest c with floor(c*U/G) <= u
 }
 
-// Grid: (H, B, d_c / kCombineThreads); one thread per latent dimension.
+// Grid: (H, B, d_c / kCombineThreads); one thread per latent dimension.  One
+// pass over the partials, kChunk at a time: every (M_i, Z_i) and O_i[d] of a
+// chunk is loaded at once, then merged online -- the running max rises to the
+// chunk's and the sums are rescaled -- so the kernel waits for memory about
+// once per chunk.  Each thread forms Z itself (a few exponentials) instead of
+// sharing it through a block reduction.
 __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const CombineParams p) {
-  __shared__ float scale[kCombineMaxParts];
-  __shared__ float red[kCombineThreads / 32];
+  constexpr int kChunk = 16;
   if (p.wait_prior) ptx::griddep_wait();
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int d = blockIdx.z * kCombineThreads + threadIdx.x;
+  if (d >= p.d_c) return;
   int64_t first, count;
   if (p.mode == 0) {
     first = (int64_t)b * p.n_split;
@@ -50,52 +55,40 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     first = b + c0;
     count = c1 - c0 + 1;
   }
-  if (count > kCombineMaxParts) count = kCombineMaxParts;  // the host never plans more
-  // M = max_i M_i (partials read in parallel)
-  float m = -INFINITY;
-  for (int64_t i = tid; i < count; i += kCombineThreads)
-    m = fmaxf(m, p.part_mz[((first + i) * p.H + h) * 2]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((tid & 31) == 0) red[tid >> 5] = m;
-  __syncthreads();
-  float M = red[0];
-#pragma unroll
-  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, red[w]);
-  __syncthreads();
-  // factors e^{M_i - M} and Z = sum_i e^{M_i - M} Z_i
-  float z = 0.f;
-  for (int64_t i = tid; i < count; i += kCombineThreads) {
-    const float* mz = p.part_mz + ((first + i) * p.H + h) * 2;
-    const float f = expf(mz[0] - M);
-    scale[i] = f;
-    z = fmaf(f, mz[1], z);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-  if ((tid & 31) == 0) red[tid >> 5] = z;
-  __syncthreads();
-  float Z = 0.f;
-#pragma unroll
-  for (int w = 0; w < kCombineThreads / 32; ++w) Z += red[w];
-  const float invZ = 1.f / Z;
-  // out[d] = sum_i f_i O_i[d] / Z with eight loads in flight
-  const int d = blockIdx.z * kCombineThreads + tid;
-  if (d >= p.d_c) return;
   const int64_t stride = (int64_t)p.H * p.d_c;
   const float* po = p.part_o + (first * p.H + h) * (int64_t)p.d_c + d;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int64_t i = 0;
-  for (; i + 8 <= count; i += 8) {
-    float v[8];
+  const float2* pmz = reinterpret_cast<const float2*>(p.part_mz) + first * p.H + h;
+  float M = -INFINITY, Z = 0.f, acc = 0.f;
+  for (int64_t i0 = 0; i0 < count; i0 += kChunk) {
+    const int n = (int)(count - i0 < kChunk ? count - i0 : kChunk);
+    float2 mz[kChunk];
+    float o[kChunk];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = po[(i + k) * stride];
+    for (int k = 0; k < kChunk; ++k) {
+      if (k < n) {
+        mz[k] = pmz[(i0 + k) * p.H];
+        o[k] = po[(i0 + k) * stride];
+      } else {
+        mz[k] = make_float2(-INFINITY, 0.f);
+        o[k] = 0.f;
+      }
+    }
+    float mc = M;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = fmaf(scale[i + k], v[k], acc[k]);
+    for (int k = 0; k < kChunk; ++k) mc = fmaxf(mc, mz[k].x);
+    if (mc == -INFINITY) continue;            // only empty partials so far
+    const float f = expf(M - mc);             // 0 while M is still -inf
+    Z *= f;
+    acc *= f;
+#pragma unroll
+    for (int k = 0; k < kChunk; ++k) {
+      const float w = expf(mz[k].x - mc);      // 0 for an empty partial (M_i = -inf)
+      Z = fmaf(w, mz[k].y, Z);
+      acc = fmaf(w, o[k], acc);
+    }
+    M = mc;
   }
-  for (; i < count; ++i) acc[0] = fmaf(scale[i], po[i * stride], acc[0]);
-  const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-  p.out[((int64_t)b * p.H + h) * p.d_c + d] = sum * invZ;
+  p.out[((int64_t)b * p.H + h) * p.d_c + d] = acc / Z;
 }
 
 }  // namespace lca
