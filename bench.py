@@ -90,8 +90,79 @@ def profiled_traffic() -> int | None:
         return None
 
 
+class NvmlSampler:
+    """Samples SM clock, power and clock-event reasons of one GPU through NVML
+    every few milliseconds from a host thread (read-only queries), so that a
+    timed region of a few tens of milliseconds still holds samples."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
+
+    def __init__(self, gpu_uuid: str | None, interval_s: float = 0.002):
+        import threading
+        self.samples: list[tuple[float, float, int]] = []
+        self.sm_max = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = (pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid) if gpu_uuid
+                      else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception:  # noqa: BLE001 - no NVML: report no samples
+            return
+        self.interval = interval_s
+        self.stop_evt = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _one(self) -> None:
+        n = self.nvml
+        sm = float(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+        pw = n.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        self.samples.append((sm, pw, int(rs)))
+
+    def _run(self) -> None:
+        while True:
+            try:
+                self._one()
+            except Exception:  # noqa: BLE001
+                return
+            if self.stop_evt.wait(self.interval):
+                return
+
+    def start(self) -> None:
+        if self.ok:
+            self.thread.start()
+
+    def stop(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "none"}
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        try:
+            self._one()                      # one sample at the end of the region
+        except Exception:  # noqa: BLE001
+            pass
+        reasons = set()
+        for name, attr, bit in self.REASONS:
+            mask = getattr(self.nvml, attr, bit)
+            if any(r & mask for _, _, r in self.samples):
+                reasons.add(name)
+        sm = [s for s, _, _ in self.samples]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": statistics.median([p for _, p, _ in self.samples]) if sm else None,
+                "source": f"NVML every {self.interval * 1e3:.0f} ms over the timed region"}
+
+
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of one GPU while the benchmark runs."""
+    """nvidia-smi samples (200 ms) of one GPU over the whole run, a cross-check
+    of the NVML samples taken over the timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -227,42 +298,65 @@ def our_arm(args) -> None:
         q_c, q_r, c_kv, k_r = dev[k % copies]
         plan.decode(q_c, q_r, c_kv, k_r, wl.L, wl.g, wl.w, out, anc if nG > 0 else None, stream)
 
-    sampler = ClockSampler(getattr(torch.cuda.get_device_properties(local), "uuid", None)
-                           and "GPU-" + str(torch.cuda.get_device_properties(local).uuid))
+    props = torch.cuda.get_device_properties(local)
+    uuid = ("GPU-" + str(props.uuid)) if getattr(props, "uuid", None) else None
+    sampler = ClockSampler(uuid)
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize()
     assert plan.device_error() == kvc.LCA_OK
 
     K = args.steps
+
+    def barrier_sync() -> None:
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # Timed region: K back-to-back steps exactly as a caller issues them (no event
+    # between the main and the combine kernel, so the combine's programmatic
+    # dependent launch overlaps the main kernel's tail).
+    e_begin = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    nvml = NvmlSampler(uuid)
+    barrier_sync()
+    nvml.start()
+    e_begin.record(stream)
+    for k in range(K):
+        step(k)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = nvml.stop()
+    if dist is not None:
+        dist.barrier()
+    t_total = max_over_ranks(e_begin.elapsed_time(e_end) * 1e-3)
+    assert plan.device_error() == kvc.LCA_OK
+
+    # Second pass of K steps for the main kernel's own duration: an event recorded
+    # on the launching stream right after each main-kernel launch.
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     for e in ev_m:          # create the events so their handles exist
         e.record(stream)
-    torch.cuda.synchronize()
-    e_begin = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e_begin.record(stream)
+    barrier_sync()
     for k in range(K):
         ev_s[k].record(stream)
         plan.set_timing_event(ev_m[k])
         step(k)
-    e_end.record(stream)
     torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
     plan.set_timing_event(None)
-    t_total = e_begin.elapsed_time(e_end) * 1e-3
-    t_main = statistics.mean(ev_s[k].elapsed_time(ev_m[k]) for k in range(K)) * 1e-3
+    main_ms = [ev_s[k].elapsed_time(ev_m[k]) for k in range(K)]
+    t_main = max_over_ranks(statistics.mean(main_ms) * 1e-3)
     assert plan.device_error() == kvc.LCA_OK
-    if dist is not None:
-        t = torch.tensor([t_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_total = float(t.item())
-    clocks = sampler.stop()
+    clocks["nvidia_smi_whole_run"] = sampler.stop()
 
     tokens_per_step = world * wl.B * wl.L
     value = tokens_per_step * K / t_total
@@ -330,6 +424,9 @@ def our_arm(args) -> None:
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "kernel": "lca_tc_kernel" if kernel == "tcgen05" else "lca_simt_kernel",
                      "algorithmic_bytes_per_launch": alg, "launch_ms": t_main * 1e3,
+                     "launch_ms_min": min(main_ms), "launch_ms_max": max(main_ms),
+                     "timing": "CUDA events on the launching stream around each main-kernel launch, "
+                               "mean over a second pass of K steps",
                      "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -342,7 +439,7 @@ def our_arm(args) -> None:
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v2lite", choices=sorted(workloads.WORKLOADS))

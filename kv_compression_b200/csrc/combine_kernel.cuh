@@ -41,6 +41,9 @@ __device__ __forceinline__ int64_t range_owner(int64_t u, int64_t U, int64_t G) 
 __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const CombineParams p) {
   constexpr int kChunk = 16;
   if (p.wait_prior) ptx::griddep_wait();
+  // The next step's main kernel may start its prologue now; it waits for this
+  // grid to complete before touching global memory.
+  ptx::griddep_launch_dependents();
   const int h = blockIdx.x, b = blockIdx.y;
   const int d = blockIdx.z * kCombineThreads + threadIdx.x;
   if (d >= p.d_c) return;

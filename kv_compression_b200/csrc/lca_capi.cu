@@ -164,8 +164,20 @@ cudaError_t launch_tc(const lca::tc::TcParams& tp, unsigned grid, cudaStream_t s
     if (e != cudaSuccess) return e;
     configured_device = device;
   }
-  lca::tc::lca_tc_kernel<LOG2G><<<grid, lca::tc::kThreads, lca::tc::kSmemAlloc, stream>>>(tp);
-  return cudaGetLastError();
+  // Programmatic stream serialization: the kernel's prologue (barrier init,
+  // TMEM allocation) may overlap the previous kernel's tail; the kernel waits on
+  // griddepcontrol before its first global access.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(lca::tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = lca::tc::kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, lca::tc::lca_tc_kernel<LOG2G>, tp);
 }
 
 cudaError_t launch_tc_g(int g, const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream,

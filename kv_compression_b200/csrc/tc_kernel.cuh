@@ -304,6 +304,12 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched as a programmatic dependent: the prologue above may overlap the end
+  // of the previous kernel in the stream, and nothing below reads or writes
+  // global memory before that kernel has completed and its writes are visible.
+  // The combine that follows may be scheduled from here on; it waits the same way.
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     // ===================================================== TMA producer
@@ -321,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     ptx::prefetch_tmap(&p.tm_k);
     ptx::prefetch_tmap(&p.tm_qc);
     ptx::prefetch_tmap(&p.tm_qr);
-    const uint64_t keep = ptx::l2_policy_evict_last();    // pairs 0-1: read again from L2
+    const uint64_t keep = ptx::l2_policy_evict_last();    // pairs 0-2: read again from L2
     const uint64_t once = ptx::l2_policy_evict_first();   // read once
     // last phase issued on each full barrier (-1: none), so that every copy can
     // be waited for before the CTA exits
