@@ -266,6 +266,33 @@ def reference_arm(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def rank_workload(wl: workloads.Workload, rank: int) -> workloads.Workload:
+    """Each rank decodes its own batch: the same shapes, inputs drawn with seed = rank."""
+    return wl.with_(seed=rank)
+
+
+def max_over_ranks(dist, v: float, device) -> float:
+    """The largest of one float over all ranks (every rank must call it); v itself
+    when there is no process group."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, wl: workloads.Workload, steps: int, t_max: float) -> float:
+    """Context tokens per second of the whole job: every rank decodes B * L tokens
+    per step, and the job takes as long as its slowest rank."""
+    return world * wl.B * wl.L * steps / t_max
+
+
+def algorithmic_flops(wl: workloads.Workload) -> int:
+    """Scores 2 H (d_c + d_r) plus the folded P.C 2 H d_c per context token."""
+    return wl.B * wl.L * (2 * wl.H * (wl.d_c + wl.d_r) + 2 * wl.H * wl.d_c)
+
+
 def our_arm(args) -> None:
     import torch
     import kv_compression_b200 as kvc
@@ -281,7 +308,7 @@ def our_arm(args) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    wl = workloads.WORKLOADS[args.workload].with_(seed=rank)   # each rank its own batch
+    wl = rank_workload(workloads.WORKLOADS[args.workload], rank)
     x = workloads.generate(wl)
     cache_bytes = x.c_kv.nbytes + x.k_r.nbytes
     copies = 1 if cache_bytes >= 4 * L2_BYTES else 2   # rotate copies so no step starts L2-warm
@@ -314,12 +341,8 @@ def our_arm(args) -> None:
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v: float) -> float:
+        return max_over_ranks(dist, v, "cuda")
 
     # Timed region: K back-to-back steps exactly as a caller issues them (no event
     # between the main and the combine kernel, so the combine's programmatic
@@ -337,7 +360,7 @@ def our_arm(args) -> None:
     clocks = nvml.stop()
     if dist is not None:
         dist.barrier()
-    t_total = max_over_ranks(e_begin.elapsed_time(e_end) * 1e-3)
+    t_total = rank_max(e_begin.elapsed_time(e_end) * 1e-3)
     assert plan.device_error() == kvc.LCA_OK
 
     # Second pass of K steps for the main kernel's own duration: an event recorded
@@ -354,15 +377,31 @@ def our_arm(args) -> None:
     torch.cuda.synchronize()
     plan.set_timing_event(None)
     main_ms = [ev_s[k].elapsed_time(ev_m[k]) for k in range(K)]
-    t_main = max_over_ranks(statistics.mean(main_ms) * 1e-3)
+    t_main = rank_max(statistics.mean(main_ms) * 1e-3)
     assert plan.device_error() == kvc.LCA_OK
     clocks["nvidia_smi_whole_run"] = sampler.stop()
 
+    # Dense MLA (mla_decode) on the same inputs: the same bytes, nothing condensed.
+    kd = max(1, min(K, 200))
+    out_d = torch.empty_like(out)
+    ed0 = torch.cuda.Event(enable_timing=True)
+    ed1 = torch.cuda.Event(enable_timing=True)
+    barrier_sync()
+    ed0.record(stream)
+    for k in range(kd):
+        q_c, q_r, c_kv, k_r = dev[k % copies]
+        plan.dense(q_c, q_r, c_kv, k_r, wl.L, out_d, stream)
+    ed1.record(stream)
+    torch.cuda.synchronize()
+    t_dense = rank_max(ed0.elapsed_time(ed1) * 1e-3)
+    assert plan.device_error() == kvc.LCA_OK
+
     tokens_per_step = world * wl.B * wl.L
-    value = tokens_per_step * K / t_total
+    value = whole_job_rate(world, wl, K, t_total)
     peaks, peak_kind = measured_peaks()
     alg = algorithmic_bytes(wl)
     achieved = alg / t_main / 1e9
+    flops = algorithmic_flops(wl)
     traffic = profiled_traffic()
 
     e2e = None
@@ -385,11 +424,7 @@ def our_arm(args) -> None:
                              h_anc if nG > 0 else None, stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        te = e0.elapsed_time(e1) * 1e-3
-        if dist is not None:
-            t = torch.tensor([te], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            te = float(t.item())
+        te = rank_max(e0.elapsed_time(e1) * 1e-3)
         h2d = hq_c.numel() * hq_c.element_size() + hq_r.numel() * hq_r.element_size() + \
             hc.numel() * hc.element_size() + hk.numel() * hk.element_size()
         d2h = h_out.numel() * 4 + (wl.B * wl.H * nG * 4)
@@ -427,10 +462,18 @@ def our_arm(args) -> None:
                      "launch_ms_min": min(main_ms), "launch_ms_max": max(main_ms),
                      "timing": "CUDA events on the launching stream around each main-kernel launch, "
                                "mean over a second pass of K steps",
-                     "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                     "flops_per_launch": flops, "achieved_tflops": flops / t_main / 1e12,
+                     "tensor_frac": flops / t_main / 1e12 / peaks["bf16_tflops"],
+                     "tensor_peak_kind": f"{peak_kind} bf16_tflops (cuBLAS burst)"},
+        "mla_decode": {"value": whole_job_rate(world, wl, kd, t_dense), "unit": UNIT,
+                       "ms_per_step": t_dense / kd * 1e3, "steps": kd,
+                       "hbm_frac": alg / (t_dense / kd) / 1e9 / peaks["hbm_gbs"],
+                       "note": "dense MLA decode over the same cache (same bytes), same kernels with n_G = 0"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 2 * K,
+        "gpu_launches_note": "timed region: main + combine per step; the instrumented and dense passes are outside it",
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
