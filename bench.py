@@ -37,6 +37,7 @@ UNIT = "context tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = ["kv_compression_b200/csrc/tc_kernel.cuh", "kv_compression_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = "profiles/lca_tc_kernel_v2lite_traffic.txt"
+TRAFFIC_WORKLOAD = "v2lite"           # the workload that capture ran on
 
 
 def workload_desc(wl: workloads.Workload) -> str:
@@ -70,11 +71,11 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic() -> int | None:
+def profiled_traffic(wl: workloads.Workload) -> int | None:
     """DRAM bytes per launch of the main kernel from the committed ncu summary,
-    or None when absent or taken on a different kernel source."""
+    or None when absent, taken on another workload or on a different kernel source."""
     path = os.path.join(ROOT, TRAFFIC_FILE)
-    if not os.path.exists(path):
+    if wl.name != TRAFFIC_WORKLOAD or not os.path.exists(path):
         return None
     kv = {}
     with open(path) as f:
@@ -402,7 +403,7 @@ def our_arm(args) -> None:
     alg = algorithmic_bytes(wl)
     achieved = alg / t_main / 1e9
     flops = algorithmic_flops(wl)
-    traffic = profiled_traffic()
+    traffic = profiled_traffic(wl)
 
     e2e = None
     if not args.no_e2e:
