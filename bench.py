@@ -1,7 +1,7 @@
 """Benchmark of the LCA decode step (one step = one lca_decode over one batch).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload v2lite] [--no-cpu-baseline] [--no-e2e]
+                  [--workload v2lite] [--g G] [--w W] [--no-cpu-baseline] [--no-e2e]
 
 Default workload: the DeepSeek-V2-Lite-shaped decode (B=8, H=16, d_c=512,
 d_r=64, L=32768, g=16, w=1024, bf16 latents, queries N(0,1)/sqrt(576)), with
@@ -245,7 +245,7 @@ def reference_arm(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = workloads.WORKLOADS[args.workload]
+    wl = with_point(workloads.WORKLOADS[args.workload], args)
     x = workloads.generate(wl)
     from oracle import oracle
     oracle.build()
@@ -265,6 +265,15 @@ def reference_arm(args) -> None:
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def with_point(wl: workloads.Workload, args) -> workloads.Workload:
+    """The workload at another (g, w) point of the same inputs (e.g. the sweep grid)."""
+    if args.g is not None:
+        wl = wl.with_(g=args.g)
+    if args.w is not None:
+        wl = wl.with_(w=args.w)
+    return wl
 
 
 def rank_workload(wl: workloads.Workload, rank: int) -> workloads.Workload:
@@ -309,7 +318,7 @@ def our_arm(args) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    wl = rank_workload(workloads.WORKLOADS[args.workload], rank)
+    wl = rank_workload(with_point(workloads.WORKLOADS[args.workload], args), rank)
     x = workloads.generate(wl)
     cache_bytes = x.c_kv.nbytes + x.k_r.nbytes
     copies = 1 if cache_bytes >= 4 * L2_BYTES else 2   # rotate copies so no step starts L2-warm
@@ -487,6 +496,8 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v2lite", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--g", type=int, default=None, help="group size (default: the workload's)")
+    ap.add_argument("--w", type=int, default=None, help="window (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
