@@ -77,7 +77,7 @@ lca_status lca_plan_destroy(lca_plan *plan);
 /* Plan options (lca_plan_set); values are int64. */
 typedef enum {
     LCA_OPT_FORCE_SIMT = 1,        /* 1: use the CUDA-core kernel even where tcgen05 applies */
-    LCA_OPT_NUM_CTAS = 2,          /* >0: CTAs of the tcgen05 kernel (default: SM count); 0: default */
+    LCA_OPT_NUM_CTAS = 2,          /* 1..SM count: CTAs of the tcgen05 kernel; 0: the SM count */
     LCA_OPT_WAIT_TIMEOUT_NS = 3,   /* bound of every in-kernel wait (default 2e9 ns) */
     LCA_OPT_DEBUG_SKIP_LOAD = 4    /* 1: the tcgen05 producer skips its first load, so the
                                       consumer's bounded wait runs out (tests the timeout path) */
@@ -102,6 +102,11 @@ lca_status lca_plan_set(lca_plan *plan, lca_option opt, int64_t value);
  *   stream     a cudaStream_t (NULL = legacy default stream)
  * The caller owns every buffer; nothing is retained after the call.  One
  * plan must not be used by two streams at once (the workspace is shared).
+ * The tcgen05 path launches two kernels, the main kernel and the split
+ * combine, both as programmatic dependents of what precedes them in the
+ * stream: each waits (griddepcontrol.wait) for the previous kernel to
+ * complete before its first global-memory access, so only their prologues
+ * overlap it.
  */
 lca_status lca_decode(lca_plan *plan, const void *q_c, const void *q_r, const void *c_kv,
                       const void *k_r, int64_t L, int g, int w, float *out, int32_t *anchor_idx,

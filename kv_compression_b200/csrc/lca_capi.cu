@@ -337,8 +337,7 @@ lca_status lca_plan_set(lca_plan* p, lca_option opt, int64_t v) {
   switch (opt) {
     case LCA_OPT_FORCE_SIMT: p->force_simt = v != 0; return LCA_OK;
     case LCA_OPT_NUM_CTAS:
-      if (v < 0 || v > 4 * (int64_t)p->num_sms) return LCA_ERR_INVALID_ARG;
-      if (v > p->num_sms) return LCA_ERR_INVALID_ARG;  // one resident wave only
+      if (v < 0 || v > p->num_sms) return LCA_ERR_INVALID_ARG;  // one resident wave only
       p->num_ctas = (int)v;
       return LCA_OK;
     case LCA_OPT_WAIT_TIMEOUT_NS:
