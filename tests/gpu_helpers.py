@@ -34,23 +34,48 @@ def make_plan(wl: workloads.Workload, opts: dict | None = None) -> kvc.Plan:
     return plan
 
 
+GUARD = 4096                      # guard elements on each side of an output buffer
+OUT_SENTINEL = -3.0e38            # exact float32 value no kernel writes
+ANC_SENTINEL = -123456789
+
+
+class Guarded:
+    """A device tensor with sentinel-filled guard regions before and after it, so a
+    write past either end of an output (there is no sanitizer on the pool) is seen."""
+
+    def __init__(self, shape, dtype, fill, sentinel):
+        self.n = int(np.prod(shape))
+        self.sentinel = sentinel
+        self.buf = torch.full((self.n + 2 * GUARD,), sentinel, dtype=dtype, device="cuda")
+        self.t = self.buf[GUARD:GUARD + self.n].view(shape)   # 16 KB in: 16-byte aligned
+        self.t.fill_(fill)
+
+    def check(self) -> None:
+        head, tail = self.buf[:GUARD], self.buf[GUARD + self.n:]
+        assert bool((head == self.sentinel).all()), "write before the start of an output"
+        assert bool((tail == self.sentinel).all()), "write past the end of an output"
+
+
 def run_lca(plan: kvc.Plan, d: DeviceInputs, g: int, w: int):
     wl = d.x.wl
     nG = kvc.num_groups(wl.L, g, w)
-    out = torch.full((wl.B, wl.H, wl.d_c), float("nan"), dtype=torch.float32, device="cuda")
-    anc = torch.full((wl.B, wl.H, max(nG, 1)), -7, dtype=torch.int32, device="cuda")
-    plan.decode(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, g, w, out, anc if nG > 0 else None)
+    out = Guarded((wl.B, wl.H, wl.d_c), torch.float32, float("nan"), OUT_SENTINEL)
+    anc = Guarded((wl.B, wl.H, max(nG, 1)), torch.int32, -7, ANC_SENTINEL)
+    plan.decode(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, g, w, out.t, anc.t if nG > 0 else None)
     torch.cuda.synchronize()
     assert plan.device_error() == kvc.LCA_OK
-    return out.cpu().numpy().astype(np.float64), anc.cpu().numpy()[:, :, :nG]
+    out.check()
+    anc.check()
+    return out.t.cpu().numpy().astype(np.float64), anc.t.cpu().numpy()[:, :, :nG]
 
 
 def run_dense(plan: kvc.Plan, d: DeviceInputs):
     wl = d.x.wl
-    out = torch.full((wl.B, wl.H, wl.d_c), float("nan"), dtype=torch.float32, device="cuda")
-    plan.dense(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, out)
+    out = Guarded((wl.B, wl.H, wl.d_c), torch.float32, float("nan"), OUT_SENTINEL)
+    plan.dense(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, out.t)
     torch.cuda.synchronize()
-    return out.cpu().numpy().astype(np.float64)
+    out.check()
+    return out.t.cpu().numpy().astype(np.float64)
 
 
 def oracle_lca(x: workloads.Inputs, g: int, w: int, rows=None, heads=None):

@@ -17,7 +17,8 @@ if not torch.cuda.is_available():
 
 import kv_compression_b200 as kvc  # noqa: E402
 import workloads  # noqa: E402
-from gpu_helpers import BF16_TOL, F32_TOL, DeviceInputs, make_plan, rel_err, run_lca  # noqa: E402
+from gpu_helpers import (ANC_SENTINEL, BF16_TOL, F32_TOL, OUT_SENTINEL, DeviceInputs,  # noqa: E402
+                         Guarded, make_plan, rel_err, run_lca)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,16 +30,18 @@ def _vp(t):
 def run_noalloc(wl, d, g, w):
     lib = kvc.load_library()
     nG = kvc.num_groups(wl.L, g, w)
-    out = torch.full((wl.B, wl.H, wl.d_c), float("nan"), dtype=torch.float32, device="cuda")
-    anc = torch.full((wl.B, wl.H, max(nG, 1)), -7, dtype=torch.int32, device="cuda")
+    out = Guarded((wl.B, wl.H, wl.d_c), torch.float32, float("nan"), OUT_SENTINEL)
+    anc = Guarded((wl.B, wl.H, max(nG, 1)), torch.int32, -7, ANC_SENTINEL)
     dt = kvc.LCA_BF16 if wl.dtype == "bf16" else kvc.LCA_F32
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     st = lib.lca_decode_noalloc(wl.B, wl.H, wl.d_c, wl.d_r, dt, _vp(d.q_c), _vp(d.q_r),
-                                _vp(d.c_kv), _vp(d.k_r), wl.L, g, w, _vp(out),
-                                _vp(anc) if nG > 0 else None, stream)
+                                _vp(d.c_kv), _vp(d.k_r), wl.L, g, w, _vp(out.t),
+                                _vp(anc.t) if nG > 0 else None, stream)
     assert st == kvc.LCA_OK, kvc.STATUS.get(st, st)
     torch.cuda.synchronize()
-    return out.cpu().numpy().astype(np.float64), anc.cpu().numpy()[:, :, :nG]
+    out.check()
+    anc.check()
+    return out.t.cpu().numpy().astype(np.float64), anc.t.cpu().numpy()[:, :, :nG]
 
 
 @pytest.mark.parametrize("wl,tol", [
