@@ -308,6 +308,18 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   // of the previous kernel in the stream, and nothing below reads or writes
   // global memory before that kernel has completed and its writes are visible.
   // The combine that follows may be scheduled from here on; it waits the same way.
+  // Start the range's first tile and query block on their way into L2 while the
+  // previous kernel may still run: an L2 prefetch returns no data to this CTA,
+  // and L2 holds every later write to those lines, so nothing read after the
+  // wait below can be stale.  (One tile: prefetching two measured no better.)
+  if (tid == 0) {
+    const int32_t frow = (int32_t)(seq0 * p.L + tile0 * kT);
+    for (int cc = 0; cc < 8; ++cc) ptx::tma_prefetch_l2_2d(&p.tm_c, 64 * cc, frow);
+    ptx::tma_prefetch_l2_2d(&p.tm_k, 0, frow);
+    const int32_t qrow = (int32_t)(seq0 * p.H + h0);
+    for (int k = 0; k < 8; ++k) ptx::tma_prefetch_l2_2d(&p.tm_qc, 64 * k, qrow);
+    ptx::tma_prefetch_l2_2d(&p.tm_qr, 0, qrow);
+  }
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
 
