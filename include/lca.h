@@ -102,6 +102,8 @@ lca_status lca_plan_set(lca_plan *plan, lca_option opt, int64_t value);
  *   stream     a cudaStream_t (NULL = legacy default stream)
  * The caller owns every buffer; nothing is retained after the call.  One
  * plan must not be used by two streams at once (the workspace is shared).
+ * The tcgen05 path needs B * L < 2^31 cache rows (its TMA row coordinates
+ * are 32-bit) and returns LCA_ERR_UNSUPPORTED otherwise.
  * The tcgen05 path launches two kernels, the main kernel and the split
  * combine, both as programmatic dependents of what precedes them in the
  * stream: each waits (griddepcontrol.wait) for the previous kernel to

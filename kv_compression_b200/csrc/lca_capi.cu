@@ -201,6 +201,7 @@ lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_k
   lca::tc::TcParams tp;
   std::memset(&tp, 0, sizeof(tp));
   const uint64_t rows = (uint64_t)p->B * (uint64_t)L;
+  if (rows > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
   const uint64_t qrows = (uint64_t)p->B * (uint64_t)p->H;
   if (!make_map(&tp.tm_c, c_kv, 512, rows, 128) || !make_map(&tp.tm_k, k_r, 64, rows, 128) ||
       !make_map(&tp.tm_qc, q_c, 512, qrows, 16) || !make_map(&tp.tm_qr, q_r, 64, qrows, 16))

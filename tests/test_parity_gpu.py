@@ -145,3 +145,9 @@ def test_argument_errors():
     assert lib.lca_plan_set(big.handle, kvc.OPT_NUM_CTAS, 10**6) == 1
     assert lib.lca_plan_set(big.handle, 99, 1) == 1
     big.close()
+    # B * L beyond the 32-bit TMA row range is refused before anything is launched
+    huge_L = (1 << 30) + 128
+    huge = kvc.Plan(2, 16, 512, 64, "bf16", huge_L)
+    assert lib.lca_decode(huge.handle, P(d.q_c), P(d.q_r), P(c), P(k), huge_L, 16, 0, P(out),
+                          P(anc), s) == 2
+    huge.close()
