@@ -168,17 +168,19 @@ int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
  * layouts and ownership as for lca_decode (L has no max_L bound).  Same
  * kernels and results as lca_decode.
  * Scratch: the split partials live in one fixed file-scope device array of
- * 16 MiB (plus 64 KiB), so the tile ranges are capped to what fits; shapes
- * with B * H * d_c > 4 Mi floats return LCA_ERR_UNSUPPORTED.  The device error
- * word in that array is cleared on `stream` at the start of every call; a
- * bounded in-kernel wait that runs out leaves outputs undefined and is not
- * reported by this call.
+ * 16 MiB of partial outputs plus 64 KiB of (max, sum) pairs, so the tile
+ * ranges are capped to what both regions hold; shapes with
+ * B * H * max(d_c, 512) > 4 Mi floats return LCA_ERR_UNSUPPORTED before
+ * anything is launched.  The device error word in that array is cleared on
+ * `stream` at the start of every call; a bounded in-kernel wait that runs out
+ * leaves outputs undefined and is not reported by this call.
  * The first call on a device looks up the scratch's address there and sets
- * the kernels' shared-memory limit; make that first call before any stream
- * capture.  Every call on a device shares the one scratch: calls that overlap
- * in time (two streams, or two host threads) race and corrupt each other's
- * results.  Errors: LCA_ERR_INVALID_ARG, LCA_ERR_UNSUPPORTED,
- * LCA_ERR_ALIGNMENT, LCA_ERR_CUDA.
+ * the kernels' shared-memory limit (thread-safe: concurrent first calls are
+ * serialised); make that first call before any stream capture.  Every call on
+ * a device shares the one scratch: calls that overlap on the GPU (two
+ * streams, or two host threads) race and corrupt each other's results.
+ * Errors: LCA_ERR_INVALID_ARG, LCA_ERR_UNSUPPORTED, LCA_ERR_ALIGNMENT,
+ * LCA_ERR_CUDA.
  */
 lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, const void *q_c,
                               const void *q_r, const void *c_kv, const void *k_r, int64_t L, int g,

@@ -5,8 +5,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "lca.h"
@@ -43,9 +45,11 @@ struct lca_plan {
 // Fixed device scratch of lca_decode_noalloc (zero at module load): split
 // partials [slots][H][d_c] and [slots][H][2] floats, then the device error
 // word (2 ints).  Only lca_decode_noalloc uses it, through the address that
-// cudaGetSymbolAddress gives for the current device.
+// cudaGetSymbolAddress gives for the current device.  A call may use at most
+// min(kNoAllocOFloats / (H d_c), kNoAllocMzFloats / (2 H)) slots, so that both
+// regions hold every slot it writes.
 constexpr size_t kNoAllocOFloats = (size_t)4 << 20;              // 16 MiB of partial outputs
-constexpr size_t kNoAllocMzFloats = kNoAllocOFloats / 256;       // (M, Z) pairs of the same slots
+constexpr size_t kNoAllocMzFloats = kNoAllocOFloats / 256;       // 64 KiB of (M, Z) pairs
 constexpr size_t kNoAllocErrOffset = kNoAllocOFloats + kNoAllocMzFloats;
 static __device__ __align__(256) float lca_noalloc_scratch[kNoAllocErrOffset + 64];
 
@@ -154,15 +158,27 @@ lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c
   return launch_combine(p, cp, stream, false);
 }
 
+constexpr int kMaxDevices = 64;
+
+// One bit per device: the kernel's shared-memory limit is set there.  Setting
+// it twice is harmless, so two threads racing on a first call only repeat it.
+bool device_flag_set(std::atomic<uint64_t>& flags, int device) {
+  return device >= 0 && device < kMaxDevices && ((flags.load(std::memory_order_acquire) >> device) & 1u);
+}
+void device_flag_mark(std::atomic<uint64_t>& flags, int device) {
+  if (device >= 0 && device < kMaxDevices)
+    flags.fetch_or(uint64_t(1) << device, std::memory_order_acq_rel);
+}
+
 template <int LOG2G>
 cudaError_t launch_tc(const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream, int device) {
-  static int configured_device = -1;
-  if (configured_device != device) {
+  static std::atomic<uint64_t> configured{0};
+  if (!device_flag_set(configured, device)) {
     cudaError_t e = cudaFuncSetAttribute(lca::tc::lca_tc_kernel<LOG2G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          lca::tc::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    configured_device = device;
+    device_flag_mark(configured, device);
   }
   // Programmatic stream serialization: the kernel's prologue (barrier init,
   // TMEM allocation) may overlap the previous kernel's tail; the kernel waits on
@@ -429,13 +445,15 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
 // this entry point runs the same kernels as lca_decode with the fixed
 // file-scope scratch above in place of a plan's workspace, and allocates
 // nothing.  The first call on a device looks up the scratch's address there
-// (cudaGetSymbolAddress) and sets the kernels' shared-memory limit.
+// (cudaGetSymbolAddress) and its SM count, under a mutex, so concurrent first
+// calls from several host threads are safe; later calls read the cached
+// values without locking.
 lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, const void* q_c,
                               const void* q_r, const void* c_kv, const void* k_r, int64_t L, int g,
                               int w, float* out, int32_t* anchor, void* stream) {
-  constexpr int kMaxDevices = 64;
-  static float* scratch[kMaxDevices] = {};   // the scratch's address, per device
-  static int sms[kMaxDevices] = {};
+  static std::atomic<float*> scratch[kMaxDevices];   // the scratch's address, per device
+  static std::atomic<int> sms[kMaxDevices];
+  static std::mutex first_call;
   if (B < 1 || H < 1 || d_c < 1 || d_r < 1 || L < 1 || g < 1 || w < 0) return LCA_ERR_INVALID_ARG;
   if (!q_c || !q_r || !c_kv || !k_r || !out) return LCA_ERR_INVALID_ARG;
   if (dt != LCA_F32 && dt != LCA_BF16) return LCA_ERR_INVALID_ARG;
@@ -444,27 +462,37 @@ lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, cons
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return LCA_ERR_UNSUPPORTED;
-  if (!scratch[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, lca_noalloc_scratch) != cudaSuccess) return LCA_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return LCA_ERR_CUDA;
-    scratch[dev] = static_cast<float*>(ptr);
+  if (!scratch[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(first_call);
+    if (!scratch[dev].load(std::memory_order_acquire)) {
+      void* ptr = nullptr;
+      int n_sm = 0;
+      if (cudaGetSymbolAddress(&ptr, lca_noalloc_scratch) != cudaSuccess) return LCA_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LCA_ERR_CUDA;
+      sms[dev].store(n_sm, std::memory_order_relaxed);
+      scratch[dev].store(static_cast<float*>(ptr), std::memory_order_release);
+    }
   }
-  // Split slots that fit the scratch; fewer than B is a size beyond its limit.
-  const int64_t cap = (int64_t)(kNoAllocOFloats / ((size_t)H * (size_t)d_c));
+  float* base = scratch[dev].load(std::memory_order_acquire);
+  // Split slots that fit BOTH regions of the scratch: partial outputs (H d_c
+  // floats a slot) and (M, Z) pairs (2 H floats a slot).  Fewer than B slots
+  // is a shape beyond the scratch's limit.
+  const int64_t cap_o = (int64_t)(kNoAllocOFloats / ((size_t)H * (size_t)d_c));
+  const int64_t cap_mz = (int64_t)(kNoAllocMzFloats / ((size_t)2 * (size_t)H));
+  const int64_t cap = std::min(cap_o, cap_mz);
   if (cap < B) return LCA_ERR_UNSUPPORTED;
   lca_plan plan;
   std::memset(&plan, 0, sizeof(plan));
   plan.B = B; plan.H = H; plan.d_c = d_c; plan.d_r = d_r; plan.dt = dt; plan.max_L = L;
   plan.device = dev;
-  plan.num_sms = sms[dev];
+  plan.num_sms = sms[dev].load(std::memory_order_relaxed);
   plan.tc_shape = dt == LCA_BF16 && d_c == lca::tc::kDC && d_r == lca::tc::kDR &&
                   (H % lca::tc::kHC) == 0;
-  plan.ws_slots = cap;
-  plan.part_o = scratch[dev];
-  plan.part_mz = scratch[dev] + kNoAllocOFloats;
-  plan.err = reinterpret_cast<int*>(scratch[dev] + kNoAllocErrOffset);
+  plan.ws_slots = cap;   // run_simt and run_tc refuse a launch that needs more slots
+  plan.part_o = base;
+  plan.part_mz = base + kNoAllocOFloats;
+  plan.err = reinterpret_cast<int*>(base + kNoAllocErrOffset);
   plan.timeout_ns = kDefaultTimeoutNs;
   if (plan.tc_shape) {   // as many tile ranges as the scratch holds partials for
     const int64_t n_hb = H / lca::tc::kHC;

@@ -65,6 +65,24 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     lib = kvc.load_library()
     buf = torch.zeros(16, dtype=torch.uint8, device="cuda")
     p = _vp(buf)
-    # B * H * d_c = 64 * 128 * 1024 floats > the 4 Mi floats of scratch
+    # B * H * d_c = 64 * 128 * 1024 floats > the 4 Mi floats of partial outputs
     st = lib.lca_decode_noalloc(64, 128, 1024, 64, kvc.LCA_BF16, p, p, p, p, 16, 1, 0, p, p, None)
     assert st == kvc.LCA_ERR_UNSUPPORTED
+    # small d_c: the partial outputs would fit, the (max, sum) pairs would not
+    # (B * H = 64 * 256 > 8192 slot-heads); refused before any launch
+    st = lib.lca_decode_noalloc(64, 256, 64, 16, kvc.LCA_BF16, p, p, p, p, 16, 1, 0, p, p, None)
+    assert st == kvc.LCA_ERR_UNSUPPORTED
+
+
+def test_noalloc_small_latent_at_the_pair_limit():
+    """d_c = 64 with B * H = 8192 slot-heads: exactly what the (max, sum) region
+    holds for one slot per sequence.  It must run inside the scratch (guard
+    regions intact) and match lca_decode."""
+    wl = workloads.small("na_edge", B=64, H=128, L=40, g=4, w=8, d_c=64, d_r=16, dtype="f32",
+                         seed=43)
+    x = workloads.generate(wl)
+    d = DeviceInputs(x)
+    ref_out, ref_anc = run_lca(make_plan(wl), d, wl.g, wl.w)
+    got_out, got_anc = run_noalloc(wl, d, wl.g, wl.w)
+    assert rel_err(got_out, ref_out) <= F32_TOL
+    assert np.array_equal(got_anc, ref_anc)
