@@ -88,21 +88,30 @@ def torch_attention(q: np.ndarray, keys: np.ndarray, vals: np.ndarray) -> np.nda
     return o[0, :, 0, :].numpy()
 
 
-def torch_lca_seq(qc, qr, C, K, g, w):
+def torch_lca_seq(qc, qr, C, K, g, w, stats=False):
     """LCA for one sequence built from library routines, per the page's steps.
-    Returns (out [H, d_c], anchor [H, n_G])."""
+    Returns (out [H, d_c], anchor [H, n_G]); with stats=True also the top-2
+    score gap of every group [H, n_G] (torch.topk; +inf for one-token groups)
+    and max |s| over the sequence [H] -- the near-tie report the GPU tests use
+    to decide which bf16 anchors must match."""
     H = qc.shape[0]
     groups, window = partition(C.shape[0], g, w)
     Ct, Kt = torch.from_numpy(C), torch.from_numpy(K)
-    outs, ancs = [], []
+    outs, ancs, gaps, amax = [], [], [], []
     for h in range(H):
         qch, qrh = torch.from_numpy(qc[h]), torch.from_numpy(qr[h])
         s = Ct @ qch + Kt @ qrh                     # full MLA score of every token
-        keys, vals, anc = [], [], []
+        amax.append(float(s.abs().max()))
+        keys, vals, anc, gap = [], [], [], []
         for G in groups:
             idx = torch.tensor(G)
             wts = torch.softmax(s[idx], dim=0)         # step 2: query-aware pooling weights
             a = G[int(torch.argmax(s[idx]))]           # step 2: highest-scoring token (first max)
+            if len(G) >= 2:
+                top = torch.topk(s[idx], 2).values
+                gap.append(float(top[0] - top[1]))
+            else:
+                gap.append(math.inf)
             cbar = wts @ Ct[idx]
             keys.append(torch.cat([cbar, Kt[a]]))
             vals.append(cbar)
@@ -115,7 +124,12 @@ def torch_lca_seq(qc, qr, C, K, g, w):
         q = np.concatenate([qc[h], qr[h]])[None]
         outs.append(torch_attention(q, keys_np, vals_np)[0])   # step 3
         ancs.append(anc)
-    return np.stack(outs), np.array(ancs, dtype=np.int32).reshape(H, len(groups))
+        gaps.append(gap)
+    out = np.stack(outs)
+    ancs = np.array(ancs, dtype=np.int32).reshape(H, len(groups))
+    if stats:
+        return out, ancs, np.array(gaps, np.float64).reshape(H, len(groups)), np.array(amax)
+    return out, ancs
 
 
 def torch_dense_seq(qc, qr, C, K):
@@ -203,6 +217,16 @@ def pin_constant_groups(lib):
         assert list(res.anchor[0, h]) == reps
 
 
+def _check_near_tie_report(res, gap, amax, where):
+    """The oracle's top-2 gaps and max |s| against torch (float64, another
+    summation order: equal to ~1e-15 relative)."""
+    tol = 1e-12 * max(float(amax.max()), 1.0)
+    assert np.allclose(res.max_abs_s[0], amax, rtol=1e-12, atol=0.0), where
+    finite = np.isfinite(gap)
+    assert np.array_equal(np.isfinite(res.tie_gap[0]), finite), where
+    assert np.all(np.abs(res.tie_gap[0][finite] - gap[finite]) <= tol), where
+
+
 def pin_brute_force(lib):
     rng = np.random.default_rng(16)
     for dtype in ("f32", "bf16"):
@@ -211,9 +235,35 @@ def pin_brute_force(lib):
             for g in range(1, L + 2):
                 for w in range(0, L + 2):
                     res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
-                    ref, anc = torch_lca_seq(widen(qc[0]), widen(qr[0]), widen(C[0]), widen(K[0]), g, w)
+                    ref, anc, gap, amax = torch_lca_seq(widen(qc[0]), widen(qr[0]), widen(C[0]),
+                                                        widen(K[0]), g, w, stats=True)
                     assert rel_err(res.out[0], ref) < REL_TOL, (dtype, L, g, w)
                     assert np.array_equal(res.anchor[0], anc), (dtype, L, g, w)
+                    _check_near_tie_report(res, gap, amax, (dtype, L, g, w))
+
+
+def pin_near_tie_report(lib):
+    """The near-tie report on longer sequences and several heads, where the
+    group maximum sits anywhere in the group and max |s| comes from a
+    negative score about half of the time (scores are shifted per head so
+    that both signs occur)."""
+    rng = np.random.default_rng(22)
+    for dtype in ("f32", "bf16"):
+        for (L, g, w, shift) in ((96, 8, 5, -3.0), (130, 16, 0, 3.0), (64, 4, 9, -2.0)):
+            qc, qr, C, K = rand_inputs(rng, 1, 4, L, 16, 8, dtype)
+            # a constant RoPE key component shifts every score of a head by the
+            # same amount (here negative or positive), which moves max |s|
+            # between the largest and the most negative score
+            if dtype == "f32":
+                K[0, :, 0] = np.float32(shift / max(abs(float(qr[0, 0, 0])), 1e-3))
+            res = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+            _, anc, gap, amax = torch_lca_seq(widen(qc[0]), widen(qr[0]), widen(C[0]), widen(K[0]),
+                                              g, w, stats=True)
+            assert np.array_equal(res.anchor[0], anc), (dtype, L, g, w)
+            _check_near_tie_report(res, gap, amax, (dtype, L, g, w))
+            # the gap is measured from the anchor: never negative, and zero
+            # only at an exact tie
+            assert np.all(res.tie_gap[0] >= 0.0)
 
 
 def pin_ties(lib):
@@ -275,5 +325,5 @@ def pin_constant_rope(lib):
 
 
 ALL_PINS = [pin_segmentation, pin_dense_vs_torch, pin_g1_dense, pin_window_dense, pin_zero_query,
-            pin_constant_groups, pin_brute_force, pin_ties, pin_formulations, pin_permutation,
-            pin_constant_rope]
+            pin_constant_groups, pin_brute_force, pin_near_tie_report, pin_ties, pin_formulations,
+            pin_permutation, pin_constant_rope]

@@ -45,6 +45,16 @@ MUTANTS = {
     # positional score uses the semantic query (transposed operand)
     "rope_score_wrong_query": ("w->sr[t] = dot_row(w->qr, k_r, t, d_r, dtype);",
                                "w->sr[t] = dot_row(w->qc, k_r, t, d_r, dtype);"),
+    # near-tie report: runner-up taken over the whole group, anchor included
+    # (every gap would be 0 and no bf16 anchor would ever be compared)
+    "tie_gap_second_includes_anchor": ("if (t != a && w->s[t] > second) second = w->s[t];",
+                                       "if (w->s[t] > second) second = w->s[t];"),
+    # near-tie report: max of s instead of max of |s|
+    "max_abs_s_signed": ("if (fabs(w->s[t]) > amax) amax = fabs(w->s[t]);",
+                         "if (w->s[t] > amax) amax = w->s[t];"),
+    # near-tie report: runner-up excludes the group's first token, not the anchor
+    "tie_gap_wrong_token": ("if (t != a && w->s[t] > second) second = w->s[t];",
+                            "if (t != t0 && w->s[t] > second) second = w->s[t];"),
 }
 
 
