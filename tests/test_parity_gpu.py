@@ -47,7 +47,7 @@ def test_small_bf16(case, kernel):
     assert plan.kernel(L, g, w) == kernel
     out, anc = run_lca(plan, DeviceInputs(x), g, w)
     ref = oracle_lca(x, g, w)
-    compare(out, anc, ref, BF16_TOL, exact_anchors=False)
+    compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=g)
 
 
 def test_ranges_spanning_sequences():
@@ -59,7 +59,7 @@ def test_ranges_spanning_sequences():
     for n in (2, 3, 6, 16):
         plan = make_plan(wl, {kvc.OPT_NUM_CTAS: n})
         out, anc = run_lca(plan, d, wl.g, wl.w)
-        compare(out, anc, ref, BF16_TOL, exact_anchors=False)
+        compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
 
 
 def test_tiny_f32_config():
@@ -108,7 +108,8 @@ def test_host_buffer_entry_point():
     anc = torch.empty(wl.B, wl.H, nG, dtype=torch.int32).pin_memory()
     plan.decode_host(host(x.q_c), host(x.q_r), host(x.c_kv), host(x.k_r), wl.L, wl.g, wl.w, out, anc)
     ref = oracle_lca(x, wl.g, wl.w)
-    compare(out.numpy().astype(np.float64), anc.numpy(), ref, BF16_TOL, exact_anchors=False)
+    compare(out.numpy().astype(np.float64), anc.numpy(), ref, BF16_TOL, exact_anchors=False, x=x,
+            g=wl.g)
 
 
 def test_argument_errors():

@@ -10,8 +10,8 @@ if not torch.cuda.is_available():
 
 import kv_compression_b200 as kvc  # noqa: E402
 import workloads  # noqa: E402
-from gpu_helpers import (BF16_TOL, DeviceInputs, compare, make_plan, oracle_lca,  # noqa: E402
-                         run_lca)
+from gpu_helpers import (ANCHOR_GAP, BF16_TOL, DeviceInputs, compare, group_scores,  # noqa: E402
+                         make_plan, oracle_dense, oracle_lca, rel_err, run_dense, run_lca)
 
 pytestmark = pytest.mark.gpu
 
@@ -36,18 +36,23 @@ def _check(name, rows, heads, points=None):
         ref = oracle_lca(x, g, w, rows=rows, heads=heads)
         sub_out = out[rows][:, heads] if heads is not None else out[rows]
         sub_anc = anc[rows][:, heads] if heads is not None else anc[rows]
-        results.append((g, w, compare(sub_out, sub_anc, ref, BF16_TOL, exact_anchors=False)))
+        results.append((g, w, compare(sub_out, sub_anc, ref, BF16_TOL, exact_anchors=False, x=x, g=g,
+                                      heads=heads)))
         del out, anc
     return x, results
 
 
 def test_v2lite_full():
     wl = workloads.WORKLOADS["v2lite"]
-    _check("v2lite", rows=list(range(wl.B)), heads=None)
+    x, _ = _check("v2lite", rows=list(range(wl.B)), heads=None)
+    # dense MLA decode (the bench's same-bytes comparison) over the whole batch
+    out = run_dense(make_plan(wl), DeviceInputs(x))
+    assert rel_err(out, oracle_dense(x)) <= BF16_TOL
 
 
 def test_v2_sampled():
-    _check("v2", rows=[0, 31], heads=[0, 1, 63, 100, 127])
+    # one head from each 16-head block of the CUDA path, both 64-head halves
+    _check("v2", rows=[0, 31], heads=[0, 17, 34, 51, 68, 85, 102, 127])
 
 
 def test_needle_sampled_and_tie_break():
@@ -57,20 +62,63 @@ def test_needle_sampled_and_tie_break():
     plan = make_plan(wl)
     _, anc = run_lca(plan, d, wl.g, wl.w)
     win0 = wl.n_groups * wl.g
-    pairs = 0
+    heads = np.arange(wl.H)
+    binding = 0
     for b in range(wl.B):
         pos = x.needle_pos[b]
         for j in np.unique(pos[pos < win0] // wl.g):
             planted = pos[(pos // wl.g) == j]
-            a = anc[b, :, j]
-            # identical planted rows score identically: an anchor on a planted
-            # token must be the lowest planted index of its group
-            on_planted = np.isin(a, planted)
-            assert np.all(a[on_planted] == planted.min())
-            pairs += len(planted) > 1
-    assert pairs > 0, "no group holds two needles; the tie-break is untested"
+            if len(planted) < 2:
+                continue
+            # double scores of the group on every head; identical planted rows
+            # score identically, so where they beat every other token by more
+            # than the near-tie gate the anchor must be the lowest planted index
+            s = group_scores(x, np.full(wl.H, b), heads, np.full(wl.H, j), wl.g)   # [H, g]
+            is_needle = np.isin(np.arange(j * wl.g, (j + 1) * wl.g), planted)
+            s_needle = s[:, is_needle].max(axis=1)
+            s_other = s[:, ~is_needle].max(axis=1)
+            amax = np.abs(s).max(axis=1)
+            wins = s_needle > s_other + ANCHOR_GAP * amax
+            assert np.all(anc[b, wins, j] == planted.min()), (b, j)
+            binding += int(wins.sum())
+    assert binding > 0, "no (group, head) where two or more needles win; the tie-break is untested"
 
 
 def test_sweep_sampled():
     wl = workloads.WORKLOADS["sweep"]
     _check("sweep", rows=[0, 15], heads=[0, 7, 15], points=list(wl.sweep))
+
+
+def test_v2lite_repeatable():
+    """The full V2-Lite decode 30 times on the same inputs: every run must give
+    bit-identical outputs and anchors (the kernels are deterministic: fixed
+    tile ranges, fixed MMA and merge order), so a rare ordering race in the
+    barrier or ring logic shows up as a difference.  The first run is also
+    checked against the oracle."""
+    wl = workloads.WORKLOADS["v2lite"]
+    x = workloads.generate(wl, threads=16)
+    d = DeviceInputs(x)
+    plan = make_plan(wl)
+    out0, anc0 = run_lca(plan, d, wl.g, wl.w)
+    ref = oracle_lca(x, wl.g, wl.w, rows=[0, wl.B - 1])
+    compare(out0[[0, wl.B - 1]], anc0[[0, wl.B - 1]], ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+    for _ in range(29):
+        out, anc = run_lca(plan, d, wl.g, wl.w)
+        assert np.array_equal(out, out0)
+        assert np.array_equal(anc, anc0)
+
+
+def test_spanning_ranges_repeatable():
+    """Tile ranges that cross sequence boundaries, at several CTA counts,
+    five runs each: bit-identical, and equal to the oracle within tolerance."""
+    wl = workloads.small("t", B=6, H=128, L=3000, g=16, w=200, seed=8)
+    x = workloads.generate(wl)
+    d = DeviceInputs(x)
+    ref = oracle_lca(x, wl.g, wl.w)
+    for n in (2, 3, 8, 16, 37, 148):
+        plan = make_plan(wl, {kvc.OPT_NUM_CTAS: n})
+        out0, anc0 = run_lca(plan, d, wl.g, wl.w)
+        compare(out0, anc0, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+        for _ in range(4):
+            out, anc = run_lca(plan, d, wl.g, wl.w)
+            assert np.array_equal(out, out0) and np.array_equal(anc, anc0), n
