@@ -1,23 +1,30 @@
 """Benchmark of the LCA decode step (one step = one lca_decode over one batch).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload v2lite] [--g G] [--w W] [--no-cpu-baseline] [--no-e2e]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--blocks R]
+                  [--impl ours|reference|ranks] [--workload v2] [--g G] [--w W]
+                  [--no-cpu-baseline] [--no-e2e] [--no-per-config]
 
-Default workload: the DeepSeek-V2-Lite-shaped decode (B=8, H=16, d_c=512,
-d_r=64, L=32768, g=16, w=1024, bf16 latents, queries N(0,1)/sqrt(576)), with
-synthetic seeded inputs.  Metric: context tokens per second (B*L per step),
-whole job over all ranks.  Under torchrun every rank runs its own batch on
-its own GPU (sequences are independent: no collective on the data path) and
-the time is the max over ranks ("weak" scaling).
+Default workload: the DeepSeek-V2-shaped decode (B=32, H=128 heads sharing one
+latent, d_c=512, d_r=64, L=65536, g=16, w=2048, bf16 latents, queries
+N(0,1)/sqrt(576)) -- the largest workload that fits one GPU -- with synthetic
+seeded inputs.  Metric: context tokens per second (B*L per step), whole job
+over all ranks, from the median of R timed blocks of K steps each.  Under
+torchrun every rank runs its own batch on its own GPU (sequences are
+independent: no collective on the data path) and the time is the max over
+ranks ("weak" scaling); `--gpus N` without torchrun starts the N ranks itself.
+The other benchmark workloads (V2-Lite, needle, the ten sweep points, the tiny
+fp32 case) are timed in the same process under "per_config".
 
 Prints one JSON line on rank 0.  `--impl reference` times the CPU oracle on
 the host cores instead (rank 0 only), on bounded samples of the same workload.
+`--impl ranks` runs only the rank plumbing (gloo, CPU) as a stand-in arm.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -38,6 +45,7 @@ L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = ["kv_compression_b200/csrc/tc_kernel.cuh", "kv_compression_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = "profiles/lca_tc_kernel_v2lite_traffic.txt"
 TRAFFIC_WORKLOAD = "v2lite"           # the workload that capture ran on
+MAIN_KERNEL_NAMES = {"tcgen05": "lca_tc_kernel", "simt": "lca_simt_kernel"}
 
 
 def workload_desc(wl: workloads.Workload) -> str:
@@ -255,7 +263,8 @@ def reference_arm(args) -> None:
         run_cpu_oracle_steps(wl, x, min(args.warmup, 1), budget / 10, nthreads)
     value, desc, secs = run_cpu_oracle_steps(wl, x, args.steps, budget, nthreads)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(args.steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, workloads/)",
@@ -303,6 +312,181 @@ def algorithmic_flops(wl: workloads.Workload) -> int:
     return wl.B * wl.L * (2 * wl.H * (wl.d_c + wl.d_r) + 2 * wl.H * wl.d_c)
 
 
+def spawn_ranks(args) -> int | None:
+    """`--gpus N` without torchrun: start N local ranks under torch.distributed.run
+    (rendezvous on 127.0.0.1) and return their exit status; None when this
+    process already is a rank (WORLD_SIZE set) or N == 1."""
+    if args.gpus <= 1 or "WORLD_SIZE" in os.environ:
+        return None
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node",
+           str(args.gpus), "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def ranks_arm(args) -> None:
+    """Stand-in for the GPU arm that exercises only the rank plumbing on CPU
+    (gloo): every rank joins, the world size and the max over ranks are
+    formed exactly as the GPU arm forms them, and rank 0 prints one line."""
+    import datetime
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    pg = None
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        pg = dist
+    t = max_over_ranks(pg, 1.0 + rank, "cpu")
+    ranks = [None] * world
+    if pg is not None:
+        dist.all_gather_object(ranks, rank)
+        dist.destroy_process_group()
+    else:
+        ranks = [0]
+    if rank == 0:
+        print(json.dumps({"impl": "ranks", "n_gpus": world, "ranks": ranks, "t_max": t}), flush=True)
+
+
+class Timer:
+    """CUDA events on the launching stream."""
+
+    def __init__(self, torch, stream):
+        self.torch, self.stream = torch, stream
+        self.a = torch.cuda.Event(enable_timing=True)
+        self.b = torch.cuda.Event(enable_timing=True)
+
+    def start(self):
+        self.a.record(self.stream)
+
+    def stop(self) -> float:
+        self.b.record(self.stream)
+        self.b.synchronize()
+        return self.a.elapsed_time(self.b) * 1e-3
+
+
+class Runner:
+    """One workload resident in HBM with its plan and outputs; `step(k)` is one
+    lca_decode over the whole batch (copies of the inputs rotated so that no
+    step starts with its cache warm in L2)."""
+
+    def __init__(self, torch, kvc, wl, stream):
+        self.torch, self.kvc, self.wl, self.stream = torch, kvc, wl, stream
+        self.x = workloads.generate(wl, threads=16)
+        self.cache_bytes = self.x.c_kv.nbytes + self.x.k_r.nbytes
+        self.copies = 1 if self.cache_bytes >= 4 * L2_BYTES else 2
+        self.dev = [(to_device(self.x.q_c, torch), to_device(self.x.q_r, torch),
+                     to_device(self.x.c_kv, torch), to_device(self.x.k_r, torch))
+                    for _ in range(self.copies)]
+        self.plan = kvc.Plan(wl.B, wl.H, wl.d_c, wl.d_r, wl.dtype, wl.L)
+        self.nG = wl.n_groups
+        self.out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32, device="cuda")
+        self.anc = torch.empty(wl.B, wl.H, max(self.nG, 1), dtype=torch.int32, device="cuda")
+
+    def kernel(self) -> str:
+        return self.plan.kernel(self.wl.L, self.wl.g, self.wl.w)
+
+    def step(self, k: int, g=None, w=None) -> None:
+        wl = self.wl
+        g = wl.g if g is None else g
+        w = wl.w if w is None else w
+        nG = (wl.L - w) // g if wl.L > w else 0
+        q_c, q_r, c_kv, k_r = self.dev[k % self.copies]
+        anc = self.anc if nG > 0 else None
+        if anc is not None and anc.shape[-1] < nG:
+            self.anc = self.torch.empty(wl.B, wl.H, nG, dtype=self.torch.int32, device="cuda")
+            anc = self.anc
+        self.plan.decode(q_c, q_r, c_kv, k_r, wl.L, g, w, self.out, anc, self.stream)
+
+    def dense(self, k: int) -> None:
+        q_c, q_r, c_kv, k_r = self.dev[k % self.copies]
+        self.plan.dense(q_c, q_r, c_kv, k_r, self.wl.L, self.out, self.stream)
+
+    def main_kernel_time(self, steps: int, g=None, w=None) -> list[float]:
+        """Per-step duration of the main kernel alone: an event recorded on the
+        launching stream before the step and, by the library, right after the
+        main-kernel launch (before the split combine)."""
+        torch = self.torch
+        ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for e in ev_m:
+            e.record(self.stream)
+        torch.cuda.synchronize()
+        for k in range(steps):
+            ev_s[k].record(self.stream)
+            self.plan.set_timing_event(ev_m[k])
+            self.step(k, g, w)
+        torch.cuda.synchronize()
+        self.plan.set_timing_event(None)
+        assert self.plan.device_error() == self.kvc.LCA_OK
+        return [ev_s[k].elapsed_time(ev_m[k]) * 1e-3 for k in range(steps)]
+
+    def free(self) -> None:
+        self.plan.close()
+        del self.dev, self.out, self.anc
+        self.torch.cuda.empty_cache()
+
+
+def timed_blocks(torch, runner, K: int, blocks: int, sync, fn=None) -> list[float]:
+    """`blocks` timed regions of exactly K back-to-back steps, each bracketed by
+    barrier + synchronize; returns each region's seconds (max over ranks is
+    taken by `sync`'s caller)."""
+    fn = fn or runner.step
+    times = []
+    for _ in range(blocks):
+        sync()
+        t = Timer(torch, runner.stream)
+        t.start()
+        for k in range(K):
+            fn(k)
+        times.append(t.stop())
+        sync()
+    return times
+
+
+def workload_fractions(wl, t_step: float, t_main: float, peaks: dict) -> dict:
+    alg = algorithmic_bytes(wl)
+    flops = algorithmic_flops(wl)
+    return {"ms_per_step": t_step * 1e3, "main_kernel_ms": t_main * 1e3,
+            "context_tokens_per_s": wl.B * wl.L / t_step,
+            "hbm_frac_whole_step": alg / t_step / 1e9 / peaks["hbm_gbs"],
+            "hbm_frac_main_kernel": alg / t_main / 1e9 / peaks["hbm_gbs"],
+            "tensor_frac_main_kernel": flops / t_main / 1e12 / peaks["bf16_tflops"]}
+
+
+def per_config(torch, kvc, stream, names: list[str], peaks: dict, steps: int) -> dict:
+    """Every other benchmark workload in the same process: whole-step and
+    main-kernel fractions (every (g, w) point of the sweep)."""
+    res = {}
+    for name in names:
+        wl = workloads.WORKLOADS[name]
+        r = Runner(torch, kvc, wl, stream)
+        points = list(wl.sweep) if wl.sweep else [(wl.g, wl.w)]
+        for (g, w) in points:
+            wlp = wl.with_(g=g, w=w)
+            key = name if not wl.sweep else f"{name} g={g} w={w}"
+            for k in range(3):
+                r.step(k, g, w)
+            torch.cuda.synchronize()
+            t = Timer(torch, stream)
+            blocks = []
+            for _ in range(3):
+                t.start()
+                for k in range(steps):
+                    r.step(k, g, w)
+                blocks.append(t.stop() / steps)
+            main = r.main_kernel_time(steps, g, w)
+            d = workload_fractions(wlp, statistics.median(blocks), statistics.mean(main), peaks)
+            d.update({"workload": workload_desc(wlp), "kernel": r.kernel() if not wl.sweep else
+                      r.plan.kernel(wl.L, g, w), "steps": steps, "blocks": 3})
+            res[key] = d
+        r.free()
+    return res
+
+
 def our_arm(args) -> None:
     import torch
     import kv_compression_b200 as kvc
@@ -319,29 +503,21 @@ def our_arm(args) -> None:
                                 device_id=torch.device("cuda", local))
 
     wl = rank_workload(with_point(workloads.WORKLOADS[args.workload], args), rank)
-    x = workloads.generate(wl)
-    cache_bytes = x.c_kv.nbytes + x.k_r.nbytes
-    copies = 1 if cache_bytes >= 4 * L2_BYTES else 2   # rotate copies so no step starts L2-warm
-    dev = [(to_device(x.q_c, torch), to_device(x.q_r, torch), to_device(x.c_kv, torch),
-            to_device(x.k_r, torch)) for _ in range(copies)]
-    plan = kvc.Plan(wl.B, wl.H, wl.d_c, wl.d_r, wl.dtype, wl.L)
-    kernel = plan.kernel(wl.L, wl.g, wl.w)
-    nG = wl.n_groups
-    out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32, device="cuda")
-    anc = torch.empty(wl.B, wl.H, max(nG, 1), dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
-
-    def step(k: int) -> None:
-        q_c, q_r, c_kv, k_r = dev[k % copies]
-        plan.decode(q_c, q_r, c_kv, k_r, wl.L, wl.g, wl.w, out, anc if nG > 0 else None, stream)
+    r = Runner(torch, kvc, wl, stream)
+    x = r.x
+    kernel = r.kernel()
+    nG = wl.n_groups
 
     props = torch.cuda.get_device_properties(local)
     uuid = ("GPU-" + str(props.uuid)) if getattr(props, "uuid", None) else None
     sampler = ClockSampler(uuid)
+    tw = Timer(torch, stream)
+    tw.start()
     for k in range(args.warmup):
-        step(k)
-    torch.cuda.synchronize()
-    assert plan.device_error() == kvc.LCA_OK
+        r.step(k)
+    t_warm = tw.stop() / max(args.warmup, 1)
+    assert r.plan.device_error() == kvc.LCA_OK
 
     K = args.steps
 
@@ -354,60 +530,37 @@ def our_arm(args) -> None:
     def rank_max(v: float) -> float:
         return max_over_ranks(dist, v, "cuda")
 
-    # Timed region: K back-to-back steps exactly as a caller issues them (no event
-    # between the main and the combine kernel, so the combine's programmatic
-    # dependent launch overlaps the main kernel's tail).
-    e_begin = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    nvml = NvmlSampler(uuid)
-    barrier_sync()
-    nvml.start()
-    e_begin.record(stream)
-    for k in range(K):
-        step(k)
-    e_end.record(stream)
-    torch.cuda.synchronize()
-    clocks = nvml.stop()
+    # Timed regions: blocks of K back-to-back steps exactly as a caller issues them
+    # (no event between the main and the combine kernel, so the combine's
+    # programmatic dependent launch overlaps the main kernel's tail).  Enough
+    # blocks for about half a second of timed work; the median block is reported.
+    blocks = args.blocks or int(min(200, max(5, math.ceil(0.5 / max(K * t_warm, 1e-6)))))
     if dist is not None:
-        dist.barrier()
-    t_total = rank_max(e_begin.elapsed_time(e_end) * 1e-3)
-    assert plan.device_error() == kvc.LCA_OK
+        blocks = int(rank_max(float(blocks)))      # every rank runs the same collective steps
+    nvml = NvmlSampler(uuid)
+    nvml.start()
+    block_s = timed_blocks(torch, r, K, blocks, barrier_sync)
+    clocks = nvml.stop()
+    block_s = [rank_max(t) for t in block_s]
+    t_total = statistics.median(block_s)
+    assert r.plan.device_error() == kvc.LCA_OK
 
-    # Second pass of K steps for the main kernel's own duration: an event recorded
-    # on the launching stream right after each main-kernel launch.
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    for e in ev_m:          # create the events so their handles exist
-        e.record(stream)
+    # The main kernel's own duration (its roofline): events on the launching stream
+    # around each main-kernel launch, over a second pass of K steps.
     barrier_sync()
-    for k in range(K):
-        ev_s[k].record(stream)
-        plan.set_timing_event(ev_m[k])
-        step(k)
-    torch.cuda.synchronize()
-    plan.set_timing_event(None)
-    main_ms = [ev_s[k].elapsed_time(ev_m[k]) for k in range(K)]
-    t_main = rank_max(statistics.mean(main_ms) * 1e-3)
-    assert plan.device_error() == kvc.LCA_OK
+    main_s = r.main_kernel_time(K)
+    t_main = rank_max(statistics.mean(main_s))
     clocks["nvidia_smi_whole_run"] = sampler.stop()
 
     # Dense MLA (mla_decode) on the same inputs: the same bytes, nothing condensed.
     kd = max(1, min(K, 200))
-    out_d = torch.empty_like(out)
-    ed0 = torch.cuda.Event(enable_timing=True)
-    ed1 = torch.cuda.Event(enable_timing=True)
     barrier_sync()
-    ed0.record(stream)
-    for k in range(kd):
-        q_c, q_r, c_kv, k_r = dev[k % copies]
-        plan.dense(q_c, q_r, c_kv, k_r, wl.L, out_d, stream)
-    ed1.record(stream)
-    torch.cuda.synchronize()
-    t_dense = rank_max(ed0.elapsed_time(ed1) * 1e-3)
-    assert plan.device_error() == kvc.LCA_OK
+    dense_s = [rank_max(t) for t in timed_blocks(torch, r, kd, 3, barrier_sync, fn=r.dense)]
+    t_dense = statistics.median(dense_s)
+    assert r.plan.device_error() == kvc.LCA_OK
 
     tokens_per_step = world * wl.B * wl.L
-    value = whole_job_rate(world, wl, K, t_total)
+    value = whole_job_rate(world, wl, K, t_total * 1.0)
     peaks, peak_kind = measured_peaks()
     alg = algorithmic_bytes(wl)
     achieved = alg / t_main / 1e9
@@ -422,87 +575,112 @@ def our_arm(args) -> None:
         hq_c, hq_r, hc, hk = pinned(x.q_c), pinned(x.q_r), pinned(x.c_kv), pinned(x.k_r)
         h_out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32).pin_memory()
         h_anc = torch.empty(wl.B, wl.H, max(nG, 1), dtype=torch.int32).pin_memory()
-        ke = max(1, min(K, 30))
-        plan.decode_host(hq_c, hq_r, hc, hk, wl.L, wl.g, wl.w, h_out, h_anc if nG > 0 else None, stream)
-        if dist is not None:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(stream)
+        ke = max(1, min(K, 10))
+        r.plan.decode_host(hq_c, hq_r, hc, hk, wl.L, wl.g, wl.w, h_out, h_anc if nG > 0 else None,
+                           stream)
+        barrier_sync()
+        te_t = Timer(torch, stream)
+        te_t.start()
         for _ in range(ke):
-            plan.decode_host(hq_c, hq_r, hc, hk, wl.L, wl.g, wl.w, h_out,
-                             h_anc if nG > 0 else None, stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        te = rank_max(e0.elapsed_time(e1) * 1e-3)
+            r.plan.decode_host(hq_c, hq_r, hc, hk, wl.L, wl.g, wl.w, h_out,
+                               h_anc if nG > 0 else None, stream)
+        te = rank_max(te_t.stop())
         h2d = hq_c.numel() * hq_c.element_size() + hq_r.numel() * hq_r.element_size() + \
             hc.numel() * hc.element_size() + hk.numel() * hk.element_size()
         d2h = h_out.numel() * 4 + (wl.B * wl.H * nG * 4)
         e2e = {"value": tokens_per_step * ke / te, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": ke,
                "path": "lca_decode_host (pinned host buffers; copies inside the timed region)"}
+        del hq_c, hq_r, hc, hk
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import oracle
         nthreads = os.cpu_count() or 1
-        res = oracle.lca(x.q_c, x.q_r, x.c_kv, x.k_r, g=wl.g, w=wl.w, nthreads=nthreads)
-        cpu = {"value": wl.B * wl.L / res.seconds, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-               "sample": f"the whole batch ({wl.B} sequences x {wl.H} heads, L={wl.L}) once, "
+        rows = sorted({0, wl.B - 1})
+        res = oracle.lca(x.q_c, x.q_r, x.c_kv, x.k_r, g=wl.g, w=wl.w, rows=rows, nthreads=nthreads)
+        cpu = {"value": len(rows) * wl.L / res.seconds, "unit": UNIT, "cores": nthreads,
+               "kind": "oracle",
+               "sample": f"sequences {rows} of the batch ({len(rows)} x {wl.H} heads, L={wl.L}), "
                          f"oracle formulation A, {res.seconds:.1f} s"}
+
+    head_kernel = kernel
+    r.free()
+    del r, x
+    pc = None
+    if rank == 0 and world == 1 and not args.no_per_config:
+        others = [n for n in ("v2lite", "v2", "needle", "sweep", "tiny_f32") if n != args.workload]
+        pc = per_config(torch, kvc, stream, others, peaks, max(5, min(K, 50)))
 
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
+    tc_peak_s = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": t_total / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "data": "synthetic (seeded, workloads/)",
-        "config": {"workload": workload_desc(wl), "kernel": kernel, "parallelism": f"replicas x{world}",
-                   "l2": (f"inputs {cache_bytes / 1e6:.0f} MB per step > 126 MB L2; "
-                          f"{copies} copies rotated, no flush"),
+        "config": {"workload": workload_desc(wl), "kernel": head_kernel, "parallelism": f"replicas x{world}",
+                   "l2": (f"inputs {r_cache_mb(wl):.0f} MB per step > 126 MB L2; "
+                          f"{1 if r_cache_mb(wl) * 1e6 >= 4 * L2_BYTES else 2} copies rotated, no flush"),
+                   "timed_blocks": blocks, "block_ms": [t * 1e3 for t in block_s],
                    "hbm_gbs_whole_step": alg / (t_total / K) / 1e9,
                    "hbm_frac_whole_step": alg / (t_total / K) / 1e9 / peaks["hbm_gbs"]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "kernel": "lca_tc_kernel" if kernel == "tcgen05" else "lca_simt_kernel",
+                     "kernel": MAIN_KERNEL_NAMES.get(head_kernel, head_kernel),
                      "algorithmic_bytes_per_launch": alg, "launch_ms": t_main * 1e3,
-                     "launch_ms_min": min(main_ms), "launch_ms_max": max(main_ms),
+                     "launch_ms_min": min(main_s) * 1e3, "launch_ms_max": max(main_s) * 1e3,
                      "timing": "CUDA events on the launching stream around each main-kernel launch, "
                                "mean over a second pass of K steps",
                      "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                      "flops_per_launch": flops, "achieved_tflops": flops / t_main / 1e12,
                      "tensor_frac": flops / t_main / 1e12 / peaks["bf16_tflops"],
-                     "tensor_peak_kind": f"{peak_kind} bf16_tflops (cuBLAS burst)"},
+                     "tensor_frac_sustained": flops / t_main / 1e12 / tc_peak_s,
+                     "tensor_peak_kind": f"{peak_kind} bf16_tflops (cuBLAS burst; sustained beside it)"},
         "mla_decode": {"value": whole_job_rate(world, wl, kd, t_dense), "unit": UNIT,
                        "ms_per_step": t_dense / kd * 1e3, "steps": kd,
                        "hbm_frac": alg / (t_dense / kd) / 1e9 / peaks["hbm_gbs"],
                        "note": "dense MLA decode over the same cache (same bytes), same kernels with n_G = 0"},
+        "per_config": pc,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 2 * K,
-        "gpu_launches_note": "timed region: main + combine per step; the instrumented and dense passes are outside it",
+        "gpu_launches_note": "per timed block of K steps: main + combine per step; the instrumented, "
+                             "dense, e2e and per-config passes are outside the timed blocks",
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
 
 
+def r_cache_mb(wl: workloads.Workload) -> float:
+    return wl.B * wl.L * (wl.d_c + wl.d_r) * wl.elem_bytes / 1e6
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="v2lite", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--blocks", type=int, default=0,
+                    help="timed blocks of --steps steps (0: enough for about 0.5 s)")
+    ap.add_argument("--impl", choices=["ours", "reference", "ranks"], default="ours")
+    ap.add_argument("--workload", default="v2", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--g", type=int, default=None, help="group size (default: the workload's)")
     ap.add_argument("--w", type=int, default=None, help="window (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     args = ap.parse_args()
+    rc = spawn_ranks(args)
+    if rc is not None:
+        sys.exit(rc)
     if args.impl == "reference":
         reference_arm(args)
+    elif args.impl == "ranks":
+        ranks_arm(args)
     else:
         our_arm(args)
 

@@ -100,8 +100,24 @@ def test_reference_arm_prints_the_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
-    assert d["config"]["workload"].startswith("v2lite")
+    assert d["config"]["workload"].startswith("v2:")
+    assert d["n_gpus"] == 1
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` without torchrun launches two local ranks itself
+    (here the CPU stand-in arm over gloo); both join and rank 0 reports the
+    world size it saw."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "ranks", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and sorted(d["ranks"]) == [0, 1] and d["t_max"] == 2.0
