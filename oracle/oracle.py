@@ -48,6 +48,12 @@ def _load(path: str) -> ctypes.CDLL:
     lib.mla_oracle_seq.restype = i32
     lib.lca_oracle_num_groups.argtypes = [i64, i32, i32]
     lib.lca_oracle_num_groups.restype = i64
+    lib.lca_oracle_condense_shared.argtypes = [i32, i32, i32, i64, i32, i64, i64, i32, vp, vp, vp,
+                                               vp, dp, dp, vp, dp, dp]
+    lib.lca_oracle_condense_shared.restype = i32
+    lib.lca_oracle_decode_stored.argtypes = [i32, i32, i32, i64, i64, i32, vp, vp, dp, dp, vp, vp,
+                                             ctypes.c_double, dp]
+    lib.lca_oracle_decode_stored.restype = i32
     return lib
 
 
@@ -149,3 +155,91 @@ def mla(q_c, q_r, c_kv, k_r, rows=None, nthreads: int = 0,
             raise RuntimeError(f"mla_oracle_seq failed with status {st}")
         out[i] = o
     return out
+
+
+@dataclass
+class StoredResult:
+    """The stored, head-shared condensed cache of one batch and its decode."""
+    cbar: np.ndarray         # [nb, n_G, d_c] float64: pooled latents
+    kanc: np.ndarray         # [nb, n_G, d_r] float64: the anchors' RoPE keys
+    anchor: np.ndarray       # [nb, n_G] int32 absolute positions
+    tie_gap: np.ndarray      # [nb, n_G] float64: top-2 gap of the head-mean score
+    max_abs_s: np.ndarray    # [nb] float64: max |head-mean score| over condensed tokens
+    out: np.ndarray | None   # [nb, H, d_c] float64: decode over [stored || window]
+    rows: list[int]
+
+
+def condense_shared(q_c, q_r, c_kv, k_r, g: int, j0: int, n: int, rows=None,
+                    lib: ctypes.CDLL | None = None):
+    """Condense groups j0 .. j0+n-1 of every sequence in ``rows`` with the
+    head-mean score of q (one entry per group, shared by all heads).
+    Returns (cbar [nb,n,d_c], kanc [nb,n,d_r], anchor [nb,n], tie_gap [nb,n], max_abs [nb])."""
+    lib = lib or load()
+    B, H, d_c = q_c.shape
+    d_r = q_r.shape[2]
+    L = c_kv.shape[1]
+    dt = _dtype_code(q_c)
+    rows = list(range(B)) if rows is None else list(rows)
+    cb = np.zeros((len(rows), n, d_c), np.float64)
+    ka = np.zeros((len(rows), n, d_r), np.float64)
+    an = np.zeros((len(rows), max(n, 1)), np.int32)
+    gp = np.zeros((len(rows), max(n, 1)), np.float64)
+    mx = np.zeros((len(rows),), np.float64)
+    for i, b in enumerate(rows):
+        qc = np.ascontiguousarray(q_c[b]); qr = np.ascontiguousarray(q_r[b])
+        ck = np.ascontiguousarray(c_kv[b]); kr = np.ascontiguousarray(k_r[b])
+        c1 = np.zeros((max(n, 1), d_c)); k1 = np.zeros((max(n, 1), max(d_r, 1)))
+        a1 = np.zeros((max(n, 1),), np.int32); g1 = np.zeros((max(n, 1),)); m1 = np.zeros((1,))
+        st = lib.lca_oracle_condense_shared(H, d_c, d_r, L, g, j0, n, dt, _ptr(qc), _ptr(qr), _ptr(ck),
+                                            _ptr(kr), _ptr(c1), _ptr(k1), _ptr(a1), _ptr(g1), _ptr(m1))
+        if st != 0:
+            raise RuntimeError(f"lca_oracle_condense_shared failed with status {st}")
+        cb[i] = c1[:n]; ka[i] = k1[:n, :d_r]; an[i] = a1; gp[i] = g1; mx[i] = m1[0]
+    return cb, ka, an[:, :n], gp[:, :n], mx
+
+
+def decode_stored(q_c, q_r, cbar, kanc, c_win, k_win, bias: float = 0.0, rows=None,
+                  lib: ctypes.CDLL | None = None) -> np.ndarray:
+    """Softmax attention of q over [stored condensed entries || window tokens].
+    q_c [B,H,d_c], q_r [B,H,d_r] stored values; cbar [nb,n,d_c], kanc [nb,n,d_r]
+    float64 (one row per sequence in ``rows``); c_win [B,n_win,d_c], k_win
+    [B,n_win,d_r] stored values; ``bias`` added to condensed logits."""
+    lib = lib or load()
+    B, H, d_c = q_c.shape
+    d_r = q_r.shape[2]
+    dt = _dtype_code(q_c)
+    rows = list(range(B)) if rows is None else list(rows)
+    n = cbar.shape[1]
+    n_win = c_win.shape[1]
+    out = np.zeros((len(rows), H, d_c), np.float64)
+    for i, b in enumerate(rows):
+        qc = np.ascontiguousarray(q_c[b]); qr = np.ascontiguousarray(q_r[b])
+        cb = np.ascontiguousarray(cbar[i], dtype=np.float64)
+        ka = np.ascontiguousarray(kanc[i], dtype=np.float64)
+        cw = np.ascontiguousarray(c_win[b]); kw = np.ascontiguousarray(k_win[b])
+        o = np.zeros((H, d_c), np.float64)
+        st = lib.lca_oracle_decode_stored(H, d_c, d_r, n, n_win, dt, _ptr(qc), _ptr(qr),
+                                          _ptr(cb) if n else None, _ptr(ka) if n else None,
+                                          _ptr(cw) if n_win else None, _ptr(kw) if n_win else None,
+                                          float(bias), _ptr(o))
+        if st != 0:
+            raise RuntimeError(f"lca_oracle_decode_stored failed with status {st}")
+        out[i] = o
+    return out
+
+
+def lca_stored(q_cond, q_r_cond, c_kv, k_r, g: int, w: int, q_c=None, q_r=None, bias: float = 0.0,
+               rows=None, lib: ctypes.CDLL | None = None) -> StoredResult:
+    """The whole stored-cache path for one batch: condense every group (n_G of
+    them, the section-2 segmentation) with the query (q_cond, q_r_cond), then
+    decode the query (q_c, q_r) -- by default the same one -- over [stored ||
+    window], the window being tokens [n_G g, L)."""
+    lib = lib or load()
+    L = c_kv.shape[1]
+    nG = num_groups(L, g, w, lib)
+    rows = list(range(q_cond.shape[0])) if rows is None else list(rows)
+    cb, ka, an, gp, mx = condense_shared(q_cond, q_r_cond, c_kv, k_r, g, 0, nG, rows, lib)
+    q_c = q_cond if q_c is None else q_c
+    q_r = q_r_cond if q_r is None else q_r
+    out = decode_stored(q_c, q_r, cb, ka, c_kv[:, nG * g:], k_r[:, nG * g:], bias, rows, lib)
+    return StoredResult(cb, ka, an, gp, mx, out, rows)

@@ -324,6 +324,133 @@ def pin_constant_rope(lib):
     assert np.array_equal(a.anchor, b.anchor)
 
 
+# ----------------------------------------------------------------------------- stored cache
+def torch_stored_seq(qc_cond, qr_cond, C, K, g, w, qc=None, qr=None, bias=0.0):
+    """The stored, head-shared condensed cache of one sequence built from
+    library routines: head-mean score (torch.mean over heads), group softmax
+    and argmax, pooled latent by matmul, then softmax attention with explicit
+    logits (the bias added to the condensed entries).  Returns (out [H, d_c],
+    anchor [n_G], cbar [n_G, d_c], gap [n_G], max |s_bar|)."""
+    groups, window = partition(C.shape[0], g, w)
+    Ct, Kt = torch.from_numpy(C), torch.from_numpy(K)
+    qcc, qrc = torch.from_numpy(qc_cond), torch.from_numpy(qr_cond)
+    s_heads = Ct @ qcc.T + Kt @ qrc.T                  # [L, H]
+    sbar = s_heads.mean(dim=1)                         # the head-mean score
+    keys, vals, anc, gaps, cbars, is_cond = [], [], [], [], [], []
+    amax = 0.0
+    for G in groups:
+        idx = torch.tensor(G)
+        sg = sbar[idx]
+        amax = max(amax, float(sg.abs().max()))
+        wts = torch.softmax(sg, dim=0)
+        a = G[int(torch.argmax(sg))]
+        gaps.append(float(torch.topk(sg, 2).values[0] - torch.topk(sg, 2).values[1]) if len(G) > 1
+                    else math.inf)
+        cbar = wts @ Ct[idx]
+        keys.append(torch.cat([cbar, Kt[a]])); vals.append(cbar); anc.append(a); cbars.append(cbar)
+        is_cond.append(True)
+    for t in window:
+        keys.append(torch.cat([Ct[t], Kt[t]])); vals.append(Ct[t]); is_cond.append(False)
+    qc = qc_cond if qc is None else qc
+    qr = qr_cond if qr is None else qr
+    q = torch.from_numpy(np.concatenate([qc, qr], axis=1))          # [H, d]
+    Kmat, Vmat = torch.stack(keys), torch.stack(vals)
+    logits = q @ Kmat.T + bias * torch.tensor(is_cond, dtype=torch.float64)[None, :]
+    out = torch.softmax(logits, dim=1) @ Vmat
+    cb = torch.stack(cbars).numpy() if cbars else np.zeros((0, C.shape[1]))
+    return out.numpy(), np.array(anc, np.int32), cb, np.array(gaps), amax
+
+
+def pin_stored_brute_force(lib):
+    rng = np.random.default_rng(30)
+    for dtype in ("f32", "bf16"):
+        for L in (1, 3, 8, 13):
+            qc, qr, C, K = rand_inputs(rng, 1, 3, L, 8, 4, dtype)
+            qc2, qr2, _, _ = rand_inputs(rng, 1, 3, L, 8, 4, dtype)
+            for g in range(1, L + 2):
+                for w in range(0, L + 2, 2):
+                    for bias in (0.0, math.log(g)):
+                        # condense with one query, decode with another
+                        res = orc.lca_stored(qc, qr, C, K, g, w, q_c=qc2, q_r=qr2, bias=bias, lib=lib)
+                        out, anc, cb, gap, amax = torch_stored_seq(
+                            widen(qc[0]), widen(qr[0]), widen(C[0]), widen(K[0]), g, w,
+                            widen(qc2[0]), widen(qr2[0]), bias)
+                        where = (dtype, L, g, w, bias)
+                        assert rel_err(res.out[0], out) < REL_TOL, where
+                        assert np.array_equal(res.anchor[0], anc), where
+                        if len(anc):
+                            assert rel_err(res.cbar[0], cb) < REL_TOL, where
+                            assert np.allclose(res.kanc[0], widen(K[0])[anc], rtol=0, atol=0), where
+                            fin = np.isfinite(gap)
+                            assert np.array_equal(np.isfinite(res.tie_gap[0]), fin), where
+                            assert np.all(np.abs(res.tie_gap[0][fin] - gap[fin]) <= 1e-12 * max(amax, 1)), where
+                            assert abs(res.max_abs_s[0] - amax) <= 1e-12 * max(amax, 1), where
+
+
+def pin_stored_g1_dense(lib):
+    """g = 1: every stored entry is a token itself, so decode over the stored
+    cache is dense MLA attention (torch SDPA)."""
+    rng = np.random.default_rng(31)
+    qc, qr, C, K = rand_inputs(rng, 2, 3, 29, 16, 8, "bf16")
+    for w in (0, 4, 29):
+        res = orc.lca_stored(qc, qr, C, K, 1, w, lib=lib)
+        for b in range(2):
+            ref = torch_dense_seq(widen(qc[b]), widen(qr[b]), widen(C[b]), widen(K[b]))
+            assert rel_err(res.out[b], ref) < REL_TOL
+            assert list(res.anchor[b]) == list(range(res.anchor.shape[1]))
+
+
+def pin_stored_single_head(lib):
+    """H = 1 and the same query for condensing and decoding: the head mean is
+    that head's score, so the stored path is the per-head LCA decode."""
+    rng = np.random.default_rng(32)
+    for (L, g, w) in ((70, 8, 9), (64, 16, 0), (33, 4, 40)):
+        qc, qr, C, K = rand_inputs(rng, 2, 1, L, 16, 8)
+        res = orc.lca_stored(qc, qr, C, K, g, w, lib=lib)
+        ref = orc.lca(qc, qr, C, K, g=g, w=w, lib=lib)
+        assert rel_err(res.out, ref.out) < REL_TOL
+        assert np.array_equal(res.anchor, ref.anchor[:, 0])
+
+
+def pin_stored_constant_groups(lib):
+    """Groups of identical tokens: each stored entry is that token.  Without a
+    bias the decode is dense attention over one representative per group;
+    with bias log g each entry counts as its g tokens, which is exactly dense
+    attention over all L tokens."""
+    rng = np.random.default_rng(33)
+    L, g, w, H = 34, 4, 5, 3
+    groups, window = partition(L, g, w)
+    qc, qr, C, K = rand_inputs(rng, 1, H, L, 16, 8)
+    reps = []
+    for G in groups:
+        C[0, G] = C[0, G[0]]; K[0, G] = K[0, G[0]]; reps.append(G[0])
+    res0 = orc.lca_stored(qc, qr, C, K, g, w, lib=lib)
+    keep = reps + window
+    ref0 = torch_dense_seq(widen(qc[0]), widen(qr[0]), widen(C[0][keep]), widen(K[0][keep]))
+    assert rel_err(res0.out[0], ref0) < REL_TOL
+    assert list(res0.anchor[0]) == reps
+    res1 = orc.lca_stored(qc, qr, C, K, g, w, bias=math.log(g), lib=lib)
+    ref1 = torch_dense_seq(widen(qc[0]), widen(qr[0]), widen(C[0]), widen(K[0]))
+    assert rel_err(res1.out[0], ref1) < REL_TOL
+
+
+def pin_stored_zero_query(lib):
+    """A zero condensing query: uniform pooling (c_bar = the group mean) and
+    the first token of each group as anchor."""
+    rng = np.random.default_rng(34)
+    _, _, C, K = rand_inputs(rng, 1, 2, 40, 16, 8)
+    qz, qrz = np.zeros((1, 2, 16), np.float32), np.zeros((1, 2, 8), np.float32)
+    cb, ka, an, gap, mx = orc.condense_shared(qz, qrz, C, K, 5, 1, 6, lib=lib)
+    for jj in range(6):
+        j = 1 + jj
+        assert rel_err(cb[0, jj][None], widen(C[0, 5 * j:5 * j + 5]).mean(axis=0)[None]) < REL_TOL
+        assert an[0, jj] == 5 * j
+        assert np.array_equal(ka[0, jj], widen(K[0, 5 * j]))
+
+
+STORED_PINS = [pin_stored_brute_force, pin_stored_g1_dense, pin_stored_single_head,
+               pin_stored_constant_groups, pin_stored_zero_query]
+
 ALL_PINS = [pin_segmentation, pin_dense_vs_torch, pin_g1_dense, pin_window_dense, pin_zero_query,
             pin_constant_groups, pin_brute_force, pin_near_tie_report, pin_ties, pin_formulations,
-            pin_permutation, pin_constant_rope]
+            pin_permutation, pin_constant_rope] + STORED_PINS

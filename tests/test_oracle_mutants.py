@@ -55,6 +55,19 @@ MUTANTS = {
     # near-tie report: runner-up excludes the group's first token, not the anchor
     "tie_gap_wrong_token": ("if (t != a && w->s[t] > second) second = w->s[t];",
                             "if (t != t0 && w->s[t] > second) second = w->s[t];"),
+    # stored cache: sum over heads instead of the mean (a different temperature)
+    "stored_sum_not_mean": ("sbar[u] /= (double)H;", "sbar[u] /= 1.0;"),
+    # stored cache: the bias on condensed logits with the wrong sign
+    "stored_bias_sign": ("double l = bias;", "double l = -bias;"),
+    # stored cache: ties go to the highest index
+    "stored_tie_break_highest": ("if (sbar[u] > m) { m = sbar[u]; a = u; }",
+                                 "if (sbar[u] >= m) { m = sbar[u]; a = u; }"),
+    # stored cache: the pooled latent reads the group's first row only
+    "stored_pool_first_row": ("cb[i] += wt * elem(c_kv, (t0 + u) * (int64_t)d_c + i, dtype);",
+                              "cb[i] += wt * elem(c_kv, (t0) * (int64_t)d_c + i, dtype);"),
+    # stored cache: the anchor key from the group's first token
+    "stored_anchor_key_first": ("kanc[jj * (int64_t)d_r + i] = elem(k_r, (t0 + a) * (int64_t)d_r + i, dtype);",
+                                "kanc[jj * (int64_t)d_r + i] = elem(k_r, (t0) * (int64_t)d_r + i, dtype);"),
 }
 
 
@@ -77,7 +90,7 @@ def test_mutant_is_caught(name, oracle_src, tmp_path):
     for pin in pins.ALL_PINS:
         try:
             pin(lib)
-        except AssertionError:
+        except (AssertionError, RuntimeError):   # a wrong value, or the oracle refusing its own output
             failures.append(pin.__name__)
     assert failures, f"mutant {name} passed every pin"
 
