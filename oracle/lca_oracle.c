@@ -491,3 +491,104 @@ int lca_oracle_decode_stored(int H, int d_c, int d_r, int64_t n_cond, int64_t n_
     free(qc); free(qr); free(ell);
     return 0;
 }
+
+/*
+ * Context sharding: the entries of one sequence ([condensed groups || window],
+ * section 2 steps 1-3 for the whole context of L_total tokens) are split by
+ * position among several holders -- one slice of tokens [pos0, pos0 + n_tok)
+ * each, cut on group boundaries inside the condensed part -- and each holder
+ * computes the partial softmax sums of the entries it holds:
+ *   M = max_e logit_e,  Z = sum_e exp(logit_e - M),  O = sum_e exp(logit_e - M) value_e,
+ * over its condensed groups (all g tokens inside the slice) and window tokens.
+ * The partials merge exactly (the online-softmax merge of the Pulsar Attention
+ * page, "Fase 2"): M* = max M_i, out = sum_i e^{M_i - M*} O_i / sum_i e^{M_i - M*} Z_i.
+ * An empty slice gives M = -inf, Z = 0, O = 0.
+ *
+ * One (sequence, head): the whole cache c_kv [L_total][d_c], k_r [L_total][d_r]
+ * is passed and only rows of the slice are read.  Writes m [1], z [1], o [d_c]
+ * and the anchors of the slice's groups (anchor [n_slice_groups], absolute).
+ * Returns 0, -1 when the slice cuts a group, -2 on allocation failure.
+ */
+int lca_oracle_partial(int d_c, int d_r, int64_t L_total, int g, int w_win, int64_t pos0,
+                       int64_t n_tok, int dtype, const void *q_c, const void *q_r,
+                       const void *c_kv, const void *k_r, double *m, double *z, double *o,
+                       int32_t *anchor)
+{
+    const int64_t nG = lca_oracle_num_groups(L_total, g, w_win);
+    const int64_t win0 = nG * g;
+    const int64_t end = pos0 + n_tok;
+    if (pos0 < 0 || n_tok < 0 || end > L_total || g < 1 ||
+        (pos0 < win0 && pos0 % g != 0) || (end < win0 && end % g != 0))
+        return -1;
+    scratch_t w;
+    if (scratch_alloc(&w, d_c, d_r, L_total, nG) != 0) {
+        scratch_free(&w);
+        return -2;
+    }
+    for (int i = 0; i < d_c; ++i) w.qc[i] = elem(q_c, i, dtype);
+    for (int i = 0; i < d_r; ++i) w.qr[i] = elem(q_r, i, dtype);
+    /* scores of the slice's tokens only */
+    for (int64_t t = pos0; t < end; ++t) {
+        w.sc[t] = dot_row(w.qc, c_kv, t, d_c, dtype);
+        w.sr[t] = dot_row(w.qr, k_r, t, d_r, dtype);
+        w.s[t] = w.sc[t] + w.sr[t];
+    }
+    const int64_t j_lo = pos0 < win0 ? pos0 / g : nG;          /* groups inside the slice */
+    const int64_t j_hi = end < win0 ? end / g : nG;
+    int64_t ne = 0;
+    for (int64_t j = j_lo; j < j_hi; ++j) {                      /* step 2 per group */
+        const int64_t t0 = j * g;
+        double mx = w.s[t0];
+        int64_t a = t0;
+        for (int64_t t = t0 + 1; t < t0 + g; ++t)
+            if (w.s[t] > mx) { mx = w.s[t]; a = t; }
+        double den = 0.0;
+        for (int64_t t = t0; t < t0 + g; ++t) den += exp(w.s[t] - mx);
+        w.gmax[j] = mx;
+        w.gden[j] = den;
+        w.ganc[j] = (int32_t)a;
+        if (anchor) anchor[j - j_lo] = (int32_t)a;
+        pooled_latent(&w, c_kv, d_c, dtype, g, j, w.cbar);
+        double l = 0.0;
+        for (int i = 0; i < d_c; ++i) l += w.qc[i] * w.cbar[i];
+        w.ell[ne++] = l + dot_row(w.qr, k_r, a, d_r, dtype);
+    }
+    const int64_t wlo = pos0 > win0 ? pos0 : win0;               /* window tokens inside */
+    for (int64_t t = wlo; t < end; ++t) w.ell[ne++] = w.s[t];
+    double M = -INFINITY;
+    for (int64_t e = 0; e < ne; ++e) if (w.ell[e] > M) M = w.ell[e];
+    double Z = 0.0;
+    for (int i = 0; i < d_c; ++i) o[i] = 0.0;
+    int64_t e = 0;
+    for (int64_t j = j_lo; j < j_hi; ++j, ++e) {
+        const double p = exp(w.ell[e] - M);
+        Z += p;
+        pooled_latent(&w, c_kv, d_c, dtype, g, j, w.cbar);
+        for (int i = 0; i < d_c; ++i) o[i] += p * w.cbar[i];
+    }
+    for (int64_t t = wlo; t < end; ++t, ++e) {
+        const double p = exp(w.ell[e] - M);
+        Z += p;
+        for (int i = 0; i < d_c; ++i) o[i] += p * elem(c_kv, t * (int64_t)d_c + i, dtype);
+    }
+    *m = M;
+    *z = Z;
+    scratch_free(&w);
+    return 0;
+}
+
+/* Merge n partials (m [n], z [n], o [n][d_c]) into out [d_c]. */
+void lca_oracle_merge(int n, int d_c, const double *m, const double *z, const double *o, double *out)
+{
+    double M = -INFINITY;
+    for (int i = 0; i < n; ++i) if (m[i] > M) M = m[i];
+    double Z = 0.0;
+    for (int k = 0; k < d_c; ++k) out[k] = 0.0;
+    for (int i = 0; i < n; ++i) {
+        if (m[i] == -INFINITY) continue;                         /* an empty slice */
+        const double f = exp(m[i] - M);
+        Z += f * z[i];
+        for (int k = 0; k < d_c; ++k) out[k] += f * o[(int64_t)i * d_c + k];
+    }
+    for (int k = 0; k < d_c; ++k) out[k] /= Z;
+}

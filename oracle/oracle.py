@@ -54,6 +54,11 @@ def _load(path: str) -> ctypes.CDLL:
     lib.lca_oracle_decode_stored.argtypes = [i32, i32, i32, i64, i64, i32, vp, vp, dp, dp, vp, vp,
                                              ctypes.c_double, dp]
     lib.lca_oracle_decode_stored.restype = i32
+    lib.lca_oracle_partial.argtypes = [i32, i32, i64, i32, i32, i64, i64, i32, vp, vp, vp, vp, dp, dp,
+                                       dp, vp]
+    lib.lca_oracle_partial.restype = i32
+    lib.lca_oracle_merge.argtypes = [i32, i32, dp, dp, dp, dp]
+    lib.lca_oracle_merge.restype = None
     return lib
 
 
@@ -243,3 +248,56 @@ def lca_stored(q_cond, q_r_cond, c_kv, k_r, g: int, w: int, q_c=None, q_r=None, 
     q_r = q_r_cond if q_r is None else q_r
     out = decode_stored(q_c, q_r, cb, ka, c_kv[:, nG * g:], k_r[:, nG * g:], bias, rows, lib)
     return StoredResult(cb, ka, an, gp, mx, out, rows)
+
+
+def slice_groups(L: int, g: int, w: int, pos0: int, n_tok: int, lib: ctypes.CDLL | None = None) -> int:
+    """Condensed groups that lie inside tokens [pos0, pos0 + n_tok)."""
+    nG = num_groups(L, g, w, lib)
+    win0 = nG * g
+    lo = pos0 // g if pos0 < win0 else nG
+    hi = (pos0 + n_tok) // g if pos0 + n_tok < win0 else nG
+    return max(0, hi - lo)
+
+
+def partial(q_c, q_r, c_kv, k_r, g: int, w: int, pos0: int, n_tok: int, rows=None,
+            lib: ctypes.CDLL | None = None):
+    """Partial softmax sums (M, Z, O) of the entries held by tokens [pos0,
+    pos0 + n_tok) of the whole context c_kv [B,L,d_c]; returns (m [nb,H],
+    z [nb,H], o [nb,H,d_c], anchor [nb,H,n_slice_groups])."""
+    lib = lib or load()
+    B, H, d_c = q_c.shape
+    d_r = q_r.shape[2]
+    L = c_kv.shape[1]
+    dt = _dtype_code(q_c)
+    rows = list(range(B)) if rows is None else list(rows)
+    ng = slice_groups(L, g, w, pos0, n_tok, lib)
+    m = np.zeros((len(rows), H)); z = np.zeros((len(rows), H)); o = np.zeros((len(rows), H, d_c))
+    an = np.zeros((len(rows), H, max(ng, 1)), np.int32)
+    esz = 4 if dt == F32 else 2
+    for i, b in enumerate(rows):
+        ck = np.ascontiguousarray(c_kv[b]); kr = np.ascontiguousarray(k_r[b])
+        for h in range(H):
+            qc = np.ascontiguousarray(q_c[b, h]); qr = np.ascontiguousarray(q_r[b, h])
+            mm = np.zeros(1); zz = np.zeros(1); oo = np.zeros(d_c); aa = np.zeros(max(ng, 1), np.int32)
+            st = lib.lca_oracle_partial(d_c, d_r, L, g, w, pos0, n_tok, dt, _ptr(qc), _ptr(qr), _ptr(ck),
+                                        _ptr(kr), _ptr(mm), _ptr(zz), _ptr(oo), _ptr(aa))
+            if st != 0:
+                raise RuntimeError(f"lca_oracle_partial failed with status {st} (slice cuts a group?)")
+            m[i, h], z[i, h], o[i, h], an[i, h] = mm[0], zz[0], oo, aa
+    del esz
+    return m, z, o, an[:, :, :ng]
+
+
+def merge(ms, zs, os_, lib: ctypes.CDLL | None = None) -> np.ndarray:
+    """Merge stacked partials ms [n,nb,H], zs [n,nb,H], os_ [n,nb,H,d_c] -> out [nb,H,d_c]."""
+    lib = lib or load()
+    ms, zs, os_ = (np.asarray(a, np.float64) for a in (ms, zs, os_))
+    n, nb, H, d_c = os_.shape
+    out = np.zeros((nb, H, d_c))
+    for b in range(nb):
+        for h in range(H):
+            m = np.ascontiguousarray(ms[:, b, h]); z = np.ascontiguousarray(zs[:, b, h])
+            o = np.ascontiguousarray(os_[:, b, h]); r = np.zeros(d_c)
+            lib.lca_oracle_merge(n, d_c, _ptr(m), _ptr(z), _ptr(o), _ptr(r))
+            out[b, h] = r
+    return out
