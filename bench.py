@@ -42,10 +42,11 @@ import workloads  # noqa: E402
 METRIC = "LCA decode context tokens/s per GPU; HBM GB/s as % of B200 peak"
 UNIT = "context tokens/s"
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCES = ["kv_compression_b200/csrc/tc_kernel.cuh", "kv_compression_b200/csrc/ptx.cuh"]
+KERNEL_SOURCES = ["kv_compression_b200/csrc/tc_kernel.cuh", "kv_compression_b200/csrc/pair_kernel.cuh",
+                  "kv_compression_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = "profiles/lca_tc_kernel_v2lite_traffic.txt"
 TRAFFIC_WORKLOAD = "v2lite"           # the workload that capture ran on
-MAIN_KERNEL_NAMES = {"tcgen05": "lca_tc_kernel", "simt": "lca_simt_kernel"}
+MAIN_KERNEL_NAMES = {"tcgen05": "lca_tc_kernel", "tcgen05_pair": "lca_pair_kernel", "simt": "lca_simt_kernel"}
 
 
 def workload_desc(wl: workloads.Workload) -> str:
@@ -282,6 +283,8 @@ def with_point(wl: workloads.Workload, args) -> workloads.Workload:
         wl = wl.with_(g=args.g)
     if args.w is not None:
         wl = wl.with_(w=args.w)
+    if getattr(args, "batch", None):
+        wl = wl.with_(B=args.batch)
     return wl
 
 
@@ -447,6 +450,65 @@ def timed_blocks(torch, runner, K: int, blocks: int, sync, fn=None) -> list[floa
     return times
 
 
+def stored_leg(torch, kvc, r, K: int, peaks: dict, t_lca: float, t_mla: float) -> dict:
+    """The stored, head-shared condensed cache on the same inputs: build it once
+    from the full cache (condense every group with this step's query, copy the
+    window), then decode over the n_G + |W| stored rows.  Enough copies of the
+    stored cache rotate that every step reads it from HBM."""
+    wl = r.wl
+    R = kvc.stored_rows(wl.L, wl.g, wl.w)
+    nG = wl.n_groups
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    row_bytes = (wl.d_c + wl.d_r) * wl.elem_bytes
+    store_bytes = wl.B * R * row_bytes
+    copies = int(min(20, max(1, math.ceil(4 * L2_BYTES / store_bytes))))
+    q_c, q_r, c_kv, k_r = r.dev[0]
+    stores = []
+    anc = torch.empty(wl.B, max(nG, 1), dtype=torch.int32, device="cuda")
+    for _ in range(copies):
+        c_st = torch.empty(wl.B, R, wl.d_c, dtype=tdt, device="cuda")
+        k_st = torch.empty(wl.B, R, wl.d_r, dtype=tdt, device="cuda")
+        r.plan.build_stored(q_c, q_r, c_kv, k_r, wl.L, wl.g, wl.w, c_st, k_st, anc if nG else None)
+        stores.append((c_st, k_st))
+    torch.cuda.synchronize()
+    tb = Timer(torch, r.stream)
+    builds = []
+    for k in range(3):                      # the build reads the whole cache once (a prefill cost)
+        tb.start()
+        r.plan.build_stored(*r.dev[k % r.copies], wl.L, wl.g, wl.w, stores[0][0], stores[0][1],
+                            anc if nG else None)
+        builds.append(tb.stop())
+    out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32, device="cuda")
+
+    def step(k: int) -> None:
+        c_st, k_st = stores[k % copies]
+        r.plan.decode_stored(q_c, q_r, c_st, k_st, R, nG, 0.0, out, r.stream)
+
+    for k in range(3):
+        step(k)
+    torch.cuda.synchronize()
+    blocks = []
+    t = Timer(torch, r.stream)
+    for _ in range(5):
+        t.start()
+        for k in range(K):
+            step(k)
+        blocks.append(t.stop() / K)
+    assert r.plan.device_error() == kvc.LCA_OK
+    ts = statistics.median(blocks)
+    alg = store_bytes + wl.B * wl.H * (wl.d_c + wl.d_r) * wl.elem_bytes + wl.B * wl.H * wl.d_c * 4
+    del stores
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ts * 1e3, "context_tokens_per_s": wl.B * wl.L / ts, "unit": UNIT,
+            "stored_rows_per_seq": R, "rows_ratio_vs_full": R / wl.L,
+            "bytes_per_step": alg, "hbm_frac": alg / ts / 1e9 / peaks["hbm_gbs"],
+            "speedup_vs_lca_decode": t_lca / ts, "speedup_vs_mla_decode": t_mla / ts,
+            "build_ms": statistics.median(builds) * 1e3, "copies_rotated": copies,
+            "kernel": r.plan.kernel(R, 1, 0),
+            "note": "lca_build_stored once (head-mean condensation with this step's query), then "
+                    "lca_decode_stored over [stored || window] per step, no bias"}
+
+
 def workload_fractions(wl, t_step: float, t_main: float, peaks: dict) -> dict:
     alg = algorithmic_bytes(wl)
     flops = algorithmic_flops(wl)
@@ -559,6 +621,12 @@ def our_arm(args) -> None:
     t_dense = statistics.median(dense_s)
     assert r.plan.device_error() == kvc.LCA_OK
 
+    stored = None
+    if not args.no_stored:
+        barrier_sync()
+        stored = stored_leg(torch, kvc, r, max(5, min(K, 200)), measured_peaks()[0], t_total / K,
+                            t_dense / kd)
+
     tokens_per_step = world * wl.B * wl.L
     value = whole_job_rate(world, wl, K, t_total * 1.0)
     peaks, peak_kind = measured_peaks()
@@ -597,12 +665,15 @@ def our_arm(args) -> None:
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import oracle
         nthreads = os.cpu_count() or 1
-        rows = sorted({0, wl.B - 1})
+        # rows 0 and B-1, then more rows until about 10 s of oracle work
+        first = oracle.lca(x.q_c, x.q_r, x.c_kv, x.k_r, g=wl.g, w=wl.w, rows=[0], nthreads=nthreads)
+        n_rows = int(max(2, min(wl.B, 10.0 / max(first.seconds, 1e-3))))
+        rows = sorted({0, wl.B - 1} | set(range(1, n_rows - 1)))
         res = oracle.lca(x.q_c, x.q_r, x.c_kv, x.k_r, g=wl.g, w=wl.w, rows=rows, nthreads=nthreads)
         cpu = {"value": len(rows) * wl.L / res.seconds, "unit": UNIT, "cores": nthreads,
                "kind": "oracle",
-               "sample": f"sequences {rows} of the batch ({len(rows)} x {wl.H} heads, L={wl.L}), "
-                         f"oracle formulation A, {res.seconds:.1f} s"}
+               "sample": f"{len(rows)} sequences of the batch (rows {rows[0]}..{rows[-1]}; all "
+                         f"{wl.H} heads, L={wl.L}), oracle formulation A, {res.seconds:.1f} s"}
 
     head_kernel = kernel
     r.free()
@@ -644,6 +715,7 @@ def our_arm(args) -> None:
                        "ms_per_step": t_dense / kd * 1e3, "steps": kd,
                        "hbm_frac": alg / (t_dense / kd) / 1e9 / peaks["hbm_gbs"],
                        "note": "dense MLA decode over the same cache (same bytes), same kernels with n_G = 0"},
+        "stored_cache": stored,
         "per_config": pc,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -670,9 +742,12 @@ def main() -> None:
     ap.add_argument("--workload", default="v2", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--g", type=int, default=None, help="group size (default: the workload's)")
     ap.add_argument("--w", type=int, default=None, help="window (default: the workload's)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per step (default: the workload's; smaller for profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--no-stored", action="store_true")
     args = ap.parse_args()
     rc = spawn_ranks(args)
     if rc is not None:

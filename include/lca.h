@@ -46,7 +46,9 @@ typedef enum {
     LCA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
     LCA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait inside a kernel ran out (see lca_get_device_error) */
     LCA_ERR_PLAN_MISMATCH = 6,   /* the plan was made for another shape / dtype / device */
-    LCA_ERR_NO_MEMORY = 7        /* device or host allocation failed */
+    LCA_ERR_NO_MEMORY = 7,       /* device or host allocation failed */
+    LCA_ERR_DEVICE_CHECK = 8     /* debug build only: a kernel index failed its range check and the
+                                    access was skipped (see lca_get_device_error) */
 } lca_status;
 
 typedef enum { LCA_F32 = 0, LCA_BF16 = 1 } lca_dtype;
@@ -60,9 +62,10 @@ typedef struct lca_plan lca_plan;
  * Allocates the plan's device workspace (split partials and the device
  * error word) once; no later call allocates device memory, except the first
  * lca_decode_host call (its staging buffers).
- * Kernels: bf16 with (d_c, d_r) = (512, 64) and H a multiple of 16 runs the
- * tcgen05/TMA kernel; every other shape with d_c <= 1024, d_r <= 256 and
- * H <= 4096 runs the CUDA-core kernel (fp32 accumulation).
+ * Kernels: bf16 with (d_c, d_r) = (512, 64) runs a tcgen05/TMA kernel -- the
+ * two-CTA kernel when H is a multiple of 128 and g <= 64, else the 16-head
+ * kernel when H is a multiple of 16; every other shape with d_c <= 1024,
+ * d_r <= 256 and H <= 4096 runs the CUDA-core kernel (fp32 accumulation).
  * Errors: LCA_ERR_INVALID_ARG (null out_plan, non-positive sizes),
  * LCA_ERR_UNSUPPORTED, LCA_ERR_NO_MEMORY, LCA_ERR_CUDA.  *out_plan is
  * written only on LCA_OK; the caller frees it with lca_plan_destroy.
@@ -79,8 +82,11 @@ typedef enum {
     LCA_OPT_FORCE_SIMT = 1,        /* 1: use the CUDA-core kernel even where tcgen05 applies */
     LCA_OPT_NUM_CTAS = 2,          /* 1..SM count: CTAs of the tcgen05 kernel; 0: the SM count */
     LCA_OPT_WAIT_TIMEOUT_NS = 3,   /* bound of every in-kernel wait (default 2e9 ns) */
-    LCA_OPT_DEBUG_SKIP_LOAD = 4    /* 1: the tcgen05 producer skips its first load, so the
+    LCA_OPT_DEBUG_SKIP_LOAD = 4,   /* 1: the tcgen05 producer skips its first load, so the
                                       consumer's bounded wait runs out (tests the timeout path) */
+    LCA_OPT_KERNEL = 5             /* 0: automatic; else the lca_plan_kernel code to use
+                                      (1 CUDA-core, 2 tcgen05, 3 tcgen05 two-CTA); a call whose
+                                      shape that kernel cannot take returns LCA_ERR_UNSUPPORTED */
 } lca_option;
 
 lca_status lca_plan_set(lca_plan *plan, lca_option opt, int64_t value);
@@ -132,6 +138,107 @@ lca_status lca_decode_host(lca_plan *plan, const void *h_q_c, const void *h_q_r,
                            const void *h_c_kv, const void *h_k_r, int64_t L, int g, int w,
                            float *h_out, int32_t *h_anchor_idx, void *stream);
 
+/*
+ * Stored, head-shared condensed cache ("Latent-Condensed Transformer for
+ * Efficient Long Context Modeling", section 4, "Eficiencia": the 128K KV cache
+ * shrinks by ~90% and decode is faster because condensed groups are kept
+ * instead of their tokens).  A group is condensed once, with the query of the
+ * step that condenses it, and the entry serves every head.  The page does not
+ * say how heads are combined; here the pooling weights and the anchor come
+ * from the mean over heads of the scores (equal to the score of the mean
+ * query):  s_bar_t = (1/H) sum_h (q_c^h . c_t + q_r^h . k_t),  w_t =
+ * softmax over the group of s_bar_t,  a_j = the lowest index with the largest
+ * s_bar_t,  entry j = (c_bar_j = sum w_t c_t, k_{a_j}).
+ */
+
+/*
+ * Condense groups j0 .. j0+n-1 of every sequence (tokens [j g, j g + g), all
+ * below L) with the head-mean score of q_c [B][H][d_c], q_r [B][H][d_r].
+ *   c_kv [B][L][d_c], k_r [B][L][d_r]   device, plan dtype (the cache to condense)
+ *   c_dst, k_dst  device, plan dtype: entry jj of sequence b is written to row
+ *                 b * dst_rows + dst_row0 + jj of a [B][dst_rows][d_c] / [d_r] buffer
+ *                 (c_bar_j rounded to the plan dtype; k_{a_j} copied as stored)
+ *   anchor   [B][n] device int32: a_j, absolute positions (may be NULL when n == 0)
+ * For condensing on eviction (a group leaving the window) or at prefill.
+ * Errors: LCA_ERR_INVALID_ARG (null pointers, (j0 + n) g > L, L > max_L,
+ * dst_row0 + n > dst_rows), LCA_ERR_PLAN_MISMATCH, LCA_ERR_CUDA.  Asynchronous
+ * on `stream`; allocates nothing.
+ */
+lca_status lca_condense(lca_plan *plan, const void *q_c, const void *q_r, const void *c_kv,
+                        const void *k_r, int64_t L, int g, int64_t j0, int64_t n, void *c_dst,
+                        void *k_dst, int64_t dst_rows, int64_t dst_row0, int32_t *anchor,
+                        void *stream);
+
+/* Rows of the stored cache lca_build_stored writes for (L, g, w): n_G + (L - n_G g);
+ * -1 if g < 1, w < 0 or L < 1. */
+int64_t lca_stored_rows(int64_t L, int g, int w);
+
+/*
+ * Build the stored cache of every sequence from a full cache at context
+ * length L (prefill): rows [0, n_G) of c_store [B][R][d_c] / k_store [B][R][d_r]
+ * (R = lca_stored_rows(L, g, w)) are the condensed groups of section 2 step 1
+ * (lca_condense with j0 = 0, n = n_G), rows [n_G, R) a copy of the window
+ * tokens [n_G g, L).  anchor [B][n_G] int32 (NULL allowed when n_G == 0).
+ * All pointers 16-byte aligned (else LCA_ERR_ALIGNMENT).  Asynchronous.
+ */
+lca_status lca_build_stored(lca_plan *plan, const void *q_c, const void *q_r, const void *c_kv,
+                            const void *k_r, int64_t L, int g, int w, void *c_store,
+                            void *k_store, int32_t *anchor, void *stream);
+
+/*
+ * Decode over a stored cache: softmax attention of every head of (q_c, q_r)
+ * over the n_rows rows of c_store [B][n_rows][d_c] / k_store [B][n_rows][d_r]
+ * (value = latent), with `bias` added to the logits of rows [0, n_cond) (the
+ * condensed entries; log(g) counts an entry as the g tokens it stands for, 0
+ * adds nothing -- the page names no bias).  out [B][H][d_c] float32.  The rows
+ * may be in any order (attention is a sum over them); n_rows <= max_L.  Same
+ * kernels, layouts and errors as mla_decode; reads (n_rows / L) of the bytes
+ * a full-cache decode reads.
+ */
+lca_status lca_decode_stored(lca_plan *plan, const void *q_c, const void *q_r,
+                             const void *c_store, const void *k_store, int64_t n_rows,
+                             int64_t n_cond, float bias, float *out, void *stream);
+
+/*
+ * Context sharding.  The entries of one decode ([condensed groups || window]
+ * over a context of L tokens) can be split by position among several holders
+ * -- one slice of tokens [pos0, pos0 + n_tok) each (for example one GPU each),
+ * cut on multiples of g inside the condensed part [0, n_G g) -- which compute
+ * partial softmax sums over the entries they hold; the partials merge exactly
+ * by the online-softmax merge (the merge of per-host softmax statistics of
+ * "Pulsar Attention", Fase 2):  M = max_i M_i,
+ *   out = sum_i e^{M_i - M} O_i / sum_i e^{M_i - M} Z_i.
+ */
+
+/* Condensed groups inside tokens [pos0, pos0 + n_tok) of a context of L tokens;
+ * -1 if the slice cuts a group (or is out of range / g < 1 / w < 0). */
+int64_t lca_slice_groups(int64_t L, int g, int w, int64_t pos0, int64_t n_tok);
+
+/*
+ * Partial decode over one slice:
+ *   c_slice [B][n_tok][d_c], k_slice [B][n_tok][d_r]  device, plan dtype: tokens
+ *            [pos0, pos0 + n_tok) of each sequence (n_tok <= max_L; 0 allowed)
+ *   L, g, w  the whole context's length, group size and window
+ *   part_mz  [B][H][2] float32, written: (M, Z) per head -- the largest logit of
+ *            the slice's entries (-inf for an empty slice) and sum_e e^{logit_e - M}
+ *   part_o   [B][H][d_c] float32, written: sum_e e^{logit_e - M} value_e
+ *   anchor   [B][H][lca_slice_groups(...)] int32, absolute positions (NULL when 0)
+ * Same kernels as lca_decode.  Errors: LCA_ERR_INVALID_ARG (a cut group among
+ * them), LCA_ERR_UNSUPPORTED, LCA_ERR_ALIGNMENT, LCA_ERR_CUDA.  Asynchronous.
+ */
+lca_status lca_decode_partial(lca_plan *plan, const void *q_c, const void *q_r,
+                              const void *c_slice, const void *k_slice, int64_t n_tok,
+                              int64_t pos0, int64_t L, int g, int w, float *part_mz,
+                              float *part_o, int32_t *anchor, void *stream);
+
+/*
+ * Merge n_parts partials stacked by part -- part_mz [n_parts][B][H][2],
+ * part_o [n_parts][B][H][d_c] (device, float32, e.g. gathered from every
+ * holder) -- into out [B][H][d_c] float32.  Asynchronous; allocates nothing.
+ */
+lca_status lca_merge_partials(lca_plan *plan, int n_parts, const float *part_mz,
+                              const float *part_o, float *out, void *stream);
+
 /* n_G for (L, g, w): floor((L - w) / g) when L > w, else 0; -1 if g < 1, w < 0 or L < 1. */
 int64_t lca_num_groups(int64_t L, int g, int w);
 
@@ -140,9 +247,11 @@ const char *lca_status_string(lca_status status);
 
 /*
  * Synchronise `stream`, read and clear the plan's device error word.
- * Returns LCA_OK, LCA_ERR_DEVICE_TIMEOUT when an in-kernel wait ran out (the
- * kernel then skipped its remaining work and left outputs undefined), or
- * LCA_ERR_CUDA when the synchronisation itself failed.
+ * Returns LCA_OK, LCA_ERR_DEVICE_CHECK when (in the range-checked debug build,
+ * liblca_checked.so) a kernel index failed its check, LCA_ERR_DEVICE_TIMEOUT
+ * when an in-kernel wait ran out (the kernel then skipped its remaining work
+ * and left outputs undefined), or LCA_ERR_CUDA when the synchronisation
+ * itself failed.
  */
 lca_status lca_get_device_error(lca_plan *plan, void *stream);
 
@@ -155,7 +264,9 @@ lca_status lca_get_device_error(lca_plan *plan, void *stream);
  */
 lca_status lca_plan_set_timing_event(lca_plan *plan, void *event);
 
-/* Which kernel a plan runs for (L, g, w): 0 = none (invalid), 1 = CUDA-core, 2 = tcgen05. */
+/* Which kernel a plan runs for (L, g, w): 0 = none (invalid), 1 = CUDA-core, 2 = tcgen05
+ * (16 heads per CTA), 3 = tcgen05 two-CTA (128 heads per cluster of two CTAs that split the
+ * latent width; H a multiple of 128, g <= 64). */
 int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
 
 /*

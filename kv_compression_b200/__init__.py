@@ -13,20 +13,24 @@ from dataclasses import dataclass
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblca.so")
+CHECKED_LIB_PATH = os.path.join(HERE, "liblca_checked.so")
 
 LCA_OK = 0
 LCA_ERR_UNSUPPORTED = 2
 LCA_ERR_DEVICE_TIMEOUT = 5
 STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED", 3: "LCA_ERR_ALIGNMENT",
           4: "LCA_ERR_CUDA", 5: "LCA_ERR_DEVICE_TIMEOUT", 6: "LCA_ERR_PLAN_MISMATCH",
-          7: "LCA_ERR_NO_MEMORY"}
+          7: "LCA_ERR_NO_MEMORY", 8: "LCA_ERR_DEVICE_CHECK"}
 LCA_F32, LCA_BF16 = 0, 1
-OPT_FORCE_SIMT, OPT_NUM_CTAS, OPT_WAIT_TIMEOUT_NS, OPT_DEBUG_SKIP_LOAD = 1, 2, 3, 4
-KERNEL_NAMES = {0: "none", 1: "simt", 2: "tcgen05"}
+OPT_FORCE_SIMT, OPT_NUM_CTAS, OPT_WAIT_TIMEOUT_NS, OPT_DEBUG_SKIP_LOAD, OPT_KERNEL = 1, 2, 3, 4, 5
+KERNEL_NAMES = {0: "none", 1: "simt", 2: "tcgen05", 3: "tcgen05_pair"}
+KERNEL_CODES = {v: k for k, v in KERNEL_NAMES.items()}
 
 EXPORTS = ["lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
            "lca_decode_host", "lca_num_groups", "lca_status_string", "lca_get_device_error",
-           "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc"]
+           "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
+           "lca_stored_rows", "lca_build_stored", "lca_decode_stored", "lca_slice_groups",
+           "lca_decode_partial", "lca_merge_partials"]
 
 
 class LcaError(RuntimeError):
@@ -62,9 +66,19 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lca_plan_set_timing_event.argtypes = [vp, vp]
     lib.lca_decode_noalloc.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i32, i32, vp,
                                        vp, vp]
+    lib.lca_condense.argtypes = [vp, vp, vp, vp, vp, i64, i32, i64, i64, vp, vp, i64, i64, vp, vp]
+    lib.lca_stored_rows.argtypes = [i64, i32, i32]
+    lib.lca_stored_rows.restype = i64
+    lib.lca_build_stored.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp]
+    lib.lca_decode_stored.argtypes = [vp, vp, vp, vp, vp, i64, i64, ctypes.c_float, vp, vp]
+    lib.lca_slice_groups.argtypes = [i64, i32, i32, i64, i64]
+    lib.lca_slice_groups.restype = i64
+    lib.lca_decode_partial.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
+    lib.lca_merge_partials.argtypes = [vp, i32, vp, vp, vp, vp]
     for name in ("lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
                  "lca_decode_host", "lca_get_device_error", "lca_plan_kernel",
-                 "lca_plan_set_timing_event", "lca_decode_noalloc"):
+                 "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
+                 "lca_build_stored", "lca_decode_stored", "lca_decode_partial", "lca_merge_partials"):
         getattr(lib, name).restype = i32
     if path == LIB_PATH:
         _lib = lib
@@ -99,12 +113,13 @@ class Plan:
     d_r: int
     dtype: str
     max_L: int
+    lib_path: str | None = None    # another build of the library (the range-checked one)
 
     def __post_init__(self):
         import torch
         if not torch.cuda.is_available():
             raise RuntimeError("kv_compression_b200 needs a CUDA device (no CPU fallback)")
-        self._lib = load_library()
+        self._lib = load_library(self.lib_path or LIB_PATH)
         h = ctypes.c_void_p()
         dt = LCA_BF16 if self.dtype == "bf16" else LCA_F32
         _check(self._lib.lca_plan_create(self.B, self.H, self.d_c, self.d_r, dt, self.max_L,
@@ -155,6 +170,39 @@ class Plan:
                                          g, w, _ptr(out), _ptr(anchor), _stream_handle(stream)),
                "lca_decode_host")
 
+    def condense(self, q_c, q_r, c_kv, k_r, L: int, g: int, j0: int, n: int, c_dst, k_dst,
+                 dst_rows: int, dst_row0: int, anchor, stream=None) -> None:
+        """lca_condense: groups j0 .. j0+n-1 into rows dst_row0.. of [B][dst_rows][d] buffers."""
+        _check(self._lib.lca_condense(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_kv), _ptr(k_r), L, g, j0, n,
+                                      _ptr(c_dst), _ptr(k_dst), dst_rows, dst_row0, _ptr(anchor),
+                                      _stream_handle(stream)), "lca_condense")
+
+    def build_stored(self, q_c, q_r, c_kv, k_r, L: int, g: int, w: int, c_store, k_store, anchor,
+                     stream=None) -> None:
+        """lca_build_stored: [condensed groups || window tokens] per sequence."""
+        _check(self._lib.lca_build_stored(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_kv), _ptr(k_r), L, g, w,
+                                          _ptr(c_store), _ptr(k_store), _ptr(anchor),
+                                          _stream_handle(stream)), "lca_build_stored")
+
+    def decode_stored(self, q_c, q_r, c_store, k_store, n_rows: int, n_cond: int, bias: float, out,
+                      stream=None) -> None:
+        """lca_decode_stored: attention over the stored rows, `bias` on the first n_cond."""
+        _check(self._lib.lca_decode_stored(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_store), _ptr(k_store),
+                                           n_rows, n_cond, float(bias), _ptr(out),
+                                           _stream_handle(stream)), "lca_decode_stored")
+
+    def decode_partial(self, q_c, q_r, c_slice, k_slice, n_tok: int, pos0: int, L: int, g: int, w: int,
+                       part_mz, part_o, anchor, stream=None) -> None:
+        """lca_decode_partial: (M, Z, O) of the entries held by tokens [pos0, pos0 + n_tok)."""
+        _check(self._lib.lca_decode_partial(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_slice), _ptr(k_slice),
+                                            n_tok, pos0, L, g, w, _ptr(part_mz), _ptr(part_o),
+                                            _ptr(anchor), _stream_handle(stream)), "lca_decode_partial")
+
+    def merge_partials(self, n_parts: int, part_mz, part_o, out, stream=None) -> None:
+        """lca_merge_partials: out from n_parts stacked partials."""
+        _check(self._lib.lca_merge_partials(self._h, n_parts, _ptr(part_mz), _ptr(part_o), _ptr(out),
+                                            _stream_handle(stream)), "lca_merge_partials")
+
     def device_error(self, stream=None) -> int:
         return int(self._lib.lca_get_device_error(self._h, _stream_handle(stream)))
 
@@ -189,3 +237,11 @@ def mla_decode(q_c, q_r, c_kv, k_r, plan: Plan | None = None, stream=None):
     out = torch.empty(B, H, d_c, dtype=torch.float32, device=q_c.device)
     plan.dense(q_c, q_r, c_kv, k_r, L, out, stream)
     return out
+
+
+def stored_rows(L: int, g: int, w: int) -> int:
+    return int(load_library().lca_stored_rows(L, g, w))
+
+
+def slice_groups(L: int, g: int, w: int, pos0: int, n_tok: int) -> int:
+    return int(load_library().lca_slice_groups(L, g, w, pos0, n_tok))

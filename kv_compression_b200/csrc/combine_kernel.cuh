@@ -5,6 +5,7 @@
 #pragma once
 #include <cstdint>
 
+#include "checks.cuh"
 #include "ptx.cuh"
 
 namespace lca {
@@ -21,11 +22,17 @@ struct CombineParams {
   //   mode 1: the units (b, tile) are cut into G contiguous ranges, range c =
   //           [c*U/G, (c+1)*U/G) with U = B * tiles_per_seq; range c writes the
   //           partial of sequence b into slot b + c.
+  //   mode 2: slots b, B + b, 2B + b, ... (n_split of them): partials stacked
+  //           by part, merged across parts (lca_merge_partials)
   int mode;
   int n_split;
   int64_t tiles_per_seq;
   int64_t G;
   int wait_prior;        // 1: launched as a programmatic dependent of the producer grid
+  float* out_mz;         // non-null: write the merged (M, Z) to out_mz [B][H][2] and the
+                         // unnormalised sum O to out (a partial for a later merge)
+  int64_t n_slots;       // slots readable in part_o / part_mz (range checks)
+  int* err;              // device error word (range checks; null: none)
 };
 
 __device__ __forceinline__ int64_t range_owner(int64_t u, int64_t U, int64_t G) {
@@ -47,10 +54,14 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
   const int h = blockIdx.x, b = blockIdx.y;
   const int d = blockIdx.z * kCombineThreads + threadIdx.x;
   if (d >= p.d_c) return;
-  int64_t first, count;
+  int64_t first, count, slot_step = 1;
   if (p.mode == 0) {
     first = (int64_t)b * p.n_split;
     count = p.n_split;
+  } else if (p.mode == 2) {
+    first = b;
+    count = p.n_split;
+    slot_step = p.B;
   } else {
     const int64_t U = (int64_t)p.B * p.tiles_per_seq;
     const int64_t c0 = range_owner((int64_t)b * p.tiles_per_seq, U, p.G);
@@ -58,7 +69,9 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     first = b + c0;
     count = c1 - c0 + 1;
   }
-  const int64_t stride = (int64_t)p.H * p.d_c;
+  if (count > 0 && p.err && !LCA_CHECK(p.err, first + (count - 1) * slot_step < p.n_slots, 0xC11))
+    count = 0;
+  const int64_t stride = (int64_t)p.H * p.d_c * slot_step;
   const float* po = p.part_o + (first * p.H + h) * (int64_t)p.d_c + d;
   const float2* pmz = reinterpret_cast<const float2*>(p.part_mz) + first * p.H + h;
   float M = -INFINITY, Z = 0.f, acc = 0.f;
@@ -69,7 +82,7 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
 #pragma unroll
     for (int k = 0; k < kChunk; ++k) {
       if (k < n) {
-        mz[k] = pmz[(i0 + k) * p.H];
+        mz[k] = pmz[(i0 + k) * slot_step * p.H];
         o[k] = po[(i0 + k) * stride];
       } else {
         mz[k] = make_float2(-INFINITY, 0.f);
@@ -91,7 +104,15 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     }
     M = mc;
   }
-  p.out[((int64_t)b * p.H + h) * p.d_c + d] = acc / Z;
+  if (p.out_mz) {
+    p.out[((int64_t)b * p.H + h) * p.d_c + d] = acc;
+    if (d == 0) {
+      p.out_mz[((int64_t)b * p.H + h) * 2 + 0] = M;
+      p.out_mz[((int64_t)b * p.H + h) * 2 + 1] = Z;
+    }
+  } else {
+    p.out[((int64_t)b * p.H + h) * p.d_c + d] = acc / Z;
+  }
 }
 
 }  // namespace lca

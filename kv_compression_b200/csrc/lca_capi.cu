@@ -12,7 +12,10 @@
 #include <new>
 
 #include "lca.h"
+#include "checks.cuh"
 #include "combine_kernel.cuh"
+#include "condense_kernel.cuh"
+#include "pair_kernel.cuh"
 #include "simt_kernel.cuh"
 #include "tc_kernel.cuh"
 
@@ -23,16 +26,21 @@ struct lca_plan {
   int device;
   int num_sms;
   bool tc_shape;           // the tcgen05 kernel can take this shape
+  bool pair_shape;         // the two-CTA tcgen05 kernel can take this shape (H % 128 == 0)
+  int pair_clusters;       // two-CTA clusters resident at once on this device
   int64_t ws_slots;
   float* part_o;           // [ws_slots][H][d_c]
   float* part_mz;          // [ws_slots][H][2]
   int* err;                // [2]: flags, where
   // options
   bool force_simt;
+  int kernel_pref;         // 0: automatic, else the lca_plan_kernel code to use
   int num_ctas;
   uint64_t timeout_ns;
   int debug_skip_load;
   cudaEvent_t timing_event;  // recorded between the main and the combine kernel when set
+  int64_t bias_rows;         // set only for the duration of an lca_decode_stored call
+  float bias;
   // lca_decode_host staging (allocated on first use)
   void* st_qc;
   void* st_qr;
@@ -104,16 +112,47 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-enum Kernel { kNone = 0, kSimt = 1, kTc = 2 };
+enum Kernel { kNone = 0, kSimt = 1, kTc = 2, kPair = 3 };
 
+// Where the rows of one call sit in the context: a whole context (win0 = n_G g,
+// pos0 = 0) or one slice of a context-sharded decode; and whether the combine
+// writes the normalised output or a partial (M, Z, unnormalised O).
+struct Slice {
+  int64_t win0;
+  int64_t pos0;
+  float* out_mz;
+};
+
+bool tc_group_ok(int64_t nG, int g, int gmax) { return nG == 0 || (is_pow2(g) && g <= gmax); }
+
+// The kernel for (n_G, g): the two-CTA tcgen05 kernel where H is a multiple of
+// 128 and g <= 64, else the 16-head tcgen05 kernel (H a multiple of 16,
+// g <= 128), else the CUDA-core kernel.  LCA_OPT_FORCE_SIMT / LCA_OPT_KERNEL
+// narrow the choice; a forced kernel that cannot take the shape gives kNone.
 Kernel choose(const lca_plan* p, int64_t nG, int g) {
-  if (p->tc_shape && !p->force_simt && (nG == 0 || (is_pow2(g) && g <= 128))) return kTc;
-  if (nG == 0 || g <= lca::kSimtTileMax) return kSimt;
+  const bool pair_ok = p->pair_shape && tc_group_ok(nG, g, lca::pair::kT);
+  const bool tc_ok = p->tc_shape && tc_group_ok(nG, g, lca::tc::kT);
+  const bool simt_ok = nG == 0 || g <= lca::kSimtTileMax;
+  int pref = p->force_simt ? kSimt : p->kernel_pref;
+  if (pref == kPair) return pair_ok ? kPair : kNone;
+  if (pref == kTc) return tc_ok ? kTc : kNone;
+  if (pref == kSimt) return simt_ok ? kSimt : kNone;
+  if (pair_ok) return kPair;
+  if (tc_ok) return kTc;
+  if (simt_ok) return kSimt;
   return kNone;
 }
 
-lca_status launch_combine(const lca_plan* p, const lca::CombineParams& cp, cudaStream_t stream,
+lca_status launch_combine(const lca_plan* p, const lca::CombineParams& cp_in, cudaStream_t stream,
                           bool pdl) {
+  lca::CombineParams cp = cp_in;
+  if (cp.mode != 2) {          // the plan's workspace; a merge reads the caller's n_split parts
+    cp.n_slots = p->ws_slots;
+    cp.err = p->err;
+  } else {
+    cp.n_slots = (int64_t)cp.n_split * p->B;
+    cp.err = p->err;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p->H, (unsigned)p->B,
                      (unsigned)((p->d_c + lca::kCombineThreads - 1) / lca::kCombineThreads));
@@ -131,7 +170,7 @@ lca_status launch_combine(const lca_plan* p, const lca::CombineParams& cp, cudaS
 
 lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                     const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
-                    cudaStream_t stream) {
+                    cudaStream_t stream, const Slice& sl) {
   const int ge = nG > 0 ? g : 1;
   const int tile = ge * std::max(1, 256 / ge);
   int64_t split_len = ceil_div(L, simt_target_splits(p));
@@ -143,6 +182,8 @@ lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c
   sp.B = p->B; sp.H = p->H; sp.d_c = p->d_c; sp.d_r = p->d_r;
   sp.L = L; sp.g = ge; sp.nG = nG; sp.split_len = split_len; sp.tile = tile;
   sp.n_split = (int)n_split; sp.anchor = anchor; sp.part_o = p->part_o; sp.part_mz = p->part_mz;
+  sp.bias_rows = p->bias_rows; sp.bias = p->bias; sp.win0 = sl.win0; sp.pos0 = sl.pos0;
+  sp.ws_slots = p->ws_slots; sp.err = p->err;
   const size_t smem = (size_t)(p->d_c + p->d_r + 4 * lca::kSimtTileMax + lca::kSimtWarps) * 4;
   dim3 grid((unsigned)n_split, (unsigned)p->H, (unsigned)p->B);
   if (p->dt == LCA_F32)
@@ -154,7 +195,7 @@ lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c
   lca::CombineParams cp = {};
   cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;
   cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 0; cp.n_split = (int)n_split;
-  cp.wait_prior = 0;
+  cp.wait_prior = 0; cp.out_mz = sl.out_mz;
   return launch_combine(p, cp, stream, false);
 }
 
@@ -213,7 +254,7 @@ cudaError_t launch_tc_g(int g, const lca::tc::TcParams& tp, unsigned grid, cudaS
 
 lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                   const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, const Slice& sl) {
   lca::tc::TcParams tp;
   std::memset(&tp, 0, sizeof(tp));
   const uint64_t rows = (uint64_t)p->B * (uint64_t)L;
@@ -226,19 +267,125 @@ lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_k
   const int64_t tps = ceil_div(L, lca::tc::kT);
   const int64_t U = (int64_t)p->B * tps;
   const int ctas = p->num_ctas > 0 ? p->num_ctas : p->num_sms;
-  const int64_t G = std::max<int64_t>(1, std::min<int64_t>(ctas / n_hb, U));
-  if ((int64_t)p->B + G - 1 > p->ws_slots) return LCA_ERR_UNSUPPORTED;
+  int64_t G = std::max<int64_t>(1, std::min<int64_t>(ctas / n_hb, U));
+  G = std::min<int64_t>(G, p->ws_slots - p->B + 1);    // range c writes slot b + c
+  if (G < 1) return LCA_ERR_UNSUPPORTED;
   tp.B = p->B; tp.H = p->H; tp.L = L; tp.nG = nG;
   tp.tiles_per_seq = tps; tp.U = U; tp.G = G; tp.n_hb = n_hb;
   tp.anchor = anchor; tp.part_o = p->part_o; tp.part_mz = p->part_mz; tp.err = p->err;
   tp.timeout_ns = p->timeout_ns; tp.debug_skip_load = p->debug_skip_load;
+  tp.bias_rows = p->bias_rows; tp.bias = p->bias; tp.win0 = sl.win0; tp.pos0 = sl.pos0;
   const unsigned grid = (unsigned)(G * n_hb);
   if (launch_tc_g(nG > 0 ? g : 1, tp, grid, stream, p->device) != cudaSuccess) return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
   lca::CombineParams cp = {};
   cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;
   cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 1; cp.tiles_per_seq = tps; cp.G = G;
-  cp.wait_prior = 1;
+  cp.wait_prior = 1; cp.out_mz = sl.out_mz;
+  return launch_combine(p, cp, stream, true);
+}
+
+template <int LOG2G>
+cudaError_t launch_pair(const lca::pair::PairParams& pp, unsigned clusters, cudaStream_t stream, int device) {
+  static std::atomic<uint64_t> configured{0};
+  if (!device_flag_set(configured, device)) {
+    cudaError_t e = cudaFuncSetAttribute(lca::pair::lca_pair_kernel<LOG2G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         lca::pair::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    device_flag_mark(configured, device);
+  }
+  // Clusters of two CTAs (one per SM), launched as a programmatic dependent
+  // like the 16-head kernel.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(lca::pair::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = lca::pair::kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, lca::pair::lca_pair_kernel<LOG2G>, pp);
+}
+
+cudaError_t launch_pair_g(int g, const lca::pair::PairParams& pp, unsigned clusters, cudaStream_t stream,
+                          int device) {
+  switch (g) {
+    case 1: return launch_pair<0>(pp, clusters, stream, device);
+    case 2: return launch_pair<1>(pp, clusters, stream, device);
+    case 4: return launch_pair<2>(pp, clusters, stream, device);
+    case 8: return launch_pair<3>(pp, clusters, stream, device);
+    case 16: return launch_pair<4>(pp, clusters, stream, device);
+    case 32: return launch_pair<5>(pp, clusters, stream, device);
+    case 64: return launch_pair<6>(pp, clusters, stream, device);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// Two-CTA clusters of the pair kernel that fit on the device at once (one
+// wave); 0 when the query fails.
+int pair_cluster_capacity(int num_sms) {
+  cudaError_t e = cudaFuncSetAttribute(lca::pair::lca_pair_kernel<4>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       lca::pair::kSmemAlloc);
+  if (e != cudaSuccess) { cudaGetLastError(); return num_sms / 2; }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
+  cfg.blockDim = dim3(lca::pair::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = lca::pair::kSmemAlloc;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, lca::pair::lca_pair_kernel<4>, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return num_sms / 2;
+  }
+  return n;
+}
+
+lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
+                    const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
+                    cudaStream_t stream, const Slice& sl) {
+  lca::pair::PairParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  const uint64_t rows = (uint64_t)p->B * (uint64_t)L;
+  if (rows > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
+  const uint64_t qrows = (uint64_t)p->B * (uint64_t)p->H;
+  if (!make_map(&pp.tm_c, c_kv, 512, rows, lca::pair::kT) ||
+      !make_map(&pp.tm_k, k_r, 64, rows, lca::pair::kT) ||
+      !make_map(&pp.tm_qc, q_c, 512, qrows, lca::pair::kHeads) ||
+      !make_map(&pp.tm_qr, q_r, 64, qrows, lca::pair::kOwn))
+    return LCA_ERR_CUDA;
+  const int n_hb = p->H / lca::pair::kHeads;
+  const int64_t tps = ceil_div(L, lca::pair::kT);
+  const int64_t U = (int64_t)p->B * tps;
+  const int64_t clusters = p->num_ctas > 0 ? std::max(1, p->num_ctas / 2) : p->pair_clusters;
+  int64_t G = std::max<int64_t>(1, std::min<int64_t>(clusters / n_hb, U));
+  G = std::min<int64_t>(G, p->ws_slots - p->B + 1);    // range c writes slot b + c
+  if (G < 1) return LCA_ERR_UNSUPPORTED;
+  pp.B = p->B; pp.H = p->H; pp.L = L; pp.nG = nG;
+  pp.tiles_per_seq = tps; pp.U = U; pp.G = G; pp.n_hb = n_hb;
+  pp.anchor = anchor; pp.part_o = p->part_o; pp.part_mz = p->part_mz; pp.err = p->err;
+  pp.timeout_ns = p->timeout_ns; pp.debug_skip_load = p->debug_skip_load;
+  pp.bias_rows = p->bias_rows; pp.bias = p->bias; pp.win0 = sl.win0; pp.pos0 = sl.pos0;
+  if (launch_pair_g(nG > 0 ? g : 1, pp, (unsigned)(G * n_hb), stream, p->device) != cudaSuccess)
+    return LCA_ERR_CUDA;
+  if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
+  lca::CombineParams cp = {};
+  cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;
+  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 1; cp.tiles_per_seq = tps; cp.G = G;
+  cp.wait_prior = 1; cp.out_mz = sl.out_mz;
   return launch_combine(p, cp, stream, true);
 }
 
@@ -252,25 +399,60 @@ lca_status check_common(const lca_plan* p, const void* q_c, const void* q_r, con
   return LCA_OK;
 }
 
+}  // namespace
+extern "C" int64_t lca_num_groups(int64_t L, int g, int w);
+namespace {
+
+// One decode over `L` cache rows of a context: n_G groups in those rows (the
+// anchor stride), window from row sl.win0, anchors offset by sl.pos0.
+lca_status decode_rows(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
+                       const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
+                       void* stream, const Slice& sl) {
+  lca_status st = check_common(p, q_c, q_r, c_kv, k_r, L, out);
+  if (st != LCA_OK) return st;
+  if (nG > 0 && !anchor) return LCA_ERR_INVALID_ARG;
+  const Kernel k = choose(p, nG, g);
+  if (k == kNone) return LCA_ERR_UNSUPPORTED;
+  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(c_kv) || !aligned16(k_r) ||
+      !aligned16(out) || (nG > 0 && !aligned16(anchor)) || (sl.out_mz && !aligned16(sl.out_mz)))
+    return LCA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k == kPair) return run_pair(p, q_c, q_r, c_kv, k_r, L, g, nG, out, anchor, s, sl);
+  if (k == kTc) return run_tc(p, q_c, q_r, c_kv, k_r, L, g, nG, out, anchor, s, sl);
+  return run_simt(p, q_c, q_r, c_kv, k_r, L, g, nG, out, anchor, s, sl);
+}
+
 lca_status decode_impl(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                        const void* k_r, int64_t L, int g, int w, float* out, int32_t* anchor,
                        void* stream, bool dense) {
-  lca_status st = check_common(p, q_c, q_r, c_kv, k_r, L, out);
-  if (st != LCA_OK) return st;
   int64_t nG = 0;
   if (!dense) {
     if (g < 1 || w < 0) return LCA_ERR_INVALID_ARG;
     nG = lca_num_groups(L, g, w);
-    if (nG > 0 && !anchor) return LCA_ERR_INVALID_ARG;
   }
-  const Kernel k = choose(p, nG, g);
-  if (k == kNone) return LCA_ERR_UNSUPPORTED;
-  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(c_kv) || !aligned16(k_r) ||
-      !aligned16(out) || (nG > 0 && !aligned16(anchor)))
-    return LCA_ERR_ALIGNMENT;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (k == kTc) return run_tc(p, q_c, q_r, c_kv, k_r, L, g, nG, out, anchor, s);
-  return run_simt(p, q_c, q_r, c_kv, k_r, L, g, nG, out, anchor, s);
+  const Slice whole = {nG * (dense ? 1 : g), 0, nullptr};
+  return decode_rows(p, q_c, q_r, c_kv, k_r, L, dense ? 1 : g, nG, out, anchor, stream, whole);
+}
+
+lca_status launch_condense(const lca_plan* p, const lca::CondenseParams& cp, cudaStream_t stream) {
+  if (cp.n <= 0) return LCA_OK;
+  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(ceil_div(cp.n, lca::kCondWarps),
+                                                                 ceil_div(4LL * p->num_sms, p->B)));
+  dim3 grid((unsigned)per_seq, (unsigned)p->B, 1);
+  const size_t smem = (size_t)(p->d_c + p->d_r) * sizeof(float);
+  if (p->dt == LCA_F32)
+    lca::lca_condense_kernel<float><<<grid, lca::kCondThreads, smem, stream>>>(cp);
+  else
+    lca::lca_condense_kernel<__nv_bfloat16><<<grid, lca::kCondThreads, smem, stream>>>(cp);
+  return cudaGetLastError() == cudaSuccess ? LCA_OK : LCA_ERR_CUDA;
+}
+
+lca_status launch_copy_rows(const lca::CopyRowsParams& rp, cudaStream_t stream) {
+  if (rp.n <= 0) return LCA_OK;
+  const int64_t total = rp.B * rp.n * (rp.row_bytes / 16);
+  const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256), 4096));
+  lca::lca_copy_rows_kernel<<<blocks, 256, 0, stream>>>(rp);
+  return cudaGetLastError() == cudaSuccess ? LCA_OK : LCA_ERR_CUDA;
 }
 
 void free_staging(lca_plan* p) {
@@ -300,6 +482,7 @@ const char* lca_status_string(lca_status s) {
     case LCA_ERR_DEVICE_TIMEOUT: return "a bounded in-kernel wait ran out";
     case LCA_ERR_PLAN_MISMATCH: return "plan made for another shape or device";
     case LCA_ERR_NO_MEMORY: return "out of memory";
+    case LCA_ERR_DEVICE_CHECK: return "a kernel index failed its range check (debug build)";
   }
   return "unknown status";
 }
@@ -323,6 +506,8 @@ lca_status lca_plan_create(int B, int H, int d_c, int d_r, lca_dtype dt, int64_t
   }
   p->tc_shape = dt == LCA_BF16 && d_c == lca::tc::kDC && d_r == lca::tc::kDR &&
                 (H % lca::tc::kHC) == 0;
+  p->pair_shape = p->tc_shape && (H % lca::pair::kHeads) == 0;
+  p->pair_clusters = p->pair_shape ? pair_cluster_capacity(p->num_sms) : 0;
   const int64_t simt_slots = (int64_t)B * simt_target_splits(p);
   const int64_t tc_slots = p->tc_shape ? (int64_t)B + p->num_sms : 0;
   p->ws_slots = std::max(simt_slots, tc_slots);
@@ -362,6 +547,10 @@ lca_status lca_plan_set(lca_plan* p, lca_option opt, int64_t v) {
       p->timeout_ns = (uint64_t)v;
       return LCA_OK;
     case LCA_OPT_DEBUG_SKIP_LOAD: p->debug_skip_load = v != 0; return LCA_OK;
+    case LCA_OPT_KERNEL:
+      if (v < 0 || v > kPair) return LCA_ERR_INVALID_ARG;
+      p->kernel_pref = (int)v;
+      return LCA_OK;
   }
   return LCA_ERR_INVALID_ARG;
 }
@@ -428,6 +617,114 @@ lca_status lca_decode_host(lca_plan* p, const void* h_q_c, const void* h_q_r, co
   return LCA_OK;
 }
 
+int64_t lca_stored_rows(int64_t L, int g, int w) {
+  const int64_t nG = lca_num_groups(L, g, w);
+  if (nG < 0) return -1;
+  return nG + (L - nG * g);
+}
+
+lca_status lca_condense(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
+                        const void* k_r, int64_t L, int g, int64_t j0, int64_t n, void* c_dst,
+                        void* k_dst, int64_t dst_rows, int64_t dst_row0, int32_t* anchor,
+                        void* stream) {
+  if (!p || !q_c || !q_r || !c_kv || !k_r || !c_dst || !k_dst || (n > 0 && !anchor))
+    return LCA_ERR_INVALID_ARG;
+  if (L < 1 || L > p->max_L || g < 1 || j0 < 0 || n < 0 || (j0 + n) * (int64_t)g > L)
+    return LCA_ERR_INVALID_ARG;
+  if (dst_row0 < 0 || dst_rows < dst_row0 + n) return LCA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
+  if (dev != p->device) return LCA_ERR_PLAN_MISMATCH;
+  lca::CondenseParams cp = {};
+  cp.q_c = q_c; cp.q_r = q_r; cp.c_kv = c_kv; cp.k_r = k_r;
+  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.d_r = p->d_r; cp.L = L; cp.g = g;
+  cp.j0 = j0; cp.n = n; cp.c_dst = c_dst; cp.k_dst = k_dst; cp.dst_rows = dst_rows;
+  cp.dst_row0 = dst_row0; cp.anchor = anchor; cp.err = p->err;
+  return launch_condense(p, cp, static_cast<cudaStream_t>(stream));
+}
+
+lca_status lca_build_stored(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
+                            const void* k_r, int64_t L, int g, int w, void* c_store, void* k_store,
+                            int32_t* anchor, void* stream) {
+  if (!p || !q_c || !q_r || !c_kv || !k_r || !c_store || !k_store) return LCA_ERR_INVALID_ARG;
+  if (L < 1 || L > p->max_L || g < 1 || w < 0) return LCA_ERR_INVALID_ARG;
+  const int64_t nG = lca_num_groups(L, g, w);
+  if (nG > 0 && !anchor) return LCA_ERR_INVALID_ARG;
+  const int64_t rows = lca_stored_rows(L, g, w);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!aligned16(c_kv) || !aligned16(k_r) || !aligned16(c_store) || !aligned16(k_store))
+    return LCA_ERR_ALIGNMENT;
+  lca_status st = lca_condense(p, q_c, q_r, c_kv, k_r, L, g, 0, nG, c_store, k_store, rows, 0,
+                               anchor, stream);
+  if (st != LCA_OK) return st;
+  const size_t es = elem_size(p->dt);
+  lca::CopyRowsParams rc = {};
+  rc.src = static_cast<const uint8_t*>(c_kv); rc.dst = static_cast<uint8_t*>(c_store);
+  rc.src_rows = L; rc.src_row0 = nG * g; rc.dst_rows = rows; rc.dst_row0 = nG; rc.n = L - nG * g;
+  rc.row_bytes = (int64_t)p->d_c * (int64_t)es; rc.B = p->B;
+  if ((st = launch_copy_rows(rc, s)) != LCA_OK) return st;
+  lca::CopyRowsParams rk = rc;
+  rk.src = static_cast<const uint8_t*>(k_r); rk.dst = static_cast<uint8_t*>(k_store);
+  rk.row_bytes = (int64_t)p->d_r * (int64_t)es;
+  return launch_copy_rows(rk, s);
+}
+
+lca_status lca_decode_stored(lca_plan* p, const void* q_c, const void* q_r, const void* c_store,
+                             const void* k_store, int64_t n_rows, int64_t n_cond, float bias,
+                             float* out, void* stream) {
+  if (!p || n_cond < 0 || n_cond > n_rows) return LCA_ERR_INVALID_ARG;
+  p->bias_rows = n_cond;
+  p->bias = bias;
+  const lca_status st =
+      decode_impl(p, q_c, q_r, c_store, k_store, n_rows, 1, 0, out, nullptr, stream, true);
+  p->bias_rows = 0;
+  p->bias = 0.f;
+  return st;
+}
+
+int64_t lca_slice_groups(int64_t L, int g, int w, int64_t pos0, int64_t n_tok) {
+  const int64_t nG = lca_num_groups(L, g, w);
+  if (nG < 0 || pos0 < 0 || n_tok < 0 || pos0 + n_tok > L) return -1;
+  const int64_t win0 = nG * g, end = pos0 + n_tok;
+  if ((pos0 < win0 && pos0 % g != 0) || (end < win0 && end % g != 0)) return -1;   // a cut group
+  const int64_t lo = pos0 < win0 ? pos0 / g : nG;
+  const int64_t hi = end < win0 ? end / g : nG;
+  return hi > lo ? hi - lo : 0;
+}
+
+lca_status lca_decode_partial(lca_plan* p, const void* q_c, const void* q_r, const void* c_slice,
+                              const void* k_slice, int64_t n_tok, int64_t pos0, int64_t L, int g,
+                              int w, float* part_mz, float* part_o, int32_t* anchor, void* stream) {
+  if (!p || !part_mz || !part_o || g < 1 || w < 0 || L < 1) return LCA_ERR_INVALID_ARG;
+  const int64_t ng = lca_slice_groups(L, g, w, pos0, n_tok);
+  if (ng < 0) return LCA_ERR_INVALID_ARG;
+  const int64_t win0 = lca_num_groups(L, g, w) * g;
+  const Slice sl = {std::max<int64_t>(0, win0 - pos0), pos0, part_mz};
+  if (n_tok == 0) {   // an empty slice: M = -inf, Z = 0, O = 0 (the combine over no parts)
+    if (!aligned16(part_mz) || !aligned16(part_o)) return LCA_ERR_ALIGNMENT;
+    lca::CombineParams cp = {};
+    cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = part_o; cp.out_mz = part_mz;
+    cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 0; cp.n_split = 0;
+    return launch_combine(p, cp, static_cast<cudaStream_t>(stream), false);
+  }
+  // a slice that starts inside the window holds no group: any g will do
+  const int gg = ng > 0 ? g : 1;
+  return decode_rows(p, q_c, q_r, c_slice, k_slice, n_tok, gg, ng, part_o, ng > 0 ? anchor : nullptr,
+                     stream, sl);
+}
+
+lca_status lca_merge_partials(lca_plan* p, int n_parts, const float* part_mz, const float* part_o,
+                              float* out, void* stream) {
+  if (!p || n_parts < 1 || !part_mz || !part_o || !out) return LCA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
+  if (dev != p->device) return LCA_ERR_PLAN_MISMATCH;
+  lca::CombineParams cp = {};
+  cp.part_o = part_o; cp.part_mz = part_mz; cp.out = out;
+  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 2; cp.n_split = n_parts;
+  return launch_combine(p, cp, static_cast<cudaStream_t>(stream), false);
+}
+
 lca_status lca_get_device_error(lca_plan* p, void* stream) {
   if (!p) return LCA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -436,6 +733,7 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
   if (cudaMemcpy(host, p->err, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess)
     return LCA_ERR_CUDA;
   if (host[0] != 0 && cudaMemset(p->err, 0, sizeof(host)) != cudaSuccess) return LCA_ERR_CUDA;
+  if (host[0] & lca::kErrCheck) return LCA_ERR_DEVICE_CHECK;
   return host[0] != 0 ? LCA_ERR_DEVICE_TIMEOUT : LCA_OK;
 }
 
@@ -445,7 +743,8 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
 // this entry point runs the same kernels as lca_decode with the fixed
 // file-scope scratch above in place of a plan's workspace, and allocates
 // nothing.  The first call on a device looks up the scratch's address there
-// (cudaGetSymbolAddress) and its SM count, under a mutex, so concurrent first
+// (cudaGetSymbolAddress), its SM count and how many two-CTA clusters fit
+// (cudaOccupancyMaxActiveClusters), under a mutex, so concurrent first
 // calls from several host threads are safe; later calls read the cached
 // values without locking.
 lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, const void* q_c,
@@ -453,6 +752,7 @@ lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, cons
                               int w, float* out, int32_t* anchor, void* stream) {
   static std::atomic<float*> scratch[kMaxDevices];   // the scratch's address, per device
   static std::atomic<int> sms[kMaxDevices];
+  static std::atomic<int> pair_clusters[kMaxDevices];
   static std::mutex first_call;
   if (B < 1 || H < 1 || d_c < 1 || d_r < 1 || L < 1 || g < 1 || w < 0) return LCA_ERR_INVALID_ARG;
   if (!q_c || !q_r || !c_kv || !k_r || !out) return LCA_ERR_INVALID_ARG;
@@ -471,6 +771,7 @@ lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, cons
       if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return LCA_ERR_CUDA;
       sms[dev].store(n_sm, std::memory_order_relaxed);
+      pair_clusters[dev].store(pair_cluster_capacity(n_sm), std::memory_order_relaxed);
       scratch[dev].store(static_cast<float*>(ptr), std::memory_order_release);
     }
   }
@@ -489,16 +790,15 @@ lca_status lca_decode_noalloc(int B, int H, int d_c, int d_r, lca_dtype dt, cons
   plan.num_sms = sms[dev].load(std::memory_order_relaxed);
   plan.tc_shape = dt == LCA_BF16 && d_c == lca::tc::kDC && d_r == lca::tc::kDR &&
                   (H % lca::tc::kHC) == 0;
-  plan.ws_slots = cap;   // run_simt and run_tc refuse a launch that needs more slots
+  plan.pair_shape = plan.tc_shape && (H % lca::pair::kHeads) == 0;
+  plan.pair_clusters = pair_clusters[dev].load(std::memory_order_relaxed);
+  // run_simt refuses a launch that needs more slots; the tensor-core paths cut
+  // the context into at most cap - B + 1 tile ranges
+  plan.ws_slots = cap;
   plan.part_o = base;
   plan.part_mz = base + kNoAllocOFloats;
   plan.err = reinterpret_cast<int*>(base + kNoAllocErrOffset);
   plan.timeout_ns = kDefaultTimeoutNs;
-  if (plan.tc_shape) {   // as many tile ranges as the scratch holds partials for
-    const int64_t n_hb = H / lca::tc::kHC;
-    plan.num_ctas = (int)std::min<int64_t>(plan.num_sms, n_hb * (cap - B + 1));
-    if (plan.num_ctas < n_hb) plan.num_ctas = (int)n_hb;
-  }
   // The kernels only OR into the error word, so it must start each call at zero.
   if (cudaMemsetAsync(plan.err, 0, 2 * sizeof(int), static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)

@@ -18,6 +18,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "checks.cuh"
+
 namespace lca {
 
 constexpr int kSimtThreads = 256;
@@ -49,6 +51,12 @@ struct SimtParams {
   int32_t* anchor;   // [B][H][nG] or null when nG == 0
   float* part_o;     // [B * n_split][H][d_c]
   float* part_mz;    // [B * n_split][H][2]
+  int64_t bias_rows; // rows [0, bias_rows) get `bias` added to their score (stored-cache
+  float bias;        // decode: the condensed entries; 0 rows otherwise)
+  int64_t win0;      // first window token, in this cache's rows (n_G g for a whole context)
+  int64_t pos0;      // position of row 0 in the context: anchors are written as pos0 + row
+  int64_t ws_slots;  // slots of part_o / part_mz (range checks)
+  int* err;          // device error word (range checks)
 };
 
 constexpr int kSimtTileMax = 1024;
@@ -99,7 +107,7 @@ lca_simt_kernel(const SimtParams p) {
   for (int i = tid; i < p.d_c; i += kSimtThreads) qc[i] = load_elem(qc_g + i);
   for (int i = tid; i < p.d_r; i += kSimtThreads) qr[i] = load_elem(qr_g + i);
 
-  const int64_t win0 = p.nG * p.g;  // first uncompressed (window) token
+  const int64_t win0 = p.win0;      // first uncompressed (window) token
   const int64_t s0 = (int64_t)split * p.split_len;
   const int64_t s1 = (p.L < s0 + p.split_len) ? p.L : s0 + p.split_len;
 
@@ -121,13 +129,14 @@ lca_simt_kernel(const SimtParams p) {
       for (int d = lane; d < p.d_r; d += 32) r = fmaf(qr[d], load_elem(krow + d), r);
       a = warp_sum(a);
       r = warp_sum(r);
-      if (lane == 0) { sc[tt] = a; sr[tt] = r; }
+      if (t0 + tt < p.bias_rows) r += p.bias;
+      if (lane == 0 && LCA_CHECK(p.err, tt < kSimtTileMax, 0xC01)) { sc[tt] = a; sr[tt] = r; }
     }
     __syncthreads();
     // ---- condense: one thread per group, starting token of the group
     for (int tt = tid; tt < n; tt += kSimtThreads) {
       const int64_t t = t0 + tt;
-      if (t < win0 && (t % p.g) == 0) {
+      if (t < win0 && (t % p.g) == 0 && LCA_CHECK(p.err, tt + p.g <= kSimtTileMax, 0xC02)) {
         float m = sc[tt] + sr[tt];
         int amax = tt;
         for (int u = tt + 1; u < tt + p.g; ++u) {
@@ -143,7 +152,8 @@ lca_simt_kernel(const SimtParams p) {
         glog[tt] = num / den + sr[amax];
         const float inv = 1.f / den;
         for (int u = tt; u < tt + p.g; ++u) pw[u] = expf(sc[u] + sr[u] - m) * inv;  // w_t
-        p.anchor[((int64_t)b * p.H + h) * p.nG + t / p.g] = (int32_t)(t0 + amax);
+        if (LCA_CHECK(p.err, t / p.g < p.nG, 0xC03))
+          p.anchor[((int64_t)b * p.H + h) * p.nG + t / p.g] = (int32_t)(p.pos0 + t0 + amax);
       }
     }
     __syncthreads();
@@ -193,6 +203,7 @@ lca_simt_kernel(const SimtParams p) {
   }
 
   const int64_t slot = (int64_t)b * p.n_split + split;
+  if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xC04)) return;
   float* po = p.part_o + (slot * p.H + h) * p.d_c;
 #pragma unroll
   for (int k = 0; k < kDPerThread; ++k) {

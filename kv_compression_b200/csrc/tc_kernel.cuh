@@ -120,6 +120,11 @@ struct TcParams {
   int* err;            // device error word [2]
   uint64_t timeout_ns;
   int debug_skip_load;
+  int64_t bias_rows;   // rows [0, bias_rows) get `bias` added to their score (stored-cache
+  float bias;          // decode with n_G = 0: the condensed entries; 0 rows otherwise)
+  int64_t win0;        // first window token, in this cache's rows (n_G g for a whole context)
+  int64_t pos0;        // position of row 0 in the context (a slice's offset): anchors are
+                       // written as pos0 + row, and groups start at rows that are multiples of g
 };
 
 struct Bars {
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   const int64_t u0 = c * p.U / p.G;
   const int64_t u1 = (c + 1) * p.U / p.G;
   const int64_t n_tiles = u1 - u0;
-  const int64_t win0 = p.nG * g;
+  const int64_t win0 = p.win0;
   // (sequence, tile within it) of the range's first tile; each role then steps
   // its own copy once per tile rather than dividing
   const int64_t seq0 = u0 / p.tiles_per_seq;
@@ -592,6 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       const int64_t t = tok0 + row;
       const bool valid = t < p.L;
       const bool grouped = t < win0;
+      if (t < p.bias_rows) {
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) s[h] += p.bias;
+      }
       const bool tile_groups = (g > 1) && (tok0 < win0);   // tile-uniform
       int32_t* anc = p.anchor + ((int64_t)b * p.H + h0 + kHH * hh) * p.nG;
 
@@ -601,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       for (int h = 0; h < kHH; ++h) { kj[h] = 0.f; ent[h] = valid ? s[h] : -INFINITY; }
       if (g == 1 && grouped) {
 #pragma unroll
-        for (int h = 0; h < kHH; ++h) anc[(int64_t)h * p.nG + t] = (int32_t)t;
+        for (int h = 0; h < kHH; ++h) anc[(int64_t)h * p.nG + t] = (int32_t)(p.pos0 + t);
       }
       if (tile_groups) {
         const int64_t jg = t / g;                 // this token's group (if grouped)
@@ -650,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
           const bool writer = g > 32 ? (lane == 0 && (q4 & (g / 32 - 1)) == 0) : (lane & (W - 1)) == 0;
           if (writer) {
 #pragma unroll
-            for (int h = 0; h < kHH; ++h) anc[(int64_t)h * p.nG + jg] = (int32_t)(tok0 + a[h]);
+            for (int h = 0; h < kHH; ++h) anc[(int64_t)h * p.nG + jg] = (int32_t)(p.pos0 + tok0 + a[h]);
           }
         }
       }

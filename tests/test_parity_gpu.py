@@ -50,6 +50,94 @@ def test_small_bf16(case, kernel):
     compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=g)
 
 
+# (B, H, L, g, w) for the two-CTA kernel (128 heads per cluster, 64-token tiles)
+PAIR = [
+    (2, 128, 1000, 16, 100),    # ragged tail (1000 = 15*64 + 40)
+    (1, 128, 4096, 4, 512),
+    (3, 128, 777, 64, 0),       # a group spans both token halves, no window
+    (2, 128, 2048, 32, 7),      # leftovers join the window
+    (1, 128, 300, 1, 0),        # g = 1: every token its own group
+    (2, 128, 500, 8, 600),      # w >= L: nothing condensed
+    (5, 128, 130, 2, 3),        # many short sequences
+    (1, 256, 1500, 16, 64),     # two head blocks
+    (1, 128, 1, 1, 0),          # a single token
+    (2, 128, 65, 32, 1),        # one full tile plus one token
+    (2, 128, 96, 32, 0),        # a tile whose second half is past L
+]
+
+
+@pytest.mark.parametrize("case", PAIR, ids=_ids)
+def test_pair_kernel_small(case):
+    """The two-CTA kernel (d_c split across a cluster, partial scores and P
+    exchanged through distributed shared memory) against the oracle."""
+    B, H, L, g, w = case
+    wl = workloads.small("t", B=B, H=H, L=L, g=g, w=w, seed=B * 1000 + L + 7)
+    x = workloads.generate(wl)
+    plan = make_plan(wl)
+    assert plan.kernel(L, g, w) == "tcgen05_pair"
+    out, anc = run_lca(plan, DeviceInputs(x), g, w)
+    ref = oracle_lca(x, g, w)
+    compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=g)
+
+
+def test_pair_kernel_matches_the_16_head_kernel():
+    """At H = 128 both tensor-core kernels take the shape; they must agree with
+    each other as closely as each agrees with the oracle."""
+    wl = workloads.small("t", B=2, H=128, L=3000, g=16, w=200, seed=21)
+    x = workloads.generate(wl)
+    d = DeviceInputs(x)
+    a_pair, anc_pair = run_lca(make_plan(wl, {kvc.OPT_KERNEL: 3}), d, wl.g, wl.w)
+    a_tc, anc_tc = run_lca(make_plan(wl, {kvc.OPT_KERNEL: 2}), d, wl.g, wl.w)
+    ref = oracle_lca(x, wl.g, wl.w)
+    compare(a_pair, anc_pair, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+    compare(a_tc, anc_tc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+    assert rel_err(a_pair, a_tc) <= BF16_TOL
+
+
+def test_pair_kernel_rescale():
+    """Scores that rise by far more than the rescale threshold inside a range:
+    token rows late in the sequence are scaled so that their scores exceed the
+    first tile's maximum by ~30 (natural log units), which forces the reference
+    max to rise and both CTAs to rescale the affected heads' O rows."""
+    wl = workloads.small("t", B=1, H=128, L=2048, g=16, w=128, seed=23)
+    x = workloads.generate(wl)
+    from workloads import bf16_bits_to_f32, f32_to_bf16_bits
+    c = bf16_bits_to_f32(x.c_kv).copy()
+    k = bf16_bits_to_f32(x.k_r).copy()
+    qdir = np.concatenate([bf16_bits_to_f32(x.q_c[0, :64]), bf16_bits_to_f32(x.q_r[0, :64])], axis=1)
+    u = qdir.mean(axis=0)
+    u /= np.linalg.norm(u)
+    for t in (700, 1300, 1333, 1990):       # several rises, one in the window
+        row = (40.0 * np.sqrt(576.0) * u).astype(np.float32)
+        c[0, t] = row[:512]
+        k[0, t] = row[512:]
+    x.c_kv = f32_to_bf16_bits(c)
+    x.k_r = f32_to_bf16_bits(k)
+    d = DeviceInputs(x)
+    plan = make_plan(wl)
+    assert plan.kernel(wl.L, wl.g, wl.w) == "tcgen05_pair"
+    out, anc = run_lca(plan, d, wl.g, wl.w)
+    ref = oracle_lca(x, wl.g, wl.w)
+    compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+    for n in (2, 4):                          # fewer, longer ranges: rises mid-range
+        out, anc = run_lca(make_plan(wl, {kvc.OPT_NUM_CTAS: n}), d, wl.g, wl.w)
+        compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+
+
+def test_pair_ranges_spanning_sequences():
+    """Few clusters: every tile range of the two-CTA kernel crosses sequence
+    boundaries (query reloads, partials in several slots)."""
+    wl = workloads.small("t", B=4, H=128, L=1000, g=16, w=50, seed=27)
+    x = workloads.generate(wl)
+    d = DeviceInputs(x)
+    ref = oracle_lca(x, wl.g, wl.w)
+    for n in (2, 4, 6, 12, 32, 148):
+        plan = make_plan(wl, {kvc.OPT_NUM_CTAS: n})
+        assert plan.kernel(wl.L, wl.g, wl.w) == "tcgen05_pair"
+        out, anc = run_lca(plan, d, wl.g, wl.w)
+        compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+
+
 def test_ranges_spanning_sequences():
     """Few CTAs: every tile range crosses sequence boundaries (query reloads)."""
     wl = workloads.small("t", B=4, H=32, L=1000, g=16, w=50, seed=7)
@@ -76,11 +164,12 @@ def test_tiny_f32_config():
     assert rel_err(dense, oracle_dense(x)) <= F32_TOL
 
 
-@pytest.mark.parametrize("kernel", ["tcgen05", "simt"])
+@pytest.mark.parametrize("kernel", ["tcgen05", "simt", "tcgen05_pair"])
 def test_dense_bf16(kernel):
-    wl = workloads.small("t", B=2, H=16, L=1500, g=1, w=0, seed=11)
+    H = 128 if kernel == "tcgen05_pair" else 16
+    wl = workloads.small("t", B=2, H=H, L=1500, g=1, w=0, seed=11)
     x = workloads.generate(wl)
-    plan = make_plan(wl, {kvc.OPT_FORCE_SIMT: 1} if kernel == "simt" else None)
+    plan = make_plan(wl, {kvc.OPT_KERNEL: kvc.KERNEL_CODES[kernel]})
     out = run_dense(plan, DeviceInputs(x))
     assert rel_err(out, oracle_dense(x)) <= BF16_TOL
 

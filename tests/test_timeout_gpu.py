@@ -33,3 +33,23 @@ def test_wait_timeout_is_reported_and_recovers():
     plan.set(kvc.OPT_DEBUG_SKIP_LOAD, 0)
     got, got_anc = run_lca(plan, d, wl.g, wl.w)
     compare(got, got_anc, oracle_lca(x, wl.g, wl.w), BF16_TOL, exact_anchors=False)
+
+
+def test_pair_kernel_wait_timeout_is_reported_and_recovers():
+    """The same on the two-CTA kernel (H = 128): the producer of each CTA skips
+    its first K_R load, so the score MMA issuer's wait runs out; the peer CTA's
+    waits for the partial scores run out in turn.  Both CTAs record the
+    timeout, leave their loops, meet at the cluster barrier and free TMEM."""
+    wl = workloads.small("t", B=2, H=128, L=1000, g=16, w=100, seed=22)
+    x = workloads.generate(wl)
+    d = DeviceInputs(x)
+    plan = make_plan(wl, {kvc.OPT_WAIT_TIMEOUT_NS: 50_000_000, kvc.OPT_DEBUG_SKIP_LOAD: 1})
+    assert plan.kernel(wl.L, wl.g, wl.w) == "tcgen05_pair"
+    out = torch.zeros(wl.B, wl.H, wl.d_c, device="cuda")
+    anc = torch.zeros(wl.B, wl.H, wl.n_groups, dtype=torch.int32, device="cuda")
+    plan.decode(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, wl.g, wl.w, out, anc)
+    assert plan.device_error() == kvc.LCA_ERR_DEVICE_TIMEOUT
+    assert plan.device_error() == kvc.LCA_OK
+    plan.set(kvc.OPT_DEBUG_SKIP_LOAD, 0)
+    got, got_anc = run_lca(plan, d, wl.g, wl.w)
+    compare(got, got_anc, oracle_lca(x, wl.g, wl.w), BF16_TOL, exact_anchors=False)
