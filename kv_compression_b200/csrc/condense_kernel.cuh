@@ -127,6 +127,124 @@ __global__ void __launch_bounds__(kCondThreads) lca_condense_kernel(const Conden
   }
 }
 
+// The same for bf16 latents with d_c = 512 and d_r = 64 (every benchmark
+// shape): lane l owns latent dims [16 l, 16 l + 16) -- two 16-byte loads a
+// row -- and RoPE dims [2 l, 2 l + 2); four tokens' rows are loaded before
+// their scores are reduced, so a warp keeps several rows in flight.
+constexpr int kCondFastDc = 512, kCondFastDr = 64, kCondBatch = 4;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(kCondThreads) lca_condense_fast_kernel(const CondenseParams p) {
+  __shared__ float cq[kCondFastDc + kCondFastDr];   // the mean query
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const __nv_bfloat16* qc_b = static_cast<const __nv_bfloat16*>(p.q_c) + (int64_t)b * p.H * kCondFastDc;
+  const __nv_bfloat16* qr_b = static_cast<const __nv_bfloat16*>(p.q_r) + (int64_t)b * p.H * kCondFastDr;
+  const float inv_h = 1.f / (float)p.H;
+  for (int d = tid; d < kCondFastDc + kCondFastDr; d += kCondThreads) {
+    float acc = 0.f;
+    if (d < kCondFastDc) {
+      for (int h = 0; h < p.H; ++h) acc += load_elem(qc_b + (int64_t)h * kCondFastDc + d);
+    } else {
+      for (int h = 0; h < p.H; ++h) acc += load_elem(qr_b + (int64_t)h * kCondFastDr + (d - kCondFastDc));
+    }
+    cq[d] = acc * inv_h;
+  }
+  __syncthreads();
+  float qc[16], qr[2];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) qc[i] = cq[16 * lane + i];
+  qr[0] = cq[kCondFastDc + 2 * lane];
+  qr[1] = cq[kCondFastDc + 2 * lane + 1];
+
+  const uint8_t* c_b = static_cast<const uint8_t*>(p.c_kv) + (int64_t)b * p.L * kCondFastDc * 2;
+  const uint8_t* k_b = static_cast<const uint8_t*>(p.k_r) + (int64_t)b * p.L * kCondFastDr * 2;
+  uint8_t* cd = static_cast<uint8_t*>(p.c_dst);
+  uint8_t* kd = static_cast<uint8_t*>(p.k_dst);
+  for (int64_t jj = (int64_t)blockIdx.x * kCondWarps + warp; jj < p.n;
+       jj += (int64_t)gridDim.x * kCondWarps) {
+    const int64_t t0 = (p.j0 + jj) * p.g;
+    if (!LCA_CHECK(p.err, t0 + p.g <= p.L && p.dst_row0 + jj < p.dst_rows, 0xC22)) continue;
+    float acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    float m = -INFINITY, den = 0.f;
+    int a = 0;
+    for (int u0 = 0; u0 < p.g; u0 += kCondBatch) {
+      uint4 cv[kCondBatch][2];
+      uint32_t kv[kCondBatch];
+#pragma unroll
+      for (int e = 0; e < kCondBatch; ++e) {
+        const int u = u0 + e < p.g ? u0 + e : p.g - 1;     // a short group repeats its last row
+        const uint4* crow = reinterpret_cast<const uint4*>(c_b + (t0 + u) * (kCondFastDc * 2)) + 2 * lane;
+        cv[e][0] = __ldg(crow);
+        cv[e][1] = __ldg(crow + 1);
+        kv[e] = __ldg(reinterpret_cast<const uint32_t*>(k_b + (t0 + u) * (kCondFastDr * 2)) + lane);
+      }
+      float part[kCondBatch];
+#pragma unroll
+      for (int e = 0; e < kCondBatch; ++e) {
+        float f[16];
+        bf16x8_to_f32(cv[e][0], f);
+        bf16x8_to_f32(cv[e][1], f + 8);
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s = fmaf(qc[i], f[i], s);
+        s = fmaf(qr[0], __uint_as_float(kv[e] << 16), s);
+        s = fmaf(qr[1], __uint_as_float(kv[e] & 0xFFFF0000u), s);
+        part[e] = s;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int e = 0; e < kCondBatch; ++e) part[e] += __shfl_xor_sync(0xffffffffu, part[e], o);
+#pragma unroll
+      for (int e = 0; e < kCondBatch; ++e) {
+        if (u0 + e >= p.g) break;                          // warp-uniform
+        const float s = part[e];                           // the same bits in every lane
+        float f[16];
+        bf16x8_to_f32(cv[e][0], f);
+        bf16x8_to_f32(cv[e][1], f + 8);
+        if (s > m) {                                       // strict: the lowest index keeps a tie
+          const float alpha = __expf(m - s);               // 0 on the first token
+          den *= alpha;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] *= alpha;
+          m = s;
+          a = u0 + e;
+        }
+        const float w = __expf(s - m);
+        den += w;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+      }
+    }
+    const float inv = 1.f / den;
+    const int64_t row = (int64_t)b * p.dst_rows + p.dst_row0 + jj;
+    uint32_t packed[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+      packed[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    uint4* cdst = reinterpret_cast<uint4*>(cd + row * (kCondFastDc * 2)) + 2 * lane;
+    cdst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    cdst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    // the anchor's RoPE key, copied as stored
+    reinterpret_cast<uint32_t*>(kd + row * (kCondFastDr * 2))[lane] =
+        __ldg(reinterpret_cast<const uint32_t*>(k_b + (t0 + a) * (kCondFastDr * 2)) + lane);
+    if (lane == 0) p.anchor[(int64_t)b * p.n + jj] = (int32_t)(t0 + a);
+  }
+}
+
 // Copy rows [src_row0, src_row0 + n) of every sequence (src_rows rows each) to
 // rows [dst_row0, dst_row0 + n) (dst_rows rows each), `row_bytes` bytes a row
 // (a multiple of 16), 16 bytes per thread.

@@ -275,6 +275,7 @@ lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_k
   tp.anchor = anchor; tp.part_o = p->part_o; tp.part_mz = p->part_mz; tp.err = p->err;
   tp.timeout_ns = p->timeout_ns; tp.debug_skip_load = p->debug_skip_load;
   tp.bias_rows = p->bias_rows; tp.bias = p->bias; tp.win0 = sl.win0; tp.pos0 = sl.pos0;
+  tp.ws_slots = p->ws_slots;
   const unsigned grid = (unsigned)(G * n_hb);
   if (launch_tc_g(nG > 0 ? g : 1, tp, grid, stream, p->device) != cudaSuccess) return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
@@ -365,7 +366,7 @@ lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c
   if (!make_map(&pp.tm_c, c_kv, 512, rows, lca::pair::kT) ||
       !make_map(&pp.tm_k, k_r, 64, rows, lca::pair::kT) ||
       !make_map(&pp.tm_qc, q_c, 512, qrows, lca::pair::kHeads) ||
-      !make_map(&pp.tm_qr, q_r, 64, qrows, lca::pair::kOwn))
+      !make_map(&pp.tm_qr, q_r, 64, qrows, lca::pair::kHeads))
     return LCA_ERR_CUDA;
   const int n_hb = p->H / lca::pair::kHeads;
   const int64_t tps = ceil_div(L, lca::pair::kT);
@@ -379,6 +380,7 @@ lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c
   pp.anchor = anchor; pp.part_o = p->part_o; pp.part_mz = p->part_mz; pp.err = p->err;
   pp.timeout_ns = p->timeout_ns; pp.debug_skip_load = p->debug_skip_load;
   pp.bias_rows = p->bias_rows; pp.bias = p->bias; pp.win0 = sl.win0; pp.pos0 = sl.pos0;
+  pp.ws_slots = p->ws_slots;
   if (launch_pair_g(nG > 0 ? g : 1, pp, (unsigned)(G * n_hb), stream, p->device) != cudaSuccess)
     return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
@@ -440,7 +442,11 @@ lca_status launch_condense(const lca_plan* p, const lca::CondenseParams& cp, cud
                                                                  ceil_div(4LL * p->num_sms, p->B)));
   dim3 grid((unsigned)per_seq, (unsigned)p->B, 1);
   const size_t smem = (size_t)(p->d_c + p->d_r) * sizeof(float);
-  if (p->dt == LCA_F32)
+  const bool fast = p->dt == LCA_BF16 && p->d_c == lca::kCondFastDc && p->d_r == lca::kCondFastDr &&
+                    aligned16(cp.c_kv) && aligned16(cp.c_dst) && aligned16(cp.k_r) && aligned16(cp.k_dst);
+  if (fast)
+    lca::lca_condense_fast_kernel<<<grid, lca::kCondThreads, 0, stream>>>(cp);
+  else if (p->dt == LCA_F32)
     lca::lca_condense_kernel<float><<<grid, lca::kCondThreads, smem, stream>>>(cp);
   else
     lca::lca_condense_kernel<__nv_bfloat16><<<grid, lca::kCondThreads, smem, stream>>>(cp);
@@ -699,7 +705,9 @@ lca_status lca_decode_partial(lca_plan* p, const void* q_c, const void* q_r, con
   const int64_t ng = lca_slice_groups(L, g, w, pos0, n_tok);
   if (ng < 0) return LCA_ERR_INVALID_ARG;
   const int64_t win0 = lca_num_groups(L, g, w) * g;
-  const Slice sl = {std::max<int64_t>(0, win0 - pos0), pos0, part_mz};
+  // The slice's own rows hold its groups: rows past n_tok (a partial last tile
+  // reads the next sequence's rows) must never count as grouped.
+  const Slice sl = {std::min<int64_t>(n_tok, std::max<int64_t>(0, win0 - pos0)), pos0, part_mz};
   if (n_tok == 0) {   // an empty slice: M = -inf, Z = 0, O = 0 (the combine over no parts)
     if (!aligned16(part_mz) || !aligned16(part_o)) return LCA_ERR_ALIGNMENT;
     lca::CombineParams cp = {};

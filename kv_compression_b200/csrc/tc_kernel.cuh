@@ -47,6 +47,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "checks.cuh"
 #include "ptx.cuh"
 
 namespace lca {
@@ -125,6 +126,7 @@ struct TcParams {
   int64_t win0;        // first window token, in this cache's rows (n_G g for a whole context)
   int64_t pos0;        // position of row 0 in the context (a slice's offset): anchors are
                        // written as pos0 + row, and groups start at rows that are multiples of g
+  int64_t ws_slots;    // slots of part_o / part_mz (range checks)
 };
 
 struct Bars {
@@ -156,14 +158,18 @@ __device__ __forceinline__ void record_timeout(volatile int* abort, const TcPara
 
 // Bounded wait.  Returns false when the CTA's abort flag is set (if honoured)
 // or when the bound runs out (then the flag and the error word are set).
+// The thread sleeps in hardware between probes (up to 1 us each, woken when
+// the phase completes), so waiting threads take no issue slots from the
+// softmax warps on their sub-partition.
 __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const TcParams& p, int where, bool honour_abort) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+  constexpr uint32_t kSleepNs = 1000;
+  if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t spin = 1;; ++spin) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
     if (honour_abort && *abort) return false;
-    if ((spin & 63u) == 0 && ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+    if ((spin & 7u) == 0 && ptx::globaltimer_ns() - t0 > p.timeout_ns) {
       record_timeout(abort, p, where);
       return false;
     }
@@ -362,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     bool ok = true;
     const int64_t T = n_tiles;
     auto issue = [&](uint64_t* full, int slot, int32_t row, int pr, uint64_t policy) {
+      if (!LCA_CHECK(p.err, slot >= 0 && slot < kNPair && pr >= 0 && pr < kPairsPerTile, 0xD01)) return;
       ptx::mbar_arrive_expect_tx(full, kPairBytes);
       uint8_t* dst = smem + kOffPair + slot * kPairBytes;
       ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, full, policy);
@@ -495,6 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       for (int pr = 0; pr < kPairsPerTile; ++pr) {   // sc += C_KV[:, pair] . q_c[pair]^T
         const int64_t n = kHeld * t + (pr - kNA);     // ring B index of a held pair
         const int cs = pr < kNA ? pr : kNA + (int)(n % kNB);   // shared-memory slot
+        if (!LCA_CHECK(p.err, cs >= 0 && cs < kNPair && buf < 2, 0xD02)) { ok = false; break; }
         ok = pr < kNA ? bounded_wait(&bb.full_as[pr], (uint32_t)t & 1, abort_flag, p, 0x203, true)
                       : bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x203, true);
         if (!ok) break;
@@ -540,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         const int m = (mm + kNA) % kPairsPerTile;   // held pairs (ring B) first, then the reloads
         const int64_t n = kHeld * j + (m - kNA);      // ring B index of a held pair
         const int cs = m >= kNA ? kNA + (int)(n % kNB) : m;  // shared-memory slot
+        if (!LCA_CHECK(p.err, cs >= 0 && cs < kNPair && m < kPairsPerTile, 0xD03)) break;
         const bool okw = m >= kNA ? bounded_wait(&bb.full_b[cs - kNA], (uint32_t)(n / kNB) & 1, abort_flag, p, 0x206, true)
                                   : bounded_wait(&bb.full_ar[m], (uint32_t)j & 1, abort_flag, p, 0x206, true);
         if (!okw) break;
@@ -610,7 +619,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       for (int h = 0; h < kHH; ++h) { kj[h] = 0.f; ent[h] = valid ? s[h] : -INFINITY; }
       if (g == 1 && grouped) {
 #pragma unroll
-        for (int h = 0; h < kHH; ++h) anc[(int64_t)h * p.nG + t] = (int32_t)(p.pos0 + t);
+        for (int h = 0; h < kHH; ++h)
+          if (LCA_CHECK(p.err, t < p.nG && h0 + kHH * hh + h < p.H, 0xD04))
+            anc[(int64_t)h * p.nG + t] = (int32_t)(p.pos0 + t);
       }
       if (tile_groups) {
         const int64_t jg = t / g;                 // this token's group (if grouped)
@@ -659,7 +670,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
           const bool writer = g > 32 ? (lane == 0 && (q4 & (g / 32 - 1)) == 0) : (lane & (W - 1)) == 0;
           if (writer) {
 #pragma unroll
-            for (int h = 0; h < kHH; ++h) anc[(int64_t)h * p.nG + jg] = (int32_t)(p.pos0 + tok0 + a[h]);
+            for (int h = 0; h < kHH; ++h)
+              if (LCA_CHECK(p.err, jg < p.nG && a[h] >= 0 && a[h] < kT, 0xD05))
+                anc[(int64_t)h * p.nG + jg] = (int32_t)(p.pos0 + tok0 + a[h]);
           }
         }
       }
@@ -736,7 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       if (i >= 2) warp_wait(&bb.o_full[buf], (uint32_t)((i - 2) >> 1) & 1, abort_flag, p, 0x305);
       // MN-major core matrices: token row -> K, head -> N (8-head blocks 2 KB apart)
       uint8_t* prow = pbase + buf * kPBytes + hh * 2048 + (row >> 3) * 128 + (row & 7) * 16;
-      *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      if (LCA_CHECK(p.err, prow + 16 <= pbase + 2 * kPBytes, 0xD06))
+        *reinterpret_cast<uint4*>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncwarp();
@@ -745,6 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       if (last_in_seg) {
         // the partial of the range's part of sequence b
         const int64_t slot = b + c;
+        const bool slot_ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xD07);
         warp_wait(&bb.o_full[buf], (uint32_t)kb & 1, abort_flag, p, 0x304);
         ptx::tc_fence_after();
 #pragma unroll 1
@@ -754,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < kHH; ++h)
-            p.part_o[(slot * p.H + h0 + kHH * hh + h) * kDC + 128 * m + row] = o[h];
+            if (slot_ok) p.part_o[(slot * p.H + h0 + kHH * hh + h) * kDC + 128 * m + row] = o[h];
         }
         ptx::tc_fence_before();
 #pragma unroll
@@ -765,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
           if (lane == 0) zred[q4 * kHC + kHH * hh + h] = z;
         }
         ptx::named_bar_sync(kSoftmaxBar, kSoftmaxThreads);
-        if (q4 == 2 && lane < kHH) {   // warps 2 and 6: heads 0-7 and 8-15
+        if (q4 == 2 && lane < kHH && slot_ok) {   // warps 2 and 6: heads 0-7 and 8-15
           float Mv = 0.f;
 #pragma unroll
           for (int h = 0; h < kHH; ++h) if (h == lane) Mv = Mh[h];

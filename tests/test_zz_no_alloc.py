@@ -46,6 +46,7 @@ def run_noalloc(wl, d, g, w):
 
 @pytest.mark.parametrize("wl,tol", [
     (workloads.small("na_bf16", B=3, H=32, L=5000, g=16, w=300, seed=41), BF16_TOL),
+    (workloads.small("na_pair", B=2, H=128, L=3000, g=16, w=300, seed=44), BF16_TOL),
     (workloads.small("na_f32", B=2, H=4, L=1500, g=8, w=100, d_c=64, d_r=16, dtype="f32",
                      seed=42), F32_TOL),
 ])
