@@ -1,7 +1,7 @@
 // pair_kernel.cuh -- LCA / dense-MLA decode for 128 heads sharing one latent,
 // on a cluster of two CTAs that split the latent width: tcgen05 tensor cores,
-// TMEM accumulators, TMA tile loads, distributed shared memory (sm_100a),
-// bf16 latents, fp32 accumulation.
+// TMEM accumulators and operands, TMA tile loads, distributed shared memory
+// (sm_100a), bf16 latents, fp32 accumulation.
 //
 // What one cluster computes ("Latent-Condensed Transformer for Efficient Long
 // Context Modeling", section 2, "O Algoritmo LCA", steps 1-3) for 128 heads of
@@ -13,43 +13,50 @@
 //   scores     S_r[128 heads x 64 tokens] = Q_c[:, dims_r] . C_KV[tile, dims_r]^T
 //              (partial over its own dims) and sr = q_r . K_R^T, in TMEM.  Each
 //              CTA sends the partial scores of its peer heads to the other CTA
-//              (st.async into its shared memory), so each head's full score
-//              sc_t = S_0 + S_1 is formed by the CTA that owns the head;
+//              (st.async into its shared memory, per lane quarter), so each
+//              head's full score sc_t = S_0 + S_1 is formed by the CTA that
+//              owns the head;
 //   condense   (step 2) two threads hold one head, 32 consecutive tokens each,
-//              so a group of g <= 32 tokens is reduced inside a thread (tree
-//              reductions): max, lowest-index argmax (the anchor a_j),
-//              e_t = e^{s_t - m_j}, den_j = sum e_t, num_j = sum e_t sc_t and the
-//              condensed logit S_j = num_j / den_j + sr_{a_j}; a 64-token group
-//              merges its two threads with a shuffle;
+//              so a group of g <= 32 tokens is reduced inside a thread: max,
+//              lowest-index argmax (the anchor a_j), e_t = e^{s_t - m_j},
+//              den_j = sum e_t, num_j = sum e_t sc_t and the condensed logit
+//              S_j = num_j / den_j + sr_{a_j}; a 64-token group merges its two
+//              threads with a shuffle;
 //   attend     (step 3) softmax over [condensed || window] against a reference
 //              max M per head: a grouped token weighs e_t e^{S_j - M} / den_j,
 //              a window token e^{s_t - M}.  The bf16 weights P[128 heads x 64
-//              tokens] (own rows written here, the peer rows copied in by the
-//              peer) feed O[128 heads x 256 dims_r] += P . C_KV[tile, dims_r] in
-//              TMEM.  M rises only when an entry exceeds it by more than 2^8; the
-//              owner then rescales the head's O row in its own TMEM at once, and
-//              the factor travels with P to the peer, which rescales its copy of
-//              the row before it accumulates that tile.
+//              tokens] are the A operand of O[128 heads x 256 dims_r] +=
+//              P . C_KV[tile, dims_r], read from TMEM: the owner writes its
+//              heads' rows there and sends them to the peer (st.async from
+//              registers), whose receiving warps write them into its TMEM.  M
+//              rises only when an entry exceeds it by more than 2^8; the factor
+//              travels with P, and whichever warp writes a head's P row also
+//              rescales that head's O row first.
 // Each CTA writes its dims of every head's partial O, the owner CTA the
 // head's (M, Z); the combine kernel merges the ranges of a sequence.
 //
 // Every C_KV byte is read from HBM once and into shared memory once (each CTA
 // loads only its half); K_R is loaded by both CTAs.
 //
+// TMEM (512 columns): O at 0 (256), partial sc in two buffers at 256 and 320,
+// sr at 384 (one buffer: it is read at the start of a tile), P in two buffers
+// at 448 and 480 (bf16 pairs), so the scores of a tile, its weights and the O
+// accumulation of the tile before overlap.
+//
 // Roles (352 threads): warp 0 lane 0 issues TMA loads; warp 1 allocates TMEM
-// and its lane 0 issues the score MMAs; warp 2 lane 0 issues the O MMAs and,
-// from the peer's rescale factors, decides whether a tile needs its peer rows
-// rescaled; warps 3-6 run the softmax of the own heads of lane quarter
-// (warp % 4); warps 7-10 ship the partial scores of the peer heads of their
-// quarter and, one tile behind, rescale and write out those heads' O rows.
-// Waits sleep in hardware (mbarrier.try_wait with a time hint) and are
-// bounded; when a bound runs out the CTA records the error, stops issuing
+// and its lane 0 issues the score MMAs; warp 2 lane 0 issues the O MMAs; warps
+// 3-6 run the softmax of the own heads of lane quarter (warp % 4); warps 7-10
+// ship the partial scores of the peer heads of their quarter one tile ahead,
+// and write the peer heads' P rows (and rescale and write out their O rows).
+// Waits suspend in hardware (mbarrier.try_wait) and are bounded; when a
+// bound runs out the CTA records the error, stops issuing
 // work, waits for its own copies and MMAs in flight, frees TMEM and exits
 // after its peer.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "checks.cuh"
 #include "ptx.cuh"
@@ -72,37 +79,43 @@ constexpr int kCAtom = kT * 128;            // [64 tokens][64 bf16] = 8 KB
 constexpr int kStage = kAtoms * kCAtom;     // 32 KB
 constexpr int kKrBytes = kT * 128;          // 8 KB
 constexpr int kQrBytes = kHeads * 128;      // q_r of all heads, 16 KB
-constexpr int kPBytes = kHeads * kT * 2;    // P[128 heads][64 tokens] bf16, 16 KB
-constexpr int kPBlockBytes = 16 * kT * 2;   // the 16 own rows of one quarter, 2 KB
 constexpr int kRecvBytes = kOwn * kT * 4;   // partial scores from the peer, 16 KB
-constexpr int kAlphaBlockBytes = 16 * 4;    // the 16 own heads' rescale factors of a quarter
-constexpr int kRemoteBytes = 4 * (kPBlockBytes + kAlphaBlockBytes);   // one tile's P message
+constexpr int kPRowBytes = kT * 2;          // one head's bf16 weights of a tile
+constexpr int kPMsgAlpha = kOwn * kPRowBytes;       // offset of the factors in a P message
+constexpr int kPMsgBytes = kPMsgAlpha + kOwn * 4;   // 64 rows of P + 64 factors = 8448 B
+// Each message travels per lane quarter: the 16 heads of quarter q come from
+// the peer's warp of the same quarter and complete their own barrier, so a
+// quarter waits only for its rows and each barrier takes a quarter of the
+// transaction updates.
+constexpr int kRecvQBytes = kRecvBytes / 4;                 // 16 heads x 64 tokens x 4 B
+constexpr int kPMsgQBytes = kPMsgBytes / 4;                 // 16 rows of P + 16 factors
 constexpr int kThreads = 32 * 11;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kSleepNs = 1000;         // a waiting thread sleeps up to 1 us per probe
 
 // shared memory map (offsets from a 1024-byte aligned base; equal in both CTAs)
 constexpr int kOffQc = 0;
 constexpr int kOffQr = kOffQc + kAtoms * kQcAtom;
 constexpr int kOffC = kOffQr + kQrBytes;
 constexpr int kOffKr = kOffC + kNS * kStage;
-constexpr int kOffP = kOffKr + kNKr * kKrBytes;
-constexpr int kOffRecv = kOffP + kPBytes;
-constexpr int kOffAlpha = kOffRecv + kRecvBytes;           // float [128]: rescale factor per head
-constexpr int kOffFlag = kOffAlpha + kHeads * 4;           // int [2]: peer rows need a rescale
-constexpr int kOffBar = kOffFlag + 16;
-constexpr int kNumBars = 2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 1 + 2 + 2;
+constexpr int kOffRecv = kOffKr + kNKr * kKrBytes;
+constexpr int kOffPMsg = kOffRecv + kRecvBytes;            // [2] P messages from the peer
+constexpr int kOffBar = kOffPMsg + 2 * kPMsgBytes;
+constexpr int kNumBars = 2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 8 + 8 + 2 + 2 + 2;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget of one sm_100 CTA");
-static_assert(kOffC % 1024 == 0 && kOffKr % 1024 == 0 && kOffP % 1024 == 0 && kOffQr % 1024 == 0,
-              "swizzle atoms");
+static_assert(kOffC % 1024 == 0 && kOffKr % 1024 == 0 && kOffQr % 1024 == 0, "swizzle atoms");
+static_assert(kOffRecv % 16 == 0 && kOffPMsg % 16 == 0 && kPMsgBytes % 16 == 0 && kOffBar % 8 == 0,
+              "st.async targets and barriers");
 
-// TMEM columns: S buffer b: partial sc at 128 b, sr at 128 b + 64;  O at 256.
-constexpr uint32_t kColO = 256;
+// TMEM columns
+constexpr uint32_t kColO = 0;       // O [128 heads x 256 dims] fp32
+constexpr uint32_t kColSc = 256;    // partial sc, buffer b at 256 + 64 b
+constexpr uint32_t kColSr = 384;    // sr
+constexpr uint32_t kColP = 448;     // P, buffer b at 448 + 32 b (64 bf16 = 32 columns a row)
 
 constexpr int kErrTimeout = 1;
 
@@ -139,16 +152,16 @@ struct Bars {
   uint64_t* kr_empty;    // [kNKr] released after the sr MMAs
   uint64_t* q_full;
   uint64_t* q_empty;
-  uint64_t* s_full;      // [2] the scores of a tile are in TMEM
-  uint64_t* s_empty;     // [2] the softmax and shipper warps have read them
-  uint64_t* recv_full;   // the peer's partial scores of a tile landed (transaction bytes)
-  uint64_t* recv_free;   // the peer has read the partial scores this CTA sent it
-  uint64_t* p_local;     // the own rows of P are written (and copied to the peer)
-  uint64_t* p_remote;    // the peer's rows of P and its rescale factors landed
-  uint64_t* lanes_ready; // the shippers are done with everything that precedes O of a tile
-  uint64_t* dec;         // [2] the O issuer's decision for a tile (flag: rescale the peer rows)
-  uint64_t* resc_done;   // the shippers rescaled the peer rows as asked
-  uint64_t* o_done;      // [2] O of a tile is done in CTA 0 / CTA 1 (both CTAs arrive)
+  uint64_t* s_full;      // [2] the scores (partial sc in buffer b, then sr) of a tile are in TMEM
+  uint64_t* sc_full;     // [2] the partial sc of a tile is in buffer b
+  uint64_t* sc_empty;    // [2] softmax and shipper warps have read partial sc buffer b
+  uint64_t* sr_empty;    // the softmax warps have read sr
+  uint64_t* recv_full;   // [4] quarter q of the peer's partial scores landed (transaction bytes)
+  uint64_t* recv_free;   // [4] the peer's quarter q has read the partial scores sent to it
+  uint64_t* pm_full;     // [2 x 4] quarter q of the peer's P message b landed (transaction bytes)
+  uint64_t* pm_free;     // [2 x 4] the peer's quarter q has read this CTA's P message b
+  uint64_t* p_tmem;      // [2] P buffer b holds the tile's 128 rows (and O rows are rescaled)
+  uint64_t* p_free;      // [2] O of the tile that used P buffer b is done (and every O before it)
   uint64_t* drain;       // [2]
 };
 
@@ -157,15 +170,17 @@ __device__ __forceinline__ void record_timeout(volatile int* abort, const PairPa
   if (atomicOr(p.err, kErrTimeout) == 0) atomicExch(p.err + 1, where);
 }
 
-// Bounded wait; the thread sleeps in hardware between probes.  `cluster`:
+// Bounded wait.  Each probe is an mbarrier.try_wait, which suspends the
+// thread in hardware until the phase completes or a short system-defined
+// limit passes (a suspend-time hint would let it sleep past the completion:
+// measured, that added up to a microsecond to every hand-off).  `cluster`:
 // acquire at cluster scope (barriers that the peer CTA arrives on or
 // completes transactions on).
 __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const PairParams& p, int where, bool honour_abort,
                                           bool cluster) {
   auto probe = [&]() {
-    return cluster ? ptx::mbar_try_wait_cluster_sleep(bar, parity, kSleepNs)
-                   : ptx::mbar_try_wait_sleep(bar, parity, kSleepNs);
+    return cluster ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
   };
   if (probe()) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
@@ -218,32 +233,35 @@ __device__ __forceinline__ float tree_sum(const float* v) {
 }
 
 // Statistics of one group held by one thread: x[0..N) the semantic scores,
-// sr[0..N) the positional ones; on return s[] holds e_t = e^{s_t - m}.
+// sr[0..N) the positional ones; on return e[] holds e_t = e^{s_t - m}.
 // m = max s_t, a = the lowest index attaining it, sra = sr_a, den = sum e_t,
 // num = sum e_t sc_t.
 template <int N>
-__device__ __forceinline__ void group_stats(const float* x, const float* sr, float* s, float& m, int& a,
+__device__ __forceinline__ void group_stats(const float* x, const float* sr, float* e, float& m, int& a,
                                             float& sra, float& den, float& num) {
+  float s[N];
 #pragma unroll
   for (int t = 0; t < N; ++t) s[t] = x[t] + sr[t];
   m = tree_max<N>(s);
-  uint32_t hit = 0;                         // bit t: s_t is the maximum
+  // scanning down, the last hit is the lowest index attaining the maximum
+  a = 0;
+  sra = sr[0];
 #pragma unroll
-  for (int t = 0; t < N; ++t) hit |= (s[t] == m ? 1u : 0u) << t;
-  a = __ffs(hit) - 1;
-  const uint32_t low = hit & (0u - hit);    // the lowest maximum only
-  float pick[N], prod[N];
-#pragma unroll
-  for (int t = 0; t < N; ++t) pick[t] = ((low >> t) & 1u) ? sr[t] : 0.f;
-  sra = tree_sum<N>(pick);
+  for (int t = N - 1; t >= 0; --t) {
+    const bool hit = s[t] == m;
+    a = hit ? t : a;
+    sra = hit ? sr[t] : sra;
+  }
   const float mb = -m * kLog2e;
+  float n0 = 0.f, n1 = 0.f;
 #pragma unroll
   for (int t = 0; t < N; ++t) {
-    s[t] = ex2(fmaf(s[t], kLog2e, mb));
-    prod[t] = s[t] * x[t];
+    e[t] = ex2(fmaf(s[t], kLog2e, mb));
+    if (t & 1) n1 = fmaf(e[t], x[t], n1);
+    else n0 = fmaf(e[t], x[t], n0);
   }
-  den = tree_sum<N>(s);
-  num = tree_sum<N>(prod);
+  den = tree_sum<N>(e);
+  num = n0 + n1;
 }
 
 template <int LOG2G>
@@ -268,22 +286,19 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.q_full = bb.kr_empty + kNKr;
   bb.q_empty = bb.q_full + 1;
   bb.s_full = bb.q_empty + 1;
-  bb.s_empty = bb.s_full + 2;
-  bb.recv_full = bb.s_empty + 2;
-  bb.recv_free = bb.recv_full + 1;
-  bb.p_local = bb.recv_free + 1;
-  bb.p_remote = bb.p_local + 1;
-  bb.lanes_ready = bb.p_remote + 1;
-  bb.dec = bb.lanes_ready + 1;
-  bb.resc_done = bb.dec + 2;
-  bb.o_done = bb.resc_done + 1;
-  bb.drain = bb.o_done + 2;
+  bb.sc_full = bb.s_full + 2;
+  bb.sc_empty = bb.sc_full + 2;
+  bb.sr_empty = bb.sc_empty + 2;
+  bb.recv_full = bb.sr_empty + 1;
+  bb.recv_free = bb.recv_full + 4;
+  bb.pm_full = bb.recv_free + 4;
+  bb.pm_free = bb.pm_full + 8;
+  bb.p_tmem = bb.pm_free + 8;
+  bb.p_free = bb.p_tmem + 2;
+  bb.drain = bb.p_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  volatile int* dec_flag = reinterpret_cast<volatile int*>(smem + kOffFlag);
-  float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
   float* recv = reinterpret_cast<float*>(smem + kOffRecv);
-  uint8_t* pbuf = smem + kOffP;
 
   const int64_t cl = blockIdx.x >> 1;
   const int hb = (int)(cl % p.n_hb);
@@ -301,6 +316,15 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   auto last_of_part = [&](int64_t i, int64_t tile) {
     return i + 1 == n_tiles || tile + 1 == p.tiles_per_seq;
   };
+  // O of tile j (and every O before it: one thread issues them in order) is
+  // done.  Waited on the P buffer's release, whose previous phase (tile j - 2)
+  // every caller has already seen when it wrote P of tile j or j + 1: a
+  // parity wait is only sound when the barrier cannot be two phases behind.
+  auto o_complete = [&](int64_t j, int where) -> bool {
+    const bool ok = warp_wait(&bb.p_free[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, where, false);
+    if (ok) ptx::tc_fence_after();
+    return ok;
+  };
 
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) { ptx::mbar_init(&bb.c_full[i], 1); ptx::mbar_init(&bb.c_empty[i], 1); }
@@ -309,22 +333,29 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     ptx::mbar_init(bb.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bb.s_full[i], 1);
-      ptx::mbar_init(&bb.s_empty[i], 8);          // 4 softmax + 4 shipper warps
-      ptx::mbar_init(&bb.dec[i], 1);
-      ptx::mbar_init(&bb.o_done[i], 1);
+      ptx::mbar_init(&bb.sc_full[i], 1);
+      ptx::mbar_init(&bb.sc_empty[i], 8);         // 4 softmax + 4 shipper warps
+      ptx::mbar_init(&bb.p_tmem[i], 8);           // 4 softmax + 4 shipper warps
+      ptx::mbar_init(&bb.p_free[i], 1);
       ptx::mbar_init(&bb.drain[i], 1);
     }
-    ptx::mbar_init(bb.recv_full, 1);              // armed with its transaction bytes
-    ptx::mbar_init(bb.recv_free, 4);              // the peer's 4 softmax warps
-    ptx::mbar_init(bb.p_local, 4);                // this CTA's 4 softmax warps
-    ptx::mbar_init(bb.p_remote, 1);               // armed with its transaction bytes
-    ptx::mbar_init(bb.lanes_ready, 4);            // the 4 shipper warps
-    ptx::mbar_init(bb.resc_done, 4);
+    ptx::mbar_init(bb.sr_empty, 4);               // the 4 softmax warps
+    for (int q = 0; q < 4; ++q) {
+      ptx::mbar_init(&bb.recv_full[q], 1);        // armed with its transaction bytes
+      ptx::mbar_init(&bb.recv_free[q], 1);        // the peer's softmax warp of quarter q
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(&bb.pm_full[4 * b + q], 1);  // armed with its transaction bytes
+        ptx::mbar_init(&bb.pm_free[4 * b + q], 1);  // the peer's receiver warp of quarter q
+      }
+    }
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
-    // phase 0 of the two barriers the peer completes with transaction bytes
-    ptx::mbar_arrive_expect_tx(bb.recv_full, kRecvBytes);
-    ptx::mbar_arrive_expect_tx(bb.p_remote, kRemoteBytes);
+    // the first phases of the barriers the peer completes with transaction bytes
+    for (int q = 0; q < 4; ++q) {
+      ptx::mbar_arrive_expect_tx(&bb.recv_full[q], kRecvQBytes);
+      ptx::mbar_arrive_expect_tx(&bb.pm_full[q], kPMsgQBytes);
+      ptx::mbar_arrive_expect_tx(&bb.pm_full[4 + q], kPMsgQBytes);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, kTmemCols);
@@ -418,8 +449,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     if (issued_q >= 0) bounded_wait(bb.q_full, issued_q & 1, abort_flag, p, 0x5F2, false, false);
   } else if (warp == 1 && lane == 0) {
     // ===================================================== score MMA issuer
-    // Tile t into S buffer t & 1:  sr[128 x 64] = q_r . K_R^T, then the partial
-    // sc[128 x 64] = Q_c[:, dims_r] . C_KV[tile, dims_r]^T.
+    // Tile t: the partial sc[128 x 64] = Q_c[:, dims_r] . C_KV[tile, dims_r]^T
+    // into buffer t & 1 (signalled on its own, for the shippers), then
+    // sr[128 x 64] = q_r . K_R^T into the one sr buffer once the softmax has
+    // read the previous tile's.
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kHeads, kT, 0, 0);   // K-major A and B
     const uint64_t d_qc = ptx::smem_desc(ptx::smem_u32(smem + kOffQc), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_qr = ptx::smem_desc(ptx::smem_u32(smem + kOffQr), 16, 1024, ptx::kSwizzle128B);
@@ -439,21 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ok = bounded_wait(bb.q_full, seg & 1, abort_flag, p, 0x600, true, false);
         if (!ok) break;
       }
-      if (t >= 2) ok = bounded_wait(&bb.s_empty[buf], (uint32_t)((t >> 1) - 1) & 1, abort_flag, p, 0x601, true, false);
+      if (t >= 2) ok = bounded_wait(&bb.sc_empty[buf], (uint32_t)((t >> 1) - 1) & 1, abort_flag, p, 0x601, true, false);
       if (ok) ok = bounded_wait(&bb.kr_full[t % kNKr], (uint32_t)(t / kNKr) & 1, abort_flag, p, 0x602, true, false);
       if (ok) ok = bounded_wait(&bb.c_full[t % kNS], (uint32_t)(t / kNS) & 1, abort_flag, p, 0x603, true, false);
       if (!ok) break;
       ptx::tc_fence_after();
-      const uint32_t d_s = tmem + 128u * buf;
       {
-        const uint64_t b0 = d_kr + (uint64_t)(((t % kNKr) * kKrBytes) >> 4);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          ptx::mma_bf16_ss(d_s + 64, d_qr + (uint64_t)((32 * k) >> 4), b0 + (uint64_t)((32 * k) >> 4), kIdescS,
-                           k > 0);
-        ptx::mma_commit(&bb.kr_empty[t % kNKr]);
-      }
-      {
+        const uint32_t d_s = tmem + kColSc + 64u * buf;
         const uint64_t b0 = d_c + (uint64_t)(((t % kNS) * kStage) >> 4);
 #pragma unroll
         for (int a = 0; a < kAtoms; ++a)
@@ -462,6 +487,18 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
             ptx::mma_bf16_ss(d_s, d_qc + (uint64_t)((a * kQcAtom + 32 * k) >> 4),
                              b0 + (uint64_t)((a * kCAtom + 32 * k) >> 4), kIdescS, (a | k) != 0);
       }
+      ptx::mma_commit(&bb.sc_full[buf]);
+      if (t >= 1 && !(ok = bounded_wait(bb.sr_empty, (uint32_t)(t - 1) & 1, abort_flag, p, 0x604, true, false)))
+        break;
+      ptx::tc_fence_after();
+      {
+        const uint64_t b0 = d_kr + (uint64_t)(((t % kNKr) * kKrBytes) >> 4);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ptx::mma_bf16_ss(tmem + kColSr, d_qr + (uint64_t)((32 * k) >> 4), b0 + (uint64_t)((32 * k) >> 4),
+                           kIdescS, k > 0);
+        ptx::mma_commit(&bb.kr_empty[t % kNKr]);
+      }
       ptx::mma_commit(&bb.s_full[buf]);
       if (last_in_seg) ptx::mma_commit(bb.q_empty);
     }
@@ -469,54 +506,25 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     bounded_wait(&bb.drain[0], 0, abort_flag, p, 0x6F0, false, false);
   } else if (warp == 2 && lane == 0) {
     // ===================================================== O MMA issuer
-    // Tile j once P is complete (own rows, the peer's rows and factors): if a
-    // peer factor is not 1, the shippers rescale those heads' O rows first
-    // (rare).  Then O[128 x 256] += P[128 x 64] . C_KV[tile, dims_r] (B read
-    // MN-major from the tile's stage), four K steps of 16 tokens; a sequence
-    // part starts afresh.  Completion is signalled in both CTAs (the peer copies
-    // its next P rows only after this O is done).
+    // Tile j once P buffer j & 1 holds all 128 rows: O[128 x 256] += P[128 x 64]
+    // . C_KV[tile, dims_r], A read from TMEM, B MN-major from the tile's stage,
+    // four K steps of 16 tokens; a sequence part starts afresh.
     constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(kHeads, kDim, 0, 1);   // A K-major, B MN-major
-    const uint64_t d_p = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_cb = ptx::smem_desc(ptx::smem_u32(smem + kOffC), kCAtom, 1024, ptx::kSwizzle128B);
-    int n_resc = 0;
     int64_t oseq = seq0, otile = tile0;
     for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile)) {
-      if (!bounded_wait(bb.p_local, (uint32_t)j & 1, abort_flag, p, 0x700, true, false)) break;
-      if (!bounded_wait(bb.p_remote, (uint32_t)j & 1, abort_flag, p, 0x701, true, true)) break;
-      if (j + 1 < n_tiles) ptx::mbar_arrive_expect_tx(bb.p_remote, kRemoteBytes);
-      // the peer heads' factors: blocks 32 q + 16 peer .. + 15 of the alpha array
-      bool resc = false;
-      if (otile > 0 && j > 0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4* a4 = reinterpret_cast<const float4*>(alpha_s + 32 * q + 16 * peer);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 a = a4[v];
-            resc = resc || a.x != 1.f || a.y != 1.f || a.z != 1.f || a.w != 1.f;
-          }
-        }
-      }
-      // lanes_ready(j) is taken before the decision is posted: the shippers
-      // complete its next phase only after reading the decision, so the
-      // barrier can never run a whole phase ahead of this wait.
-      if (!bounded_wait(bb.lanes_ready, (uint32_t)j & 1, abort_flag, p, 0x702, true, false)) break;
-      dec_flag[j & 1] = resc ? 1 : 0;
-      ptx::mbar_arrive(&bb.dec[j & 1]);
-      if (resc) {
-        if (!bounded_wait(bb.resc_done, (uint32_t)n_resc & 1, abort_flag, p, 0x703, true, false)) break;
-        ++n_resc;
-      }
+      const int buf = (int)(j & 1);
+      if (!bounded_wait(&bb.p_tmem[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x700, true, false)) break;
       ptx::tc_fence_after();
       const uint32_t acc0 = (j > 0 && otile > 0) ? 1u : 0u;
       const int cs = (int)(j % kNS);
       const uint64_t b0 = d_cb + (uint64_t)((cs * kStage) >> 4);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        ptx::mma_bf16_ss(tmem + kColO, d_p + (uint64_t)((32 * k) >> 4), b0 + (uint64_t)((2048 * k) >> 4), kIdescO,
-                         k > 0 ? 1u : acc0);
+        ptx::mma_bf16_ts(tmem + kColO, tmem + kColP + 32u * buf + 8u * k, b0 + (uint64_t)((2048 * k) >> 4),
+                         kIdescO, k > 0 ? 1u : acc0);
       ptx::mma_commit(&bb.c_empty[cs]);
-      ptx::mma_commit_multicast(&bb.o_done[r], (uint16_t)0x3);
+      ptx::mma_commit(&bb.p_free[buf]);
     }
     ptx::mma_commit(&bb.drain[1]);
     bounded_wait(&bb.drain[1], 0, abort_flag, p, 0x7F0, false, false);
@@ -525,30 +533,26 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     // Thread (hi, k): head m = 32 q + 16 r + hi, tokens 32 k .. 32 k + 31 of a tile.
     const int q = warp & 3;
     const int hi = lane & 15, k = lane >> 4;
-    const int m = 32 * q + 16 * r + hi;          // TMEM lane, P row, alpha index
-    const int ol = 16 * q + hi;                  // row in the receive buffer
+    const int m = 32 * q + 16 * r + hi;          // TMEM lane
+    const int ol = 16 * q + hi;                  // row in the receive buffers (here and at the peer)
     const int h = h0 + m;
     const uint32_t lanes = (uint32_t)(32 * q + 16 * r) << 16;
-    const bool armer = q == 0;                   // arms recv_full for the next tile
-    const uint32_t peer_recv_free = ptx::mapa(ptx::smem_u32(bb.recv_free), peer);
-    const uint32_t peer_p_remote = ptx::mapa(ptx::smem_u32(bb.p_remote), peer);
-    uint8_t* my_rows = pbuf + (32 * q + 16 * r) * 128;
-    float* my_alpha = alpha_s + 32 * q + 16 * r;
-    const uint32_t peer_rows = ptx::mapa(ptx::smem_u32(my_rows), peer);
-    const uint32_t peer_alpha = ptx::mapa(ptx::smem_u32(my_alpha), peer);
-    bool copy_pending = false;
+    const uint32_t peer_recv_free = ptx::mapa(ptx::smem_u32(&bb.recv_free[q]), peer);
+    const uint32_t peer_pm = ptx::mapa(ptx::smem_u32(smem + kOffPMsg), peer);
+    const uint32_t peer_pm_full0 = ptx::mapa(ptx::smem_u32(&bb.pm_full[q]), peer);
+    const uint32_t peer_pm_full1 = ptx::mapa(ptx::smem_u32(&bb.pm_full[4 + q]), peer);
     float M = -INFINITY, Z = 0.f;
     int64_t cseq = seq0, ctile = tile0;
-    for (int64_t i = 0; i < n_tiles; ++i, step(cseq, ctile)) {
+    int64_t i = 0;
+    for (; i < n_tiles; ++i, step(cseq, ctile)) {
       const int64_t b = cseq, tile = ctile;
       const int buf = (int)(i & 1);
       if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x800, false)) break;
-      if (!warp_wait(bb.recv_full, (uint32_t)i & 1, abort_flag, p, 0x801, true)) break;
+      if (!warp_wait(&bb.recv_full[q], (uint32_t)i & 1, abort_flag, p, 0x801, true)) break;
       ptx::tc_fence_after();
-      // x: the partial sc, then sc;  sr;  s: the full score, then e_t or the weight
-      float x[kHalfT], sr[kHalfT], s[kHalfT];
-      ptx::tmem_ld16x2_32(tmem + lanes + 128u * buf, x);
-      ptx::tmem_ld16x2_32(tmem + lanes + 128u * buf + 64u, sr);
+      float x[kHalfT], sr[kHalfT];
+      ptx::tmem_ld16x2_32(tmem + lanes + kColSc + 64u * buf, x);
+      ptx::tmem_ld16x2_32(tmem + lanes + kColSr, sr);
       ptx::tmem_wait_ld();
       {  // the peer's partial scores over its dims (16-byte chunks swizzled by head)
         const float* rrow = recv + ol * kT;
@@ -562,108 +566,163 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        ptx::mbar_arrive(&bb.s_empty[buf]);
-        if (armer && i + 1 < n_tiles) ptx::mbar_arrive_expect_tx(bb.recv_full, kRecvBytes);
-        ptx::mbar_arrive_remote(peer_recv_free);   // the peer may send the next tile's partials
+        ptx::mbar_arrive(&bb.sc_empty[buf]);
+        ptx::mbar_arrive(bb.sr_empty);
+        // this quarter's buffer takes the next tile's partials: armed before the
+        // peer may send them
+        if (i + 1 < n_tiles) ptx::mbar_arrive_expect_tx(&bb.recv_full[q], kRecvQBytes);
+        ptx::mbar_arrive_remote(peer_recv_free);
       }
 
       const int64_t tok0 = tile * kT + kHalfT * k;
-      // Some of this thread's groups are condensed: the window starts at a
-      // multiple of g, which may fall inside the thread's 32 tokens, so the
-      // choice is made per group (grp[]).  For g = 64 a group is the whole
-      // tile, and the choice is the same for both threads of a head.
-      const bool half_groups = (g > 1) && (tok0 < win0);
-      bool grp[NGT];
-#pragma unroll
-      for (int gi = 0; gi < NGT; ++gi) grp[gi] = half_groups && (tok0 + gi * GW < win0);
       int32_t* anc = p.anchor + ((int64_t)b * p.H + h) * p.nG;
+      const bool first = i == 0 || tile == 0;
+      float alpha = 1.f;
+      uint32_t pk[kHalfT / 2];
 
-      // ---- step 2: condense; a grouped token's weight is e_t * f[group]
-      float f[NGT], Sg[NGT], deng[NGT], ent = -INFINITY;
-      if constexpr (g == 1) {
+      // Steps 2 and 3 for this thread's 32 tokens.  kFast: the whole tile is
+      // condensed (g > 1, tile before the window), so no per-token choice.
+      auto tile_math = [&](auto fast_tag) {
+        constexpr bool kFast = decltype(fast_tag)::value;
+        float s[kHalfT];
+        // Some of this thread's groups are condensed: the window starts at a
+        // multiple of g, which may fall inside the thread's 32 tokens, so the
+        // choice is made per group (grp[]).  For g = 64 a group is the whole
+        // tile, and the choice is the same for both threads of a head.
+        const bool half_groups = kFast || ((g > 1) && (tok0 < win0));
+        bool grp[NGT];
 #pragma unroll
-        for (int t = 0; t < kHalfT; ++t)
-          if (tok0 + t < win0 && LCA_CHECK(p.err, tok0 + t < p.nG, 0xE05))
-            anc[tok0 + t] = (int32_t)(p.pos0 + tok0 + t);
-      }
-      if (half_groups) {
-        int ag[NGT];
-        float srag[NGT], numg[NGT], mg[NGT];
+        for (int gi = 0; gi < NGT; ++gi) grp[gi] = kFast || (half_groups && (tok0 + gi * GW < win0));
+
+        float f[NGT], Sg[NGT], deng[NGT], own_den[NGT], ent = -INFINITY;
+        if constexpr (!kFast && g == 1) {
 #pragma unroll
-        for (int gi = 0; gi < NGT; ++gi) {
-          group_stats<GW>(x + gi * GW, sr + gi * GW, s + gi * GW, mg[gi], ag[gi], srag[gi], deng[gi],
-                          numg[gi]);
-          ag[gi] += gi * GW + kHalfT * k;          // tile-relative
-          f[gi] = 1.f;
+          for (int t = 0; t < kHalfT; ++t)
+            if (tok0 + t < win0 && LCA_CHECK(p.err, tok0 + t < p.nG, 0xE05))
+              anc[tok0 + t] = (int32_t)(p.pos0 + tok0 + t);
         }
-        if constexpr (g > kHalfT) {
-          // a 64-token group: merge the head's two threads (half 0 first, so
-          // both form the same bits; a tie keeps half 0's anchor)
-          const float om = __shfl_xor_sync(0xffffffffu, mg[0], 16);
-          const float od = __shfl_xor_sync(0xffffffffu, deng[0], 16);
-          const float on = __shfl_xor_sync(0xffffffffu, numg[0], 16);
-          const float os = __shfl_xor_sync(0xffffffffu, srag[0], 16);
-          const int oa = __shfl_xor_sync(0xffffffffu, ag[0], 16);
-          const float m0 = k == 0 ? mg[0] : om, m1 = k == 0 ? om : mg[0];
-          const float d0 = k == 0 ? deng[0] : od, d1 = k == 0 ? od : deng[0];
-          const float n0 = k == 0 ? numg[0] : on, n1 = k == 0 ? on : numg[0];
-          const float s0 = k == 0 ? srag[0] : os, s1 = k == 0 ? os : srag[0];
-          const int a0 = k == 0 ? ag[0] : oa, a1 = k == 0 ? oa : ag[0];
-          const float mm = fmaxf(m0, m1);
-          const float f0 = ex2((m0 - mm) * kLog2e), f1 = ex2((m1 - mm) * kLog2e);
-          deng[0] = d0 * f0 + d1 * f1;
-          numg[0] = n0 * f0 + n1 * f1;
-          const bool take1 = m1 > m0;
-          srag[0] = take1 ? s1 : s0;
-          ag[0] = take1 ? a1 : a0;
-          f[0] = k == 0 ? f0 : f1;                 // this thread's e_t are relative to its own max
-        }
-#pragma unroll
-        for (int gi = 0; gi < NGT; ++gi) {
-          Sg[gi] = __fdividef(numg[gi], deng[gi]) + srag[gi];
-          if (grp[gi]) ent = fmaxf(ent, Sg[gi]);
-        }
-        if (g <= kHalfT || k == 0) {
+        if (half_groups) {
+          int ag[NGT];
+          float srag[NGT], numg[NGT], mg[NGT];
 #pragma unroll
           for (int gi = 0; gi < NGT; ++gi) {
-            const int64_t jg = (tile * kT + (g <= kHalfT ? kHalfT * k + gi * GW : 0)) / g;
-            if (grp[gi] && LCA_CHECK(p.err, jg >= 0 && jg < p.nG && ag[gi] >= 0 && ag[gi] < kT, 0xE04))
-              anc[jg] = (int32_t)(p.pos0 + tile * kT + ag[gi]);
+            group_stats<GW>(x + gi * GW, sr + gi * GW, s + gi * GW, mg[gi], ag[gi], srag[gi], deng[gi],
+                            numg[gi]);
+            ag[gi] += gi * GW + kHalfT * k;          // tile-relative
+            own_den[gi] = deng[gi];
+            f[gi] = 1.f;
+          }
+          if constexpr (g > kHalfT) {
+            // a 64-token group: merge the head's two threads (half 0 first, so
+            // both form the same bits; a tie keeps half 0's anchor)
+            const float om = __shfl_xor_sync(0xffffffffu, mg[0], 16);
+            const float od = __shfl_xor_sync(0xffffffffu, deng[0], 16);
+            const float on = __shfl_xor_sync(0xffffffffu, numg[0], 16);
+            const float os = __shfl_xor_sync(0xffffffffu, srag[0], 16);
+            const int oa = __shfl_xor_sync(0xffffffffu, ag[0], 16);
+            const float m0 = k == 0 ? mg[0] : om, m1 = k == 0 ? om : mg[0];
+            const float d0 = k == 0 ? deng[0] : od, d1 = k == 0 ? od : deng[0];
+            const float n0 = k == 0 ? numg[0] : on, n1 = k == 0 ? on : numg[0];
+            const float s0 = k == 0 ? srag[0] : os, s1 = k == 0 ? os : srag[0];
+            const int a0 = k == 0 ? ag[0] : oa, a1 = k == 0 ? oa : ag[0];
+            const float mm = fmaxf(m0, m1);
+            const float f0 = ex2((m0 - mm) * kLog2e), f1 = ex2((m1 - mm) * kLog2e);
+            deng[0] = d0 * f0 + d1 * f1;
+            numg[0] = n0 * f0 + n1 * f1;
+            const bool take1 = m1 > m0;
+            srag[0] = take1 ? s1 : s0;
+            ag[0] = take1 ? a1 : a0;
+            f[0] = k == 0 ? f0 : f1;                 // this thread's e_t are relative to its own max
+          }
+#pragma unroll
+          for (int gi = 0; gi < NGT; ++gi) {
+            Sg[gi] = __fdividef(numg[gi], deng[gi]) + srag[gi];
+            if (grp[gi]) ent = fmaxf(ent, Sg[gi]);
+          }
+          if (g <= kHalfT || k == 0) {
+#pragma unroll
+            for (int gi = 0; gi < NGT; ++gi) {
+              const int64_t jg = (tile * kT + (g <= kHalfT ? kHalfT * k + gi * GW : 0)) / g;
+              if (grp[gi] && LCA_CHECK(p.err, jg >= 0 && jg < p.nG && ag[gi] >= 0 && ag[gi] < kT, 0xE04))
+                anc[jg] = (int32_t)(p.pos0 + tile * kT + ag[gi]);
+            }
+          }
+          if constexpr (!kFast) {
+#pragma unroll
+            for (int gi = 0; gi < NGT; ++gi) {
+              if (!grp[gi]) {   // a window group inside this half: its tokens stand for themselves
+#pragma unroll
+                for (int t = 0; t < GW; ++t) {
+                  s[gi * GW + t] = x[gi * GW + t] + sr[gi * GW + t];
+                  if (tok0 + gi * GW + t < p.L) ent = fmaxf(ent, s[gi * GW + t]);
+                }
+              }
+            }
+          }
+        } else {   // window tokens (and g = 1): the entry is the token itself
+#pragma unroll
+          for (int t = 0; t < kHalfT; ++t) {
+            s[t] = x[t] + sr[t] + (tok0 + t < p.bias_rows ? p.bias : 0.f);
+            if (tok0 + t < p.L) ent = fmaxf(ent, s[t]);
           }
         }
+
+        // ---- step 3: the head's reference max (both threads of the head agree)
+        const float tmax = fmaxf(ent, __shfl_xor_sync(0xffffffffu, ent, 16));
+        if (first) {
+          M = tmax;
+        } else if ((tmax - M) * kLog2e > kRescaleLog2) {
+          alpha = ex2((M - tmax) * kLog2e);
+          M = tmax;
+        }
+        Z *= alpha;
+
+        // ---- per-token weights (this thread's 32 bf16 of its head's P row); Z
+        // gains e^{S_j - M} per whole condensed group in this thread (the
+        // tokens' weights sum to it), its share for a split 64-token group,
+        // and each window token's weight
+        if (half_groups) {
 #pragma unroll
-        for (int gi = 0; gi < NGT; ++gi) {
-          if (!grp[gi]) {   // a window group inside this half: its tokens stand for themselves
-#pragma unroll
-            for (int t = 0; t < GW; ++t) {
-              s[gi * GW + t] = x[gi * GW + t] + sr[gi * GW + t];
-              if (tok0 + gi * GW + t < p.L) ent = fmaxf(ent, s[gi * GW + t]);
+          for (int gi = 0; gi < NGT; ++gi) {
+            if (grp[gi]) {
+              const float eS = ex2((Sg[gi] - M) * kLog2e);
+              if constexpr (g > kHalfT) {
+                f[gi] *= __fdividef(eS, deng[gi]);
+                Z += own_den[gi] * f[gi];
+              } else {
+                f[gi] = __fdividef(eS, deng[gi]);
+                Z += eS;
+              }
             }
           }
         }
-      } else {   // window tokens (and g = 1): the entry is the token itself
+        const float mb = -M * kLog2e;
 #pragma unroll
-        for (int t = 0; t < kHalfT; ++t) {
-          s[t] = x[t] + sr[t] + (tok0 + t < p.bias_rows ? p.bias : 0.f);
-          if (tok0 + t < p.L) ent = fmaxf(ent, s[t]);
+        for (int t2 = 0; t2 < kHalfT / 2; ++t2) {
+          float pv[2];
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int t = 2 * t2 + e2;
+            float v;
+            if (kFast || grp[t / GW]) {
+              v = s[t] * f[t / GW];
+            } else {
+              v = tok0 + t < p.L ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
+              Z += v;
+            }
+            pv[e2] = v;
+          }
+          pk[t2] = pack_bf16x2(pv[0], pv[1]);
         }
-      }
-
-      // ---- step 3: the head's reference max (both threads of the head agree)
+      };
+      const bool fast = g > 1 && (tile + 1) * kT <= win0;   // warp-uniform
+      if (fast) tile_math(std::true_type{});
+      else tile_math(std::false_type{});
       if (*abort_flag) break;
-      const float tmax = fmaxf(ent, __shfl_xor_sync(0xffffffffu, ent, 16));
-      const bool first = i == 0 || tile == 0;
-      float alpha = 1.f;
-      if (first) {
-        M = tmax;
-      } else if ((tmax - M) * kLog2e > kRescaleLog2) {
-        alpha = ex2((M - tmax) * kLog2e);
-        M = tmax;
-      }
+
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        // this head's O row must be complete before it is scaled here
-        Z *= alpha;
-        if (!warp_wait(&bb.o_done[r], (uint32_t)(i - 1) & 1, abort_flag, p, 0x803, false)) break;
+        // this head's O row must be complete (O of tile i - 1) before it is scaled here
+        if (!o_complete(i - 1, 0x803)) break;
         ptx::tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -677,71 +736,37 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         }
         ptx::tmem_wait_st();
       }
-      // the previous copy of this warp's rows and factors has read them
-      if (lane == 0 && copy_pending) {
-        ptx::bulk_wait_group_read0();
-        copy_pending = false;
-      }
-      __syncwarp();
-      if (k == 0) my_alpha[hi] = alpha;      // travels to the peer with P
-
-      // ---- per-token weights, this thread's 64 bytes of its head's P row
-      uint32_t pk[kHalfT / 2];
-      if (half_groups) {
-#pragma unroll
-        for (int gi = 0; gi < NGT; ++gi)
-          if (grp[gi]) f[gi] *= __fdividef(ex2((Sg[gi] - M) * kLog2e), deng[gi]);
-      }
-      const float mb = -M * kLog2e;
-#pragma unroll
-      for (int t2 = 0; t2 < kHalfT / 2; ++t2) {
-        float pv[2];
-#pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {
-          const int t = 2 * t2 + e2;
-          float v;
-          if (grp[t / GW]) v = s[t] * f[t / GW];
-          else v = tok0 + t < p.L ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
-          pv[e2] = v;
-        }
-        pk[t2] = pack_bf16x2(pv[0], pv[1]);
-        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pk[t2]);
-        Z += __low2float(v) + __high2float(v);   // Z from the rounded P
-      }
-      // the own P rows are free once O of the previous tile is done here
-      if (i >= 1 && !warp_wait(&bb.o_done[r], (uint32_t)(i - 1) & 1, abort_flag, p, 0x804, false)) break;
+      // ---- this head's P row and factor to the peer (its buffer `buf` is free
+      // once the peer's receivers read the message of tile i - 2)
+      if (i >= 2 && !warp_wait(&bb.pm_free[4 * buf + q], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x805, true))
+        break;
       {
-        uint8_t* prow = pbuf + m * 128;
+        // 16-byte stores into the peer's shared memory, each completing its
+        // bytes on the peer's barrier of this quarter and buffer
+        const uint32_t base = peer_pm + (uint32_t)(buf * kPMsgBytes);
+        const uint32_t bar = buf ? peer_pm_full1 : peer_pm_full0;
+        const uint32_t row = base + (uint32_t)(ol * kPRowBytes);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int phys = (4 * k + j) ^ (m & 7);
-          *reinterpret_cast<uint4*>(prow + 16 * phys) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
+        for (int j = 0; j < 4; ++j)
+          ptx::st_async_v4(row + 16u * (uint32_t)((4 * k + j) ^ (ol & 7)), pk[4 * j], pk[4 * j + 1],
+                           pk[4 * j + 2], pk[4 * j + 3], bar);
+        if (k == 0) ptx::st_async_b32(base + (uint32_t)(kPMsgAlpha + 4 * ol), __float_as_uint(alpha), bar);
       }
-      ptx::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        // the peer's P rows are free once O of the previous tile is done there
-        bool okp = true;
-        if (i >= 1) okp = bounded_wait(&bb.o_done[peer], (uint32_t)(i - 1) & 1, abort_flag, p, 0x805, true, true);
-        if (okp) {
-          ptx::bulk_copy_to_peer(peer_rows, my_rows, kPBlockBytes, peer_p_remote);
-          ptx::bulk_copy_to_peer(peer_alpha, my_alpha, kAlphaBlockBytes, peer_p_remote);
-          ptx::bulk_commit_group();
-          copy_pending = true;
-        }
-      }
+      // ---- this head's P row into TMEM (buffer `buf` is free once O of tile i - 2 is done)
+      if (i >= 2 && !warp_wait(&bb.p_free[buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x804, false)) break;
+      ptx::tc_fence_after();
+      ptx::tmem_st16x2_16(tmem + lanes + kColP + 32u * buf, pk);
+      ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bb.p_local);
+      if (lane == 0) ptx::mbar_arrive(&bb.p_tmem[buf]);
 
       if (last_of_part(i, tile)) {
         // the partial of the range's part of sequence b: this head's O row over
         // this CTA's dims, and (owner) its (M, Z)
         const int64_t slot = b + c;
         const bool slot_ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xE06);
-        if (!warp_wait(&bb.o_done[r], (uint32_t)i & 1, abort_flag, p, 0x806, false)) break;
+        if (!o_complete(i, 0x806)) break;
         ptx::tc_fence_after();
         float* dst = p.part_o + (slot * p.H + h) * (int64_t)kDC + kDim * r + 32 * k;
 #pragma unroll 1
@@ -764,32 +789,75 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         Z = 0.f;
       }
     }
-    if (lane == 0) {
-      if (copy_pending) ptx::bulk_wait_group_read0();
-      // the peer's last O-completion signal has landed here before this CTA exits
-      if (n_tiles > 0) bounded_wait(&bb.o_done[peer], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x8F0, true, true);
+    // The peer's releases of the last two P messages have landed here before
+    // this CTA exits.
+    if (lane == 0 && i == n_tiles) {
+      for (int64_t t = n_tiles - 2; t < n_tiles; ++t)
+        if (t >= 0 && !bounded_wait(&bb.pm_free[4 * (t & 1) + q], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x8F0,
+                                    true, true))
+          break;
     }
   } else if (warp >= 7) {
-    // ===================================================== shipper (peer heads of quarter q)
+    // ===================================================== shipper / receiver (peer heads of quarter q)
     // Thread (hi, k): peer head m = 32 q + 16 peer + hi, tokens 32 k .. of a tile.
-    // Per tile i: send the head's partial scores to the peer; then, one tile
-    // behind, do what O of tile i - 1 needs of these heads' O rows here: the
-    // rescale the O issuer asked for (rare), and at the end of a sequence part
-    // the write-out of the partial.
+    // Iteration i: send the partial scores of tile i + 1 to the peer, then take
+    // the peer's P rows of tile i: rescale these heads' O rows if the factor
+    // asks for it, write the rows into P buffer i & 1, and at the end of a
+    // sequence part write out these heads' O rows.
     const int q = warp & 3;
     const int hi = lane & 15, k = lane >> 4;
     const int m = 32 * q + 16 * peer + hi;
-    const int olp = 16 * q + hi;                 // the head's row in the peer's receive buffer
+    const int olp = 16 * q + hi;                 // the head's row in the receive buffers
     const uint32_t lanes = (uint32_t)(32 * q + 16 * peer) << 16;
     const uint32_t peer_row = ptx::mapa(ptx::smem_u32(recv + olp * kT), peer);
-    const uint32_t peer_recv_full = ptx::mapa(ptx::smem_u32(bb.recv_full), peer);
-    bool ok = true;
-    // what O of tile j needs done first (rescale), and the write-out at a part end
-    auto behind = [&](int64_t j, int64_t b, int64_t tile) -> bool {
-      if (!warp_wait(&bb.dec[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x902, false)) return false;
-      if (dec_flag[j & 1]) {
-        const float a = alpha_s[m];
-        if (!warp_wait(&bb.o_done[r], (uint32_t)(j - 1) & 1, abort_flag, p, 0x903, false)) return false;
+    const uint32_t peer_recv_full = ptx::mapa(ptx::smem_u32(&bb.recv_full[q]), peer);
+    const uint32_t peer_pm_free0 = ptx::mapa(ptx::smem_u32(&bb.pm_free[q]), peer);
+    const uint32_t peer_pm_free1 = ptx::mapa(ptx::smem_u32(&bb.pm_free[4 + q]), peer);
+    auto ship = [&](int64_t t) -> bool {
+      const int buf = (int)(t & 1);
+      if (!warp_wait(&bb.sc_full[buf], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x900, false)) return false;
+      ptx::tc_fence_after();
+      float v[32];
+      ptx::tmem_ld16x2_32(tmem + lanes + kColSc + 64u * buf, v);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bb.sc_empty[buf]);
+      if (t >= 1 && !warp_wait(&bb.recv_free[q], (uint32_t)(t - 1) & 1, abort_flag, p, 0x901, true)) return false;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        ptx::st_async_v4(peer_row + 16u * (uint32_t)((8 * k + j) ^ (olp & 15)), __float_as_uint(v[4 * j]),
+                         __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
+                         __float_as_uint(v[4 * j + 3]), peer_recv_full);
+      return true;
+    };
+    bool ok = n_tiles > 0 ? ship(0) : true;
+    int64_t bseq = seq0, btile = tile0;
+    int64_t i = 0;
+    for (; i < n_tiles && ok; ++i, step(bseq, btile)) {
+      if (i + 1 < n_tiles && !(ok = ship(i + 1))) break;
+      const int buf = (int)(i & 1);
+      if (!(ok = warp_wait(&bb.pm_full[4 * buf + q], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x902, true))) break;
+      uint32_t pk[kHalfT / 2];
+      const uint8_t* pm = smem + kOffPMsg + buf * kPMsgBytes;
+      {
+        const uint8_t* row = pm + olp * kPRowBytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * ((4 * k + j) ^ (olp & 7)));
+          pk[4 * j] = v.x; pk[4 * j + 1] = v.y; pk[4 * j + 2] = v.z; pk[4 * j + 3] = v.w;
+        }
+      }
+      const float a = *reinterpret_cast<const float*>(pm + kPMsgAlpha + 4 * olp);
+      __syncwarp();
+      // this quarter of buffer `buf` takes the message of tile i + 2 next: armed
+      // before the peer may send it
+      if (lane == 0) {
+        if (i + 2 < n_tiles) ptx::mbar_arrive_expect_tx(&bb.pm_full[4 * buf + q], kPMsgQBytes);
+        ptx::mbar_arrive_remote(buf ? peer_pm_free1 : peer_pm_free0);
+      }
+      if (__any_sync(0xffffffffu, a != 1.f)) {
+        if (!(ok = o_complete(i - 1, 0x903))) break;
         ptx::tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -802,14 +870,20 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           ptx::tmem_st16x2_32(ta, o);
         }
         ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bb.resc_done);
       }
-      if (last_of_part(j, tile)) {
-        const int64_t slot = b + c;
-        if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xE08)) return false;
-        if (!warp_wait(&bb.o_done[r], (uint32_t)j & 1, abort_flag, p, 0x904, false)) return false;
+      if (i >= 2 && !(ok = warp_wait(&bb.p_free[buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x904, false)))
+        break;
+      ptx::tc_fence_after();
+      ptx::tmem_st16x2_16(tmem + lanes + kColP + 32u * buf, pk);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bb.p_tmem[buf]);
+      if (last_of_part(i, btile)) {
+        const int64_t slot = bseq + c;
+        ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xE08);
+        if (!ok) break;
+        if (!(ok = o_complete(i, 0x905))) break;
         ptx::tc_fence_after();
         float* dst = p.part_o + (slot * p.H + h0 + m) * (int64_t)kDC + kDim * r + 32 * k;
 #pragma unroll 1
@@ -823,39 +897,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         }
         ptx::tc_fence_before();
       }
-      return true;
-    };
-    int64_t bseq = seq0, btile = tile0;          // (sequence, tile) of tile i - 1
-    int64_t i = 0;
-    for (; i < n_tiles && ok; ++i) {
-      const int buf = (int)(i & 1);
-      if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x900, false)) break;
-      ptx::tc_fence_after();
-      float v[32];
-      ptx::tmem_ld16x2_32(tmem + lanes + 128u * buf, v);
-      ptx::tmem_wait_ld();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&bb.s_empty[buf]);
-      if (i >= 1 && !warp_wait(bb.recv_free, (uint32_t)(i - 1) & 1, abort_flag, p, 0x901, true)) break;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        ptx::st_async_v4(peer_row + 16u * (uint32_t)((8 * k + j) ^ (olp & 15)), __float_as_uint(v[4 * j]),
-                         __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
-                         __float_as_uint(v[4 * j + 3]), peer_recv_full);
-      if (i >= 1) {
-        ok = behind(i - 1, bseq, btile);
-        step(bseq, btile);
-      }
-      __syncwarp();
-      if (ok && lane == 0) ptx::mbar_arrive(bb.lanes_ready);
     }
-    if (ok && i == n_tiles && n_tiles > 0) {
-      behind(n_tiles - 1, bseq, btile);
-      // the peer's release of the last tile has landed here before this CTA exits
-      if (lane == 0)
-        bounded_wait(bb.recv_free, (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true, true);
-    }
+    // the peer's release of the last partial scores has landed here before this CTA exits
+    if (ok && i == n_tiles && n_tiles > 0 && lane == 0)
+      bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true, true);
   }
 
   // ===================================================== teardown

@@ -403,6 +403,19 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, u
       : "memory");
 }
 
+// Plain (weak) 16- and 4-byte stores into another CTA's shared memory, at a
+// shared::cluster address from mapa.  Made visible to the owner by a later
+// mbarrier.arrive.release.cluster of the same thread on the owner's barrier.
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_b32(uint32_t cluster_addr, uint32_t a) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(a) : "memory");
+}
+
 // 4-byte store into another CTA's shared memory; completes 4 transaction bytes
 // on `cluster_bar` (an mbarrier of that same CTA).
 __device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t a, uint32_t cluster_bar) {

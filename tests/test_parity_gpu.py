@@ -138,6 +138,24 @@ def test_pair_ranges_spanning_sequences():
         compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
 
 
+def test_pair_short_ranges_repeatable():
+    """Ranges of one and two tiles with a partial last tile (L = 3000): each
+    range's partial is written out only after the O of both its tiles is
+    complete.  Repeated runs at several cluster counts must all match the
+    oracle (a missed wait shows up as rows that differ from run to run)."""
+    for L, w, seed in ((3000, 300, 44), (3000, 200, 21)):
+        wl = workloads.small("t", B=2, H=128, L=L, g=16, w=w, seed=seed)
+        x = workloads.generate(wl)
+        d = DeviceInputs(x)
+        ref = oracle_lca(x, wl.g, wl.w)
+        for n in (124, 126, 148, 40):
+            plan = make_plan(wl, {kvc.OPT_NUM_CTAS: n})
+            assert plan.kernel(wl.L, wl.g, wl.w) == "tcgen05_pair"
+            for _ in range(3):
+                out, anc = run_lca(plan, d, wl.g, wl.w)
+                compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+
+
 def test_ranges_spanning_sequences():
     """Few CTAs: every tile range crosses sequence boundaries (query reloads)."""
     wl = workloads.small("t", B=4, H=32, L=1000, g=16, w=50, seed=7)
