@@ -365,9 +365,9 @@ lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c
   const uint64_t qrows = (uint64_t)p->B * (uint64_t)p->H;
   if (!make_map(&pp.tm_c, c_kv, 512, rows, lca::pair::kT) ||
       !make_map(&pp.tm_k, k_r, 64, rows, lca::pair::kT) ||
-      !make_map(&pp.tm_qc, q_c, 512, qrows, lca::pair::kHeads) ||
-      !make_map(&pp.tm_qr, q_r, 64, qrows, lca::pair::kHeads))
+      !make_map(&pp.tm_qc, q_c, 512, qrows, lca::pair::kHeads))
     return LCA_ERR_CUDA;
+  pp.q_r = static_cast<const __nv_bfloat16*>(q_r);
   const int n_hb = p->H / lca::pair::kHeads;
   const int64_t tps = ceil_div(L, lca::pair::kT);
   const int64_t U = (int64_t)p->B * tps;

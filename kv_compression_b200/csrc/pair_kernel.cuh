@@ -11,11 +11,11 @@
 // (m / 16) % 2 == r, so every lane quarter -- every SM sub-partition -- holds
 // 16 own heads and 16 of the other CTA's ("peer") heads.
 //   scores     S_r[128 heads x 64 tokens] = Q_c[:, dims_r] . C_KV[tile, dims_r]^T
-//              (partial over its own dims) and sr = q_r . K_R^T, in TMEM.  Each
-//              CTA sends the partial scores of its peer heads to the other CTA
-//              (st.async into its shared memory, per lane quarter), so each
-//              head's full score sc_t = S_0 + S_1 is formed by the CTA that
-//              owns the head;
+//              (partial over its own dims) and sr = q_r . K_R^T, in TMEM (q_r
+//              itself sits in TMEM as the A operand).  Each CTA sends the
+//              partial scores of its peer heads to the other CTA (st.async into
+//              its shared memory, per lane quarter), so each head's full score
+//              sc_t = S_0 + S_1 is formed by the CTA that owns the head;
 //   condense   (step 2) two threads hold one head, 32 consecutive tokens each,
 //              so a group of g <= 32 tokens is reduced inside a thread: max,
 //              lowest-index argmax (the anchor a_j), e_t = e^{s_t - m_j},
@@ -26,12 +26,14 @@
 //              max M per head: a grouped token weighs e_t e^{S_j - M} / den_j,
 //              a window token e^{s_t - M}.  The bf16 weights P[128 heads x 64
 //              tokens] are the A operand of O[128 heads x 256 dims_r] +=
-//              P . C_KV[tile, dims_r], read from TMEM: the owner writes its
-//              heads' rows there and sends them to the peer (st.async from
-//              registers), whose receiving warps write them into its TMEM.  M
-//              rises only when an entry exceeds it by more than 2^8; the factor
-//              travels with P, and whichever warp writes a head's P row also
-//              rescales that head's O row first.
+//              P . C_KV[tile, dims_r], read from shared memory: the owner
+//              writes its heads' rows into its own P buffer and copies them
+//              (bulk shared-to-distributed-shared copies) into the peer's, so
+//              O of a tile starts as soon as both halves have landed.  M rises
+//              only when an entry exceeds it by more than 2^8; the owner
+//              rescales its O rows, and the factor travels with P so that the
+//              O MMA issuer of the other CTA has its receiving warps rescale
+//              that CTA's copy of the rows first (rare).
 // Each CTA writes its dims of every head's partial O, the owner CTA the
 // head's (M, Z); the combine kernel merges the ranges of a sequence.
 //
@@ -39,19 +41,21 @@
 // loads only its half); K_R is loaded by both CTAs.
 //
 // TMEM (512 columns): O at 0 (256), partial sc in two buffers at 256 and 320,
-// sr at 384 (one buffer: it is read at the start of a tile), P in two buffers
-// at 448 and 480 (bf16 pairs), so the scores of a tile, its weights and the O
-// accumulation of the tile before overlap.
+// sr at 384 (one buffer: it is read at the start of a tile), q_r of a sequence
+// in two buffers at 448 and 480 (bf16 pairs).
 //
 // Roles (352 threads): warp 0 lane 0 issues TMA loads; warp 1 allocates TMEM
-// and its lane 0 issues the score MMAs; warp 2 lane 0 issues the O MMAs; warps
-// 3-6 run the softmax of the own heads of lane quarter (warp % 4); warps 7-10
-// ship the partial scores of the peer heads of their quarter one tile ahead,
-// and write the peer heads' P rows (and rescale and write out their O rows).
-// Waits suspend in hardware (mbarrier.try_wait) and are bounded; when a
-// bound runs out the CTA records the error, stops issuing
-// work, waits for its own copies and MMAs in flight, frees TMEM and exits
-// after its peer.
+// and its lane 0 issues the score MMAs; warp 2 lane 0 issues the O MMAs and
+// decides, from the peer's factors, whether a tile needs the peer rows
+// rescaled; warps 3-6 run the softmax of the own heads of lane quarter
+// (warp % 4) and load each sequence's q_r into TMEM; warps 7-10 ship the
+// partial scores of the peer heads of their quarter a tile ahead and, one tile
+// behind, rescale (on request) and write out those heads' O rows.
+// Completion of O is only ever waited on barriers whose every phase the
+// waiter observes in order (a parity wait on a barrier two phases ahead would
+// pass early).  Waits suspend in hardware (mbarrier.try_wait) and are bounded;
+// when a bound runs out the CTA records the error, stops issuing work, waits
+// for its own copies and MMAs in flight, frees TMEM and exits after its peer.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -78,17 +82,14 @@ constexpr int kQcAtom = kHeads * 128;       // [128 heads][64 bf16] = 16 KB
 constexpr int kCAtom = kT * 128;            // [64 tokens][64 bf16] = 8 KB
 constexpr int kStage = kAtoms * kCAtom;     // 32 KB
 constexpr int kKrBytes = kT * 128;          // 8 KB
-constexpr int kQrBytes = kHeads * 128;      // q_r of all heads, 16 KB
+constexpr int kPBytes = kHeads * kT * 2;    // P[128 heads][64 tokens] bf16, K-major, 16 KB
 constexpr int kRecvBytes = kOwn * kT * 4;   // partial scores from the peer, 16 KB
-constexpr int kPRowBytes = kT * 2;          // one head's bf16 weights of a tile
-constexpr int kPMsgAlpha = kOwn * kPRowBytes;       // offset of the factors in a P message
-constexpr int kPMsgBytes = kPMsgAlpha + kOwn * 4;   // 64 rows of P + 64 factors = 8448 B
-// Each message travels per lane quarter: the 16 heads of quarter q come from
-// the peer's warp of the same quarter and complete their own barrier, so a
+// Messages travel per lane quarter: the 16 heads of quarter q come from the
+// peer's warp of the same quarter and complete their own barrier, so a
 // quarter waits only for its rows and each barrier takes a quarter of the
 // transaction updates.
-constexpr int kRecvQBytes = kRecvBytes / 4;                 // 16 heads x 64 tokens x 4 B
-constexpr int kPMsgQBytes = kPMsgBytes / 4;                 // 16 rows of P + 16 factors
+constexpr int kRecvQBytes = kRecvBytes / 4;               // 16 heads x 64 tokens x 4 B
+constexpr int kPQBytes = 16 * kT * 2 + 16 * 4;            // 16 rows of P + their 16 factors
 constexpr int kThreads = 32 * 11;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -96,26 +97,26 @@ constexpr float kRescaleLog2 = 8.f;
 
 // shared memory map (offsets from a 1024-byte aligned base; equal in both CTAs)
 constexpr int kOffQc = 0;
-constexpr int kOffQr = kOffQc + kAtoms * kQcAtom;
-constexpr int kOffC = kOffQr + kQrBytes;
+constexpr int kOffC = kOffQc + kAtoms * kQcAtom;
 constexpr int kOffKr = kOffC + kNS * kStage;
-constexpr int kOffRecv = kOffKr + kNKr * kKrBytes;
-constexpr int kOffPMsg = kOffRecv + kRecvBytes;            // [2] P messages from the peer
-constexpr int kOffBar = kOffPMsg + 2 * kPMsgBytes;
-constexpr int kNumBars = 2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 8 + 8 + 2 + 2 + 2;
+constexpr int kOffP = kOffKr + kNKr * kKrBytes;            // [2] P tiles
+constexpr int kOffRecv = kOffP + 2 * kPBytes;
+constexpr int kOffAlpha = kOffRecv + kRecvBytes;           // [2][128] float: the rescale factor per head
+constexpr int kOffFlag = kOffAlpha + 2 * kHeads * 4;       // int [2]: peer rows need a rescale
+constexpr int kOffBar = kOffFlag + 16;
+constexpr int kNumBars = 52;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget of one sm_100 CTA");
-static_assert(kOffC % 1024 == 0 && kOffKr % 1024 == 0 && kOffQr % 1024 == 0, "swizzle atoms");
-static_assert(kOffRecv % 16 == 0 && kOffPMsg % 16 == 0 && kPMsgBytes % 16 == 0 && kOffBar % 8 == 0,
-              "st.async targets and barriers");
+static_assert(kOffC % 1024 == 0 && kOffKr % 1024 == 0 && kOffP % 1024 == 0, "swizzle atoms");
+static_assert(kOffRecv % 16 == 0 && kOffAlpha % 16 == 0 && kOffBar % 8 == 0, "st.async targets and barriers");
 
 // TMEM columns
 constexpr uint32_t kColO = 0;       // O [128 heads x 256 dims] fp32
 constexpr uint32_t kColSc = 256;    // partial sc, buffer b at 256 + 64 b
 constexpr uint32_t kColSr = 384;    // sr
-constexpr uint32_t kColP = 448;     // P, buffer b at 448 + 32 b (64 bf16 = 32 columns a row)
+constexpr uint32_t kColQr = 448;    // q_r, buffer b at 448 + 32 b (64 bf16 = 32 columns a row)
 
 constexpr int kErrTimeout = 1;
 
@@ -123,7 +124,7 @@ struct PairParams {
   CUtensorMap tm_c;    // c_kv as [B*L rows][512], box [64 rows][64], 128B swizzle
   CUtensorMap tm_k;    // k_r  as [B*L rows][64],  box [64 rows][64], 128B swizzle
   CUtensorMap tm_qc;   // q_c  as [B*H rows][512], box [128 rows][64], 128B swizzle
-  CUtensorMap tm_qr;   // q_r  as [B*H rows][64],  box [128 rows][64], 128B swizzle
+  const __nv_bfloat16* q_r;   // [B][H][64]
   int B, H;
   int64_t L;
   int64_t nG;          // condensed groups in these rows (0: dense attention)
@@ -150,18 +151,24 @@ struct Bars {
   uint64_t* c_empty;     // [kNS] released after O of that tile
   uint64_t* kr_full;     // [kNKr]
   uint64_t* kr_empty;    // [kNKr] released after the sr MMAs
-  uint64_t* q_full;
-  uint64_t* q_empty;
+  uint64_t* q_full;      // Q_c of a sequence landed
+  uint64_t* q_empty;     // the last score MMA of a sequence is done
+  uint64_t* qr_full;     // [2] q_r of sequence segment s is in TMEM buffer s & 1
+  uint64_t* qr_empty;    // [2] the last sr MMA that read buffer s & 1 is done
   uint64_t* s_full;      // [2] the scores (partial sc in buffer b, then sr) of a tile are in TMEM
   uint64_t* sc_full;     // [2] the partial sc of a tile is in buffer b
   uint64_t* sc_empty;    // [2] softmax and shipper warps have read partial sc buffer b
   uint64_t* sr_empty;    // the softmax warps have read sr
   uint64_t* recv_full;   // [4] quarter q of the peer's partial scores landed (transaction bytes)
   uint64_t* recv_free;   // [4] the peer's quarter q has read the partial scores sent to it
-  uint64_t* pm_full;     // [2 x 4] quarter q of the peer's P message b landed (transaction bytes)
-  uint64_t* pm_free;     // [2 x 4] the peer's quarter q has read this CTA's P message b
-  uint64_t* p_tmem;      // [2] P buffer b holds the tile's 128 rows (and O rows are rescaled)
-  uint64_t* p_free;      // [2] O of the tile that used P buffer b is done (and every O before it)
+  uint64_t* p_local;     // the own rows of P buffer i & 1 are written
+  uint64_t* p_remote;    // [2 x 4] quarter q of the peer's rows of P buffer b landed (transaction bytes)
+  uint64_t* p_free;      // [2 x 2] index 2 c + b: O of CTA c done with P buffer b (and every O before)
+  uint64_t* lanes_ready; // the shippers finished what precedes O of a tile (the tile before's rows)
+  uint64_t* dec;         // [2] the O issuer's decision for a tile (flag: rescale the peer rows)
+  uint64_t* resc_go;     // every O issued before a rescale request is done
+  uint64_t* resc_done;   // the shippers rescaled the peer rows as asked
+  uint64_t* part_done;   // the last O of a sequence part is done (one phase per part)
   uint64_t* drain;       // [2]
 };
 
@@ -172,10 +179,8 @@ __device__ __forceinline__ void record_timeout(volatile int* abort, const PairPa
 
 // Bounded wait.  Each probe is an mbarrier.try_wait, which suspends the
 // thread in hardware until the phase completes or a short system-defined
-// limit passes (a suspend-time hint would let it sleep past the completion:
-// measured, that added up to a microsecond to every hand-off).  `cluster`:
-// acquire at cluster scope (barriers that the peer CTA arrives on or
-// completes transactions on).
+// limit passes.  `cluster`: acquire at cluster scope (barriers that the peer
+// CTA arrives on or completes transactions on).
 __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const PairParams& p, int where, bool honour_abort,
                                           bool cluster) {
@@ -285,20 +290,31 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.kr_empty = bb.kr_full + kNKr;
   bb.q_full = bb.kr_empty + kNKr;
   bb.q_empty = bb.q_full + 1;
-  bb.s_full = bb.q_empty + 1;
+  bb.qr_full = bb.q_empty + 1;
+  bb.qr_empty = bb.qr_full + 2;
+  bb.s_full = bb.qr_empty + 2;
   bb.sc_full = bb.s_full + 2;
   bb.sc_empty = bb.sc_full + 2;
   bb.sr_empty = bb.sc_empty + 2;
   bb.recv_full = bb.sr_empty + 1;
   bb.recv_free = bb.recv_full + 4;
-  bb.pm_full = bb.recv_free + 4;
-  bb.pm_free = bb.pm_full + 8;
-  bb.p_tmem = bb.pm_free + 8;
-  bb.p_free = bb.p_tmem + 2;
-  bb.drain = bb.p_free + 2;
+  bb.p_local = bb.recv_free + 4;
+  bb.p_remote = bb.p_local + 1;
+  bb.p_free = bb.p_remote + 8;
+  bb.lanes_ready = bb.p_free + 4;
+  bb.dec = bb.lanes_ready + 1;
+  bb.resc_go = bb.dec + 2;
+  bb.resc_done = bb.resc_go + 1;
+  bb.part_done = bb.resc_done + 1;
+  bb.drain = bb.part_done + 1;
+  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 1 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 ==
+                    kNumBars,
+                "barrier count");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  volatile int* dec_flag = reinterpret_cast<volatile int*>(smem + kOffFlag);
   float* recv = reinterpret_cast<float*>(smem + kOffRecv);
+  float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);   // [2][128]
 
   const int64_t cl = blockIdx.x >> 1;
   const int hb = (int)(cl % p.n_hb);
@@ -316,15 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   auto last_of_part = [&](int64_t i, int64_t tile) {
     return i + 1 == n_tiles || tile + 1 == p.tiles_per_seq;
   };
-  // O of tile j (and every O before it: one thread issues them in order) is
-  // done.  Waited on the P buffer's release, whose previous phase (tile j - 2)
-  // every caller has already seen when it wrote P of tile j or j + 1: a
-  // parity wait is only sound when the barrier cannot be two phases behind.
-  auto o_complete = [&](int64_t j, int where) -> bool {
-    const bool ok = warp_wait(&bb.p_free[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, where, false);
-    if (ok) ptx::tc_fence_after();
-    return ok;
-  };
 
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) { ptx::mbar_init(&bb.c_full[i], 1); ptx::mbar_init(&bb.c_empty[i], 1); }
@@ -332,29 +339,34 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     ptx::mbar_init(bb.q_full, 1);
     ptx::mbar_init(bb.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bb.qr_full[i], 4);          // the 4 softmax warps
+      ptx::mbar_init(&bb.qr_empty[i], 1);
       ptx::mbar_init(&bb.s_full[i], 1);
       ptx::mbar_init(&bb.sc_full[i], 1);
       ptx::mbar_init(&bb.sc_empty[i], 8);         // 4 softmax + 4 shipper warps
-      ptx::mbar_init(&bb.p_tmem[i], 8);           // 4 softmax + 4 shipper warps
-      ptx::mbar_init(&bb.p_free[i], 1);
+      ptx::mbar_init(&bb.dec[i], 1);
       ptx::mbar_init(&bb.drain[i], 1);
     }
+    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bb.p_free[i], 1);   // one O commit (multicast)
     ptx::mbar_init(bb.sr_empty, 4);               // the 4 softmax warps
     for (int q = 0; q < 4; ++q) {
       ptx::mbar_init(&bb.recv_full[q], 1);        // armed with its transaction bytes
       ptx::mbar_init(&bb.recv_free[q], 1);        // the peer's softmax warp of quarter q
-      for (int b = 0; b < 2; ++b) {
-        ptx::mbar_init(&bb.pm_full[4 * b + q], 1);  // armed with its transaction bytes
-        ptx::mbar_init(&bb.pm_free[4 * b + q], 1);  // the peer's receiver warp of quarter q
-      }
+      ptx::mbar_init(&bb.p_remote[q], 1);         // armed with its transaction bytes
+      ptx::mbar_init(&bb.p_remote[4 + q], 1);
     }
+    ptx::mbar_init(bb.p_local, 4);                // the 4 softmax warps
+    ptx::mbar_init(bb.lanes_ready, 4);            // the 4 shipper warps
+    ptx::mbar_init(bb.resc_go, 1);
+    ptx::mbar_init(bb.resc_done, 4);
+    ptx::mbar_init(bb.part_done, 1);
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
     // the first phases of the barriers the peer completes with transaction bytes
     for (int q = 0; q < 4; ++q) {
       ptx::mbar_arrive_expect_tx(&bb.recv_full[q], kRecvQBytes);
-      ptx::mbar_arrive_expect_tx(&bb.pm_full[q], kPMsgQBytes);
-      ptx::mbar_arrive_expect_tx(&bb.pm_full[4 + q], kPMsgQBytes);
+      ptx::mbar_arrive_expect_tx(&bb.p_remote[q], kPQBytes);
+      ptx::mbar_arrive_expect_tx(&bb.p_remote[4 + q], kPQBytes);
     }
   }
   if (warp == 1) {
@@ -387,7 +399,6 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     ptx::prefetch_tmap(&p.tm_c);
     ptx::prefetch_tmap(&p.tm_k);
     ptx::prefetch_tmap(&p.tm_qc);
-    ptx::prefetch_tmap(&p.tm_qr);
     const uint64_t once = ptx::l2_policy_evict_first();
     int issued_c[kNS], issued_k[kNKr];
 #pragma unroll
@@ -405,11 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ++seg;
         if (seg >= 1) ok = bounded_wait(bb.q_empty, (seg - 1) & 1, abort_flag, p, 0x500, true, false);
         if (!ok) break;
-        ptx::mbar_arrive_expect_tx(bb.q_full, kAtoms * kQcAtom + kQrBytes);
+        ptx::mbar_arrive_expect_tx(bb.q_full, kAtoms * kQcAtom);
         const int32_t qrow = (int32_t)(b * p.H + h0);
         for (int a = 0; a < kAtoms; ++a)
           ptx::tma_load_2d(smem + kOffQc + a * kQcAtom, &p.tm_qc, kDim * r + 64 * a, qrow, bb.q_full);
-        ptx::tma_load_2d(smem + kOffQr, &p.tm_qr, 0, qrow, bb.q_full);
         issued_q = seg;
       }
       const int32_t row = (int32_t)(b * p.L + ptile * kT);
@@ -451,11 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     // ===================================================== score MMA issuer
     // Tile t: the partial sc[128 x 64] = Q_c[:, dims_r] . C_KV[tile, dims_r]^T
     // into buffer t & 1 (signalled on its own, for the shippers), then
-    // sr[128 x 64] = q_r . K_R^T into the one sr buffer once the softmax has
-    // read the previous tile's.
+    // sr[128 x 64] = q_r . K_R^T (A from TMEM) into the one sr buffer once the
+    // softmax has read the previous tile's.
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kHeads, kT, 0, 0);   // K-major A and B
     const uint64_t d_qc = ptx::smem_desc(ptx::smem_u32(smem + kOffQc), 16, 1024, ptx::kSwizzle128B);
-    const uint64_t d_qr = ptx::smem_desc(ptx::smem_u32(smem + kOffQr), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_c = ptx::smem_desc(ptx::smem_u32(smem + kOffC), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_kr = ptx::smem_desc(ptx::smem_u32(smem + kOffKr), 16, 1024, ptx::kSwizzle128B);
     int seg = -1;
@@ -466,9 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       const int64_t b = sseq;
       const bool last_in_seg = last_of_part(t, stile);
       const int buf = (int)(t & 1);
+      bool new_seg = false;
       if (b != cur_b) {
         cur_b = b;
         ++seg;
+        new_seg = true;
         ok = bounded_wait(bb.q_full, seg & 1, abort_flag, p, 0x600, true, false);
         if (!ok) break;
       }
@@ -488,43 +499,84 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
                              b0 + (uint64_t)((a * kCAtom + 32 * k) >> 4), kIdescS, (a | k) != 0);
       }
       ptx::mma_commit(&bb.sc_full[buf]);
-      if (t >= 1 && !(ok = bounded_wait(bb.sr_empty, (uint32_t)(t - 1) & 1, abort_flag, p, 0x604, true, false)))
-        break;
+      if (t >= 1) ok = bounded_wait(bb.sr_empty, (uint32_t)(t - 1) & 1, abort_flag, p, 0x604, true, false);
+      if (ok && new_seg) ok = bounded_wait(&bb.qr_full[seg & 1], (uint32_t)(seg >> 1) & 1, abort_flag, p, 0x605, true, false);
+      if (!ok) break;
       ptx::tc_fence_after();
       {
+        const uint32_t a_qr = tmem + kColQr + 32u * (uint32_t)(seg & 1);
         const uint64_t b0 = d_kr + (uint64_t)(((t % kNKr) * kKrBytes) >> 4);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          ptx::mma_bf16_ss(tmem + kColSr, d_qr + (uint64_t)((32 * k) >> 4), b0 + (uint64_t)((32 * k) >> 4),
-                           kIdescS, k > 0);
+          ptx::mma_bf16_ts(tmem + kColSr, a_qr + 8u * k, b0 + (uint64_t)((32 * k) >> 4), kIdescS, k > 0);
         ptx::mma_commit(&bb.kr_empty[t % kNKr]);
       }
       ptx::mma_commit(&bb.s_full[buf]);
-      if (last_in_seg) ptx::mma_commit(bb.q_empty);
+      if (last_in_seg) {
+        ptx::mma_commit(bb.q_empty);
+        ptx::mma_commit(&bb.qr_empty[seg & 1]);
+      }
     }
     ptx::mma_commit(&bb.drain[0]);
     bounded_wait(&bb.drain[0], 0, abort_flag, p, 0x6F0, false, false);
   } else if (warp == 2 && lane == 0) {
     // ===================================================== O MMA issuer
-    // Tile j once P buffer j & 1 holds all 128 rows: O[128 x 256] += P[128 x 64]
-    // . C_KV[tile, dims_r], A read from TMEM, B MN-major from the tile's stage,
-    // four K steps of 16 tokens; a sequence part starts afresh.
+    // Tile j once P buffer j & 1 is complete (own rows, the peer's rows and
+    // factors) and the shippers are done with the tile before: if a peer
+    // factor is not 1, the shippers rescale those heads' O rows first (rare).
+    // Then O[128 x 256] += P[128 x 64] . C_KV[tile, dims_r] (A K-major from
+    // the P buffer, B MN-major from the tile's stage), four K steps of 16
+    // tokens; a sequence part starts afresh.  The release of the P buffer is
+    // signalled in both CTAs (each writes into the other's).
     constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(kHeads, kDim, 0, 1);   // A K-major, B MN-major
+    const uint64_t d_p = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_cb = ptx::smem_desc(ptx::smem_u32(smem + kOffC), kCAtom, 1024, ptx::kSwizzle128B);
+    int n_resc = 0;
     int64_t oseq = seq0, otile = tile0;
     for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile)) {
       const int buf = (int)(j & 1);
-      if (!bounded_wait(&bb.p_tmem[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x700, true, false)) break;
+      if (!bounded_wait(bb.p_local, (uint32_t)j & 1, abort_flag, p, 0x700, true, false)) break;
+      bool ok = true;
+      for (int q = 0; q < 4 && ok; ++q)
+        ok = bounded_wait(&bb.p_remote[4 * buf + q], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x701, true, true);
+      if (!ok) break;
+      // this buffer takes the peer's rows of tile j + 2 next; the peer writes
+      // them only after this CTA's O of tile j is done
+      if (j + 2 < n_tiles)
+        for (int q = 0; q < 4; ++q) ptx::mbar_arrive_expect_tx(&bb.p_remote[4 * buf + q], kPQBytes);
+      if (!bounded_wait(bb.lanes_ready, (uint32_t)j & 1, abort_flag, p, 0x702, true, false)) break;
+      bool resc = false;
+      if (j > 0 && otile > 0) {
+        const float* al = alpha_s + kHeads * buf;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4* a4 = reinterpret_cast<const float4*>(al + 32 * q + 16 * peer);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 a = a4[v];
+            resc = resc || a.x != 1.f || a.y != 1.f || a.z != 1.f || a.w != 1.f;
+          }
+        }
+      }
+      if (resc) ptx::mma_commit(bb.resc_go);       // lands once every O issued so far is done
+      dec_flag[j & 1] = resc ? 1 : 0;
+      ptx::mbar_arrive(&bb.dec[j & 1]);
+      if (resc) {
+        if (!bounded_wait(bb.resc_done, (uint32_t)n_resc & 1, abort_flag, p, 0x703, true, false)) break;
+        ++n_resc;
+      }
       ptx::tc_fence_after();
       const uint32_t acc0 = (j > 0 && otile > 0) ? 1u : 0u;
       const int cs = (int)(j % kNS);
+      const uint64_t a0 = d_p + (uint64_t)((buf * kPBytes) >> 4);
       const uint64_t b0 = d_cb + (uint64_t)((cs * kStage) >> 4);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        ptx::mma_bf16_ts(tmem + kColO, tmem + kColP + 32u * buf + 8u * k, b0 + (uint64_t)((2048 * k) >> 4),
-                         kIdescO, k > 0 ? 1u : acc0);
+        ptx::mma_bf16_ss(tmem + kColO, a0 + (uint64_t)((32 * k) >> 4), b0 + (uint64_t)((2048 * k) >> 4), kIdescO,
+                         k > 0 ? 1u : acc0);
       ptx::mma_commit(&bb.c_empty[cs]);
-      ptx::mma_commit(&bb.p_free[buf]);
+      ptx::mma_commit_multicast(&bb.p_free[2 * r + buf], (uint16_t)0x3);
+      if (last_of_part(j, otile)) ptx::mma_commit(bb.part_done);
     }
     ptx::mma_commit(&bb.drain[1]);
     bounded_wait(&bb.drain[1], 0, abort_flag, p, 0x7F0, false, false);
@@ -533,18 +585,46 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     // Thread (hi, k): head m = 32 q + 16 r + hi, tokens 32 k .. 32 k + 31 of a tile.
     const int q = warp & 3;
     const int hi = lane & 15, k = lane >> 4;
-    const int m = 32 * q + 16 * r + hi;          // TMEM lane
-    const int ol = 16 * q + hi;                  // row in the receive buffers (here and at the peer)
+    const int m = 32 * q + 16 * r + hi;          // TMEM lane, P row, factor index
+    const int mp = 32 * q + 16 * peer + hi;      // the peer head of the same lane slot
+    const int ol = 16 * q + hi;                  // row in the receive buffer
     const int h = h0 + m;
     const uint32_t lanes = (uint32_t)(32 * q + 16 * r) << 16;
+    const uint32_t lanes_peer = (uint32_t)(32 * q + 16 * peer) << 16;
     const uint32_t peer_recv_free = ptx::mapa(ptx::smem_u32(&bb.recv_free[q]), peer);
-    const uint32_t peer_pm = ptx::mapa(ptx::smem_u32(smem + kOffPMsg), peer);
-    const uint32_t peer_pm_full0 = ptx::mapa(ptx::smem_u32(&bb.pm_full[q]), peer);
-    const uint32_t peer_pm_full1 = ptx::mapa(ptx::smem_u32(&bb.pm_full[4 + q]), peer);
+    const uint32_t peer_p_remote0 = ptx::mapa(ptx::smem_u32(&bb.p_remote[q]), peer);
+    const uint32_t peer_p_remote1 = ptx::mapa(ptx::smem_u32(&bb.p_remote[4 + q]), peer);
+    const int row0 = 32 * q + 16 * r;            // this warp's 16 P rows (2 KB) and factors
+    bool copy_pending = false;
+    // q_r of sequence `seq` (segment s) into TMEM buffer s & 1, both lane
+    // halves of this quarter: this thread's 32 dims of its own and its peer head
+    auto load_qr = [&](int64_t seq, int s) -> bool {
+      if (s >= 2 && !warp_wait(&bb.qr_empty[s & 1], (uint32_t)((s >> 1) - 1) & 1, abort_flag, p, 0x807, false))
+        return false;
+      uint32_t own[16], oth[16];
+      const uint4* src_own = reinterpret_cast<const uint4*>(p.q_r + ((int64_t)seq * p.H + h0 + m) * kDR + 32 * k);
+      const uint4* src_oth = reinterpret_cast<const uint4*>(p.q_r + ((int64_t)seq * p.H + h0 + mp) * kDR + 32 * k);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 a = __ldg(src_own + v), b2 = __ldg(src_oth + v);
+        own[4 * v] = a.x; own[4 * v + 1] = a.y; own[4 * v + 2] = a.z; own[4 * v + 3] = a.w;
+        oth[4 * v] = b2.x; oth[4 * v + 1] = b2.y; oth[4 * v + 2] = b2.z; oth[4 * v + 3] = b2.w;
+      }
+      ptx::tc_fence_after();
+      ptx::tmem_st16x2_16(tmem + lanes + kColQr + 32u * (uint32_t)(s & 1), own);
+      ptx::tmem_st16x2_16(tmem + lanes_peer + kColQr + 32u * (uint32_t)(s & 1), oth);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bb.qr_full[s & 1]);
+      return true;
+    };
     float M = -INFINITY, Z = 0.f;
     int64_t cseq = seq0, ctile = tile0;
+    int seg = 0;
     int64_t i = 0;
-    for (; i < n_tiles; ++i, step(cseq, ctile)) {
+    bool ok = n_tiles > 0 ? load_qr(seq0, 0) : true;
+    for (; i < n_tiles && ok; ++i, step(cseq, ctile)) {
       const int64_t b = cseq, tile = ctile;
       const int buf = (int)(i & 1);
       if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x800, false)) break;
@@ -572,6 +652,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         // peer may send them
         if (i + 1 < n_tiles) ptx::mbar_arrive_expect_tx(&bb.recv_full[q], kRecvQBytes);
         ptx::mbar_arrive_remote(peer_recv_free);
+      }
+      // the next sequence's q_r, for the sr MMA of the tile after this one
+      if (last_of_part(i, tile) && i + 1 < n_tiles) {
+        ++seg;
+        if (!load_qr(b + 1, seg)) break;
       }
 
       const int64_t tok0 = tile * kT + kHalfT * k;
@@ -721,8 +806,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       if (*abort_flag) break;
 
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        // this head's O row must be complete (O of tile i - 1) before it is scaled here
-        if (!o_complete(i - 1, 0x803)) break;
+        // this head's O row must be complete (O of tile i - 1) before it is
+        // scaled here; this warp saw buffer (i - 1) & 1's earlier release when
+        // it wrote P of tile i - 1
+        const int pb = (int)((i - 1) & 1);
+        if (!warp_wait(&bb.p_free[2 * r + pb], (uint32_t)((i - 1) >> 1) & 1, abort_flag, p, 0x803, true)) break;
         ptx::tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -735,38 +823,49 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           ptx::tmem_st16x2_32(ta, o);
         }
         ptx::tmem_wait_st();
+        ptx::tc_fence_before();
       }
-      // ---- this head's P row and factor to the peer (its buffer `buf` is free
-      // once the peer's receivers read the message of tile i - 2)
-      if (i >= 2 && !warp_wait(&bb.pm_free[4 * buf + q], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x805, true))
+      // ---- this head's P row and factor into this CTA's P buffer (free once
+      // its O of tile i - 2 is done; the previous copy out of it has read it)
+      if (i >= 2 && !warp_wait(&bb.p_free[2 * r + buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x804, true))
         break;
+      if (lane == 0 && copy_pending) {
+        ptx::bulk_wait_group_read0();
+        copy_pending = false;
+      }
+      __syncwarp();
       {
-        // 16-byte stores into the peer's shared memory, each completing its
-        // bytes on the peer's barrier of this quarter and buffer
-        const uint32_t base = peer_pm + (uint32_t)(buf * kPMsgBytes);
-        const uint32_t bar = buf ? peer_pm_full1 : peer_pm_full0;
-        const uint32_t row = base + (uint32_t)(ol * kPRowBytes);
+        uint8_t* row = smem + kOffP + buf * kPBytes + m * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          ptx::st_async_v4(row + 16u * (uint32_t)((4 * k + j) ^ (ol & 7)), pk[4 * j], pk[4 * j + 1],
-                           pk[4 * j + 2], pk[4 * j + 3], bar);
-        if (k == 0) ptx::st_async_b32(base + (uint32_t)(kPMsgAlpha + 4 * ol), __float_as_uint(alpha), bar);
+          *reinterpret_cast<uint4*>(row + 16 * ((4 * k + j) ^ (m & 7))) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        if (k == 0) alpha_s[kHeads * buf + m] = alpha;
       }
-      // ---- this head's P row into TMEM (buffer `buf` is free once O of tile i - 2 is done)
-      if (i >= 2 && !warp_wait(&bb.p_free[buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x804, false)) break;
-      ptx::tc_fence_after();
-      ptx::tmem_st16x2_16(tmem + lanes + kColP + 32u * buf, pk);
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();                 // visible to the MMA's and the copy's reads
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&bb.p_tmem[buf]);
+      // ---- the same 16 rows and factors into the peer's P buffer (free once
+      // the peer's O of tile i - 2 is done): two bulk copies, same offsets
+      if (i >= 2 && !warp_wait(&bb.p_free[2 * peer + buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x805, true))
+        break;
+      if (lane == 0) {
+        const uint32_t bar = buf ? peer_p_remote1 : peer_p_remote0;
+        const uint8_t* rows = smem + kOffP + buf * kPBytes + row0 * 128;
+        const float* fac = alpha_s + kHeads * buf + row0;
+        ptx::bulk_copy_to_peer(ptx::mapa(ptx::smem_u32(rows), peer), rows, 16 * 128, bar);
+        ptx::bulk_copy_to_peer(ptx::mapa(ptx::smem_u32(fac), peer), fac, 16 * 4, bar);
+        ptx::bulk_commit_group();
+        copy_pending = true;
+        ptx::mbar_arrive(bb.p_local);
+      }
 
       if (last_of_part(i, tile)) {
         // the partial of the range's part of sequence b: this head's O row over
-        // this CTA's dims, and (owner) its (M, Z)
+        // this CTA's dims, and (owner) its (M, Z).  O of tile i is done when
+        // buffer i & 1 is released (this warp saw its previous release above).
         const int64_t slot = b + c;
         const bool slot_ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xE06);
-        if (!o_complete(i, 0x806)) break;
+        if (!warp_wait(&bb.p_free[2 * r + buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x806, true)) break;
         ptx::tc_fence_after();
         float* dst = p.part_o + (slot * p.H + h) * (int64_t)kDC + kDim * r + 32 * k;
 #pragma unroll 1
@@ -789,30 +888,29 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         Z = 0.f;
       }
     }
-    // The peer's releases of the last two P messages have landed here before
-    // this CTA exits.
-    if (lane == 0 && i == n_tiles) {
+    if (lane == 0 && copy_pending) ptx::bulk_wait_group_read0();
+    // The peer O issuer's releases of the last two P buffers (multicast into
+    // this CTA's shared memory) have landed before this CTA exits.
+    if (lane == 0 && q == 0 && i == n_tiles) {
       for (int64_t t = n_tiles - 2; t < n_tiles; ++t)
-        if (t >= 0 && !bounded_wait(&bb.pm_free[4 * (t & 1) + q], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x8F0,
+        if (t >= 0 && !bounded_wait(&bb.p_free[2 * peer + (t & 1)], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x8F0,
                                     true, true))
           break;
     }
   } else if (warp >= 7) {
-    // ===================================================== shipper / receiver (peer heads of quarter q)
+    // ===================================================== shipper (peer heads of quarter q)
     // Thread (hi, k): peer head m = 32 q + 16 peer + hi, tokens 32 k .. of a tile.
-    // Iteration i: send the partial scores of tile i + 1 to the peer, then take
-    // the peer's P rows of tile i: rescale these heads' O rows if the factor
-    // asks for it, write the rows into P buffer i & 1, and at the end of a
-    // sequence part write out these heads' O rows.
+    // Iteration i: send the partial scores of tile i + 1 to the peer; then, one
+    // tile behind, do what O of tile i - 1 asked of these heads' O rows: the
+    // rescale (rare), and at the end of a sequence part the write-out.
     const int q = warp & 3;
     const int hi = lane & 15, k = lane >> 4;
     const int m = 32 * q + 16 * peer + hi;
-    const int olp = 16 * q + hi;                 // the head's row in the receive buffers
+    const int olp = 16 * q + hi;                 // the head's row in the peer's receive buffer
     const uint32_t lanes = (uint32_t)(32 * q + 16 * peer) << 16;
     const uint32_t peer_row = ptx::mapa(ptx::smem_u32(recv + olp * kT), peer);
     const uint32_t peer_recv_full = ptx::mapa(ptx::smem_u32(&bb.recv_full[q]), peer);
-    const uint32_t peer_pm_free0 = ptx::mapa(ptx::smem_u32(&bb.pm_free[q]), peer);
-    const uint32_t peer_pm_free1 = ptx::mapa(ptx::smem_u32(&bb.pm_free[4 + q]), peer);
+    int n_resc = 0, n_part = 0;
     auto ship = [&](int64_t t) -> bool {
       const int buf = (int)(t & 1);
       if (!warp_wait(&bb.sc_full[buf], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x900, false)) return false;
@@ -831,33 +929,14 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
                          __float_as_uint(v[4 * j + 3]), peer_recv_full);
       return true;
     };
-    bool ok = n_tiles > 0 ? ship(0) : true;
-    int64_t bseq = seq0, btile = tile0;
-    int64_t i = 0;
-    for (; i < n_tiles && ok; ++i, step(bseq, btile)) {
-      if (i + 1 < n_tiles && !(ok = ship(i + 1))) break;
-      const int buf = (int)(i & 1);
-      if (!(ok = warp_wait(&bb.pm_full[4 * buf + q], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x902, true))) break;
-      uint32_t pk[kHalfT / 2];
-      const uint8_t* pm = smem + kOffPMsg + buf * kPMsgBytes;
-      {
-        const uint8_t* row = pm + olp * kPRowBytes;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * ((4 * k + j) ^ (olp & 7)));
-          pk[4 * j] = v.x; pk[4 * j + 1] = v.y; pk[4 * j + 2] = v.z; pk[4 * j + 3] = v.w;
-        }
-      }
-      const float a = *reinterpret_cast<const float*>(pm + kPMsgAlpha + 4 * olp);
-      __syncwarp();
-      // this quarter of buffer `buf` takes the message of tile i + 2 next: armed
-      // before the peer may send it
-      if (lane == 0) {
-        if (i + 2 < n_tiles) ptx::mbar_arrive_expect_tx(&bb.pm_full[4 * buf + q], kPMsgQBytes);
-        ptx::mbar_arrive_remote(buf ? peer_pm_free1 : peer_pm_free0);
-      }
-      if (__any_sync(0xffffffffu, a != 1.f)) {
-        if (!(ok = o_complete(i - 1, 0x903))) break;
+    // what O of tile j needed of these heads' rows, done after O of tile j
+    auto behind = [&](int64_t j, int64_t b, int64_t tile) -> bool {
+      if (!warp_wait(&bb.dec[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x902, false)) return false;
+      if (dec_flag[j & 1]) {
+        // every O before tile j is done (one phase per request, seen in order)
+        const float a = alpha_s[kHeads * (j & 1) + m];
+        if (!warp_wait(bb.resc_go, (uint32_t)n_resc & 1, abort_flag, p, 0x903, false)) return false;
+        ++n_resc;
         ptx::tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -870,20 +949,16 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           ptx::tmem_st16x2_32(ta, o);
         }
         ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bb.resc_done);
       }
-      if (i >= 2 && !(ok = warp_wait(&bb.p_free[buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x904, false)))
-        break;
-      ptx::tc_fence_after();
-      ptx::tmem_st16x2_16(tmem + lanes + kColP + 32u * buf, pk);
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&bb.p_tmem[buf]);
-      if (last_of_part(i, btile)) {
-        const int64_t slot = bseq + c;
-        ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xE08);
-        if (!ok) break;
-        if (!(ok = o_complete(i, 0x905))) break;
+      if (last_of_part(j, tile)) {
+        const int64_t slot = b + c;
+        if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xE08)) return false;
+        // the last O of the part is done (one phase per part, seen in order)
+        if (!warp_wait(bb.part_done, (uint32_t)n_part & 1, abort_flag, p, 0x904, false)) return false;
+        ++n_part;
         ptx::tc_fence_after();
         float* dst = p.part_o + (slot * p.H + h0 + m) * (int64_t)kDC + kDim * r + 32 * k;
 #pragma unroll 1
@@ -897,10 +972,26 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         }
         ptx::tc_fence_before();
       }
+      return true;
+    };
+    bool ok = n_tiles > 0 ? ship(0) : true;
+    int64_t bseq = seq0, btile = tile0;          // (sequence, tile) of tile i - 1
+    int64_t i = 0;
+    for (; i < n_tiles && ok; ++i) {
+      if (i + 1 < n_tiles && !(ok = ship(i + 1))) break;
+      if (i >= 1) {
+        if (!(ok = behind(i - 1, bseq, btile))) break;
+        step(bseq, btile);
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bb.lanes_ready);
     }
-    // the peer's release of the last partial scores has landed here before this CTA exits
-    if (ok && i == n_tiles && n_tiles > 0 && lane == 0)
-      bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true, true);
+    if (ok && i == n_tiles && n_tiles > 0) {
+      behind(n_tiles - 1, bseq, btile);
+      // the peer's release of the last partial scores has landed here before this CTA exits
+      if (lane == 0)
+        bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true, true);
+    }
   }
 
   // ===================================================== teardown
