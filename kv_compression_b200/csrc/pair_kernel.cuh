@@ -177,20 +177,21 @@ __device__ __forceinline__ void record_timeout(volatile int* abort, const PairPa
   if (atomicOr(p.err, kErrTimeout) == 0) atomicExch(p.err + 1, where);
 }
 
-// Bounded wait.  Each probe is an mbarrier.try_wait, which suspends the
-// thread in hardware until the phase completes or a short system-defined
-// limit passes.  `cluster`: acquire at cluster scope (barriers that the peer
-// CTA arrives on or completes transactions on).
-__device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          const PairParams& p, int where, bool honour_abort,
-                                          bool cluster) {
-  auto probe = [&]() {
-    return cluster ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
-  };
-  if (probe()) return true;
+// Bounded wait.  Each probe is an mbarrier.try_wait at CTA scope, which
+// suspends the thread in hardware until the phase completes or a short
+// system-defined limit passes.  The first probe is inline (most waits find
+// the phase complete); the loop with its time bound is out of line.  CTA scope
+// suffices for every barrier here, including those the peer completes: data
+// from the peer lands in this CTA's shared memory before its transaction bytes
+// complete the phase (st.async, bulk copies), and the peer's remote arrivals
+// and multicast MMA commits only report that it has finished reading or
+// writing its own copies.  A cluster-scope acquire on each probe measured
+// about 0.3 us per wait.
+__device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               const PairParams& p, int where, bool honour_abort) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t spin = 1;; ++spin) {
-    if (probe()) return true;
+    if (ptx::mbar_try_wait(bar, parity)) return true;
     if (honour_abort && *abort) return false;
     if ((spin & 7u) == 0 && ptx::globaltimer_ns() - t0 > p.timeout_ns) {
       record_timeout(abort, p, where);
@@ -199,10 +200,16 @@ __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             const PairParams& p, int where, bool honour_abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return bounded_wait_slow(bar, parity, abort, p, where, honour_abort);
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          const PairParams& p, int where, bool cluster) {
+                                          const PairParams& p, int where) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, abort, p, where, true, cluster);
+  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, abort, p, where, true);
   __syncwarp();
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       if (b != cur_b) {
         cur_b = b;
         ++seg;
-        if (seg >= 1) ok = bounded_wait(bb.q_empty, (seg - 1) & 1, abort_flag, p, 0x500, true, false);
+        if (seg >= 1) ok = bounded_wait(bb.q_empty, (seg - 1) & 1, abort_flag, p, 0x500, true);
         if (!ok) break;
         ptx::mbar_arrive_expect_tx(bb.q_full, kAtoms * kQcAtom);
         const int32_t qrow = (int32_t)(b * p.H + h0);
@@ -426,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       {
         const int ks = (int)(i % kNKr);
         const int kk = (int)(i / kNKr);
-        if (kk >= 1) ok = bounded_wait(&bb.kr_empty[ks], (kk - 1) & 1, abort_flag, p, 0x501, true, false);
+        if (kk >= 1) ok = bounded_wait(&bb.kr_empty[ks], (kk - 1) & 1, abort_flag, p, 0x501, true);
         if (!ok) break;
         if (!(p.debug_skip_load && i == 0)) {
           ptx::mbar_arrive_expect_tx(&bb.kr_full[ks], kKrBytes);
@@ -438,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       {
         const int cs = (int)(i % kNS);
         const int ck = (int)(i / kNS);
-        if (ck >= 1) ok = bounded_wait(&bb.c_empty[cs], (ck - 1) & 1, abort_flag, p, 0x502, true, false);
+        if (ck >= 1) ok = bounded_wait(&bb.c_empty[cs], (ck - 1) & 1, abort_flag, p, 0x502, true);
         if (!ok) break;
         if (!LCA_CHECK(p.err, cs < kNS && (int64_t)row < (int64_t)p.B * p.L, 0xE01)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bb.c_full[cs], kStage);
@@ -452,11 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     // Let every copy this thread started land before the CTA can exit.
 #pragma unroll
     for (int i = 0; i < kNS; ++i)
-      if (issued_c[i] >= 0) bounded_wait(&bb.c_full[i], issued_c[i] & 1, abort_flag, p, 0x5F0, false, false);
+      if (issued_c[i] >= 0) bounded_wait(&bb.c_full[i], issued_c[i] & 1, abort_flag, p, 0x5F0, false);
 #pragma unroll
     for (int i = 0; i < kNKr; ++i)
-      if (issued_k[i] >= 0) bounded_wait(&bb.kr_full[i], issued_k[i] & 1, abort_flag, p, 0x5F1, false, false);
-    if (issued_q >= 0) bounded_wait(bb.q_full, issued_q & 1, abort_flag, p, 0x5F2, false, false);
+      if (issued_k[i] >= 0) bounded_wait(&bb.kr_full[i], issued_k[i] & 1, abort_flag, p, 0x5F1, false);
+    if (issued_q >= 0) bounded_wait(bb.q_full, issued_q & 1, abort_flag, p, 0x5F2, false);
   } else if (warp == 1 && lane == 0) {
     // ===================================================== score MMA issuer
     // Tile t: the partial sc[128 x 64] = Q_c[:, dims_r] . C_KV[tile, dims_r]^T
@@ -480,12 +487,12 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         cur_b = b;
         ++seg;
         new_seg = true;
-        ok = bounded_wait(bb.q_full, seg & 1, abort_flag, p, 0x600, true, false);
+        ok = bounded_wait(bb.q_full, seg & 1, abort_flag, p, 0x600, true);
         if (!ok) break;
       }
-      if (t >= 2) ok = bounded_wait(&bb.sc_empty[buf], (uint32_t)((t >> 1) - 1) & 1, abort_flag, p, 0x601, true, false);
-      if (ok) ok = bounded_wait(&bb.kr_full[t % kNKr], (uint32_t)(t / kNKr) & 1, abort_flag, p, 0x602, true, false);
-      if (ok) ok = bounded_wait(&bb.c_full[t % kNS], (uint32_t)(t / kNS) & 1, abort_flag, p, 0x603, true, false);
+      if (t >= 2) ok = bounded_wait(&bb.sc_empty[buf], (uint32_t)((t >> 1) - 1) & 1, abort_flag, p, 0x601, true);
+      if (ok) ok = bounded_wait(&bb.kr_full[t % kNKr], (uint32_t)(t / kNKr) & 1, abort_flag, p, 0x602, true);
+      if (ok) ok = bounded_wait(&bb.c_full[t % kNS], (uint32_t)(t / kNS) & 1, abort_flag, p, 0x603, true);
       if (!ok) break;
       ptx::tc_fence_after();
       {
@@ -499,8 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
                              b0 + (uint64_t)((a * kCAtom + 32 * k) >> 4), kIdescS, (a | k) != 0);
       }
       ptx::mma_commit(&bb.sc_full[buf]);
-      if (t >= 1) ok = bounded_wait(bb.sr_empty, (uint32_t)(t - 1) & 1, abort_flag, p, 0x604, true, false);
-      if (ok && new_seg) ok = bounded_wait(&bb.qr_full[seg & 1], (uint32_t)(seg >> 1) & 1, abort_flag, p, 0x605, true, false);
+      if (t >= 1) ok = bounded_wait(bb.sr_empty, (uint32_t)(t - 1) & 1, abort_flag, p, 0x604, true);
+      if (ok && new_seg) ok = bounded_wait(&bb.qr_full[seg & 1], (uint32_t)(seg >> 1) & 1, abort_flag, p, 0x605, true);
       if (!ok) break;
       ptx::tc_fence_after();
       {
@@ -518,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       }
     }
     ptx::mma_commit(&bb.drain[0]);
-    bounded_wait(&bb.drain[0], 0, abort_flag, p, 0x6F0, false, false);
+    bounded_wait(&bb.drain[0], 0, abort_flag, p, 0x6F0, false);
   } else if (warp == 2 && lane == 0) {
     // ===================================================== O MMA issuer
     // Tile j once P buffer j & 1 is complete (own rows, the peer's rows and
@@ -535,16 +542,16 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     int64_t oseq = seq0, otile = tile0;
     for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile)) {
       const int buf = (int)(j & 1);
-      if (!bounded_wait(bb.p_local, (uint32_t)j & 1, abort_flag, p, 0x700, true, false)) break;
+      if (!bounded_wait(bb.p_local, (uint32_t)j & 1, abort_flag, p, 0x700, true)) break;
       bool ok = true;
       for (int q = 0; q < 4 && ok; ++q)
-        ok = bounded_wait(&bb.p_remote[4 * buf + q], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x701, true, true);
+        ok = bounded_wait(&bb.p_remote[4 * buf + q], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x701, true);
       if (!ok) break;
       // this buffer takes the peer's rows of tile j + 2 next; the peer writes
       // them only after this CTA's O of tile j is done
       if (j + 2 < n_tiles)
         for (int q = 0; q < 4; ++q) ptx::mbar_arrive_expect_tx(&bb.p_remote[4 * buf + q], kPQBytes);
-      if (!bounded_wait(bb.lanes_ready, (uint32_t)j & 1, abort_flag, p, 0x702, true, false)) break;
+      if (!bounded_wait(bb.lanes_ready, (uint32_t)j & 1, abort_flag, p, 0x702, true)) break;
       bool resc = false;
       if (j > 0 && otile > 0) {
         const float* al = alpha_s + kHeads * buf;
@@ -562,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       dec_flag[j & 1] = resc ? 1 : 0;
       ptx::mbar_arrive(&bb.dec[j & 1]);
       if (resc) {
-        if (!bounded_wait(bb.resc_done, (uint32_t)n_resc & 1, abort_flag, p, 0x703, true, false)) break;
+        if (!bounded_wait(bb.resc_done, (uint32_t)n_resc & 1, abort_flag, p, 0x703, true)) break;
         ++n_resc;
       }
       ptx::tc_fence_after();
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       if (last_of_part(j, otile)) ptx::mma_commit(bb.part_done);
     }
     ptx::mma_commit(&bb.drain[1]);
-    bounded_wait(&bb.drain[1], 0, abort_flag, p, 0x7F0, false, false);
+    bounded_wait(&bb.drain[1], 0, abort_flag, p, 0x7F0, false);
   } else if (warp >= 3 && warp <= 6) {
     // ===================================================== softmax (own heads of quarter q)
     // Thread (hi, k): head m = 32 q + 16 r + hi, tokens 32 k .. 32 k + 31 of a tile.
@@ -599,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     // q_r of sequence `seq` (segment s) into TMEM buffer s & 1, both lane
     // halves of this quarter: this thread's 32 dims of its own and its peer head
     auto load_qr = [&](int64_t seq, int s) -> bool {
-      if (s >= 2 && !warp_wait(&bb.qr_empty[s & 1], (uint32_t)((s >> 1) - 1) & 1, abort_flag, p, 0x807, false))
+      if (s >= 2 && !warp_wait(&bb.qr_empty[s & 1], (uint32_t)((s >> 1) - 1) & 1, abort_flag, p, 0x807))
         return false;
       uint32_t own[16], oth[16];
       const uint4* src_own = reinterpret_cast<const uint4*>(p.q_r + ((int64_t)seq * p.H + h0 + m) * kDR + 32 * k);
@@ -627,8 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     for (; i < n_tiles && ok; ++i, step(cseq, ctile)) {
       const int64_t b = cseq, tile = ctile;
       const int buf = (int)(i & 1);
-      if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x800, false)) break;
-      if (!warp_wait(&bb.recv_full[q], (uint32_t)i & 1, abort_flag, p, 0x801, true)) break;
+      if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x800)) break;
+      if (!warp_wait(&bb.recv_full[q], (uint32_t)i & 1, abort_flag, p, 0x801)) break;
       ptx::tc_fence_after();
       float x[kHalfT], sr[kHalfT];
       ptx::tmem_ld16x2_32(tmem + lanes + kColSc + 64u * buf, x);
@@ -810,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         // scaled here; this warp saw buffer (i - 1) & 1's earlier release when
         // it wrote P of tile i - 1
         const int pb = (int)((i - 1) & 1);
-        if (!warp_wait(&bb.p_free[2 * r + pb], (uint32_t)((i - 1) >> 1) & 1, abort_flag, p, 0x803, true)) break;
+        if (!warp_wait(&bb.p_free[2 * r + pb], (uint32_t)((i - 1) >> 1) & 1, abort_flag, p, 0x803)) break;
         ptx::tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -827,7 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       }
       // ---- this head's P row and factor into this CTA's P buffer (free once
       // its O of tile i - 2 is done; the previous copy out of it has read it)
-      if (i >= 2 && !warp_wait(&bb.p_free[2 * r + buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x804, true))
+      if (i >= 2 && !warp_wait(&bb.p_free[2 * r + buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x804))
         break;
       if (lane == 0 && copy_pending) {
         ptx::bulk_wait_group_read0();
@@ -846,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       __syncwarp();
       // ---- the same 16 rows and factors into the peer's P buffer (free once
       // the peer's O of tile i - 2 is done): two bulk copies, same offsets
-      if (i >= 2 && !warp_wait(&bb.p_free[2 * peer + buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x805, true))
+      if (i >= 2 && !warp_wait(&bb.p_free[2 * peer + buf], (uint32_t)((i >> 1) - 1) & 1, abort_flag, p, 0x805))
         break;
       if (lane == 0) {
         const uint32_t bar = buf ? peer_p_remote1 : peer_p_remote0;
@@ -865,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         // buffer i & 1 is released (this warp saw its previous release above).
         const int64_t slot = b + c;
         const bool slot_ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xE06);
-        if (!warp_wait(&bb.p_free[2 * r + buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x806, true)) break;
+        if (!warp_wait(&bb.p_free[2 * r + buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x806)) break;
         ptx::tc_fence_after();
         float* dst = p.part_o + (slot * p.H + h) * (int64_t)kDC + kDim * r + 32 * k;
 #pragma unroll 1
@@ -893,8 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     // this CTA's shared memory) have landed before this CTA exits.
     if (lane == 0 && q == 0 && i == n_tiles) {
       for (int64_t t = n_tiles - 2; t < n_tiles; ++t)
-        if (t >= 0 && !bounded_wait(&bb.p_free[2 * peer + (t & 1)], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x8F0,
-                                    true, true))
+        if (t >= 0 && !bounded_wait(&bb.p_free[2 * peer + (t & 1)], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x8F0, true))
           break;
     }
   } else if (warp >= 7) {
@@ -913,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     int n_resc = 0, n_part = 0;
     auto ship = [&](int64_t t) -> bool {
       const int buf = (int)(t & 1);
-      if (!warp_wait(&bb.sc_full[buf], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x900, false)) return false;
+      if (!warp_wait(&bb.sc_full[buf], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x900)) return false;
       ptx::tc_fence_after();
       float v[32];
       ptx::tmem_ld16x2_32(tmem + lanes + kColSc + 64u * buf, v);
@@ -921,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bb.sc_empty[buf]);
-      if (t >= 1 && !warp_wait(&bb.recv_free[q], (uint32_t)(t - 1) & 1, abort_flag, p, 0x901, true)) return false;
+      if (t >= 1 && !warp_wait(&bb.recv_free[q], (uint32_t)(t - 1) & 1, abort_flag, p, 0x901)) return false;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         ptx::st_async_v4(peer_row + 16u * (uint32_t)((8 * k + j) ^ (olp & 15)), __float_as_uint(v[4 * j]),
@@ -931,11 +937,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     };
     // what O of tile j needed of these heads' rows, done after O of tile j
     auto behind = [&](int64_t j, int64_t b, int64_t tile) -> bool {
-      if (!warp_wait(&bb.dec[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x902, false)) return false;
+      if (!warp_wait(&bb.dec[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x902)) return false;
       if (dec_flag[j & 1]) {
         // every O before tile j is done (one phase per request, seen in order)
         const float a = alpha_s[kHeads * (j & 1) + m];
-        if (!warp_wait(bb.resc_go, (uint32_t)n_resc & 1, abort_flag, p, 0x903, false)) return false;
+        if (!warp_wait(bb.resc_go, (uint32_t)n_resc & 1, abort_flag, p, 0x903)) return false;
         ++n_resc;
         ptx::tc_fence_after();
 #pragma unroll 1
@@ -957,7 +963,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         const int64_t slot = b + c;
         if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xE08)) return false;
         // the last O of the part is done (one phase per part, seen in order)
-        if (!warp_wait(bb.part_done, (uint32_t)n_part & 1, abort_flag, p, 0x904, false)) return false;
+        if (!warp_wait(bb.part_done, (uint32_t)n_part & 1, abort_flag, p, 0x904)) return false;
         ++n_part;
         ptx::tc_fence_after();
         float* dst = p.part_o + (slot * p.H + h0 + m) * (int64_t)kDC + kDim * r + 32 * k;
@@ -990,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       behind(n_tiles - 1, bseq, btile);
       // the peer's release of the last partial scores has landed here before this CTA exits
       if (lane == 0)
-        bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true, true);
+        bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true);
     }
   }
 
