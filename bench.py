@@ -42,10 +42,15 @@ import workloads  # noqa: E402
 METRIC = "LCA decode context tokens/s per GPU; HBM GB/s as % of B200 peak"
 UNIT = "context tokens/s"
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCES = ["kv_compression_b200/csrc/tc_kernel.cuh", "kv_compression_b200/csrc/pair_kernel.cuh",
-                  "kv_compression_b200/csrc/ptx.cuh"]
-TRAFFIC_FILE = "profiles/lca_tc_kernel_v2lite_traffic.txt"
-TRAFFIC_WORKLOAD = "v2lite"           # the workload that capture ran on
+# committed ncu DRAM-traffic summaries of the main kernel, per workload, and
+# the sources of that kernel (a summary counts only while they are unchanged)
+_CSRC = "kv_compression_b200/csrc/"
+TRAFFIC_FILES = {
+    "v2lite": ("profiles/lca_tc_kernel_v2lite_traffic.txt",
+               [_CSRC + "tc_kernel.cuh", _CSRC + "ptx.cuh", _CSRC + "checks.cuh"]),
+    "v2": ("profiles/lca_pair_kernel_v2_traffic.txt",
+           [_CSRC + "pair_kernel.cuh", _CSRC + "ptx.cuh", _CSRC + "checks.cuh"]),
+}
 MAIN_KERNEL_NAMES = {"tcgen05": "lca_tc_kernel", "tcgen05_pair": "lca_pair_kernel", "simt": "lca_simt_kernel"}
 
 
@@ -72,27 +77,31 @@ def measured_peaks() -> tuple[dict, str]:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(sources: list[str]) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(wl: workloads.Workload) -> int | None:
-    """DRAM bytes per launch of the main kernel from the committed ncu summary,
-    or None when absent, taken on another workload or on a different kernel source."""
-    path = os.path.join(ROOT, TRAFFIC_FILE)
-    if wl.name != TRAFFIC_WORKLOAD or not os.path.exists(path):
+    """DRAM bytes per launch of the main kernel from the committed ncu summary
+    for this workload, or None when absent, taken at another batch size or on a
+    different kernel source."""
+    entry = TRAFFIC_FILES.get(wl.name)
+    path = os.path.join(ROOT, entry[0]) if entry else None
+    if not path or not os.path.exists(path):
         return None
     kv = {}
     with open(path) as f:
         for line in f:
-            if ":" in line:
+            if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("source_sha256") != kernel_source_sha():
+    if kv.get("source_sha256") != kernel_source_sha(entry[1]):
+        return None
+    if "batch" in kv and int(kv["batch"]) != wl.B:
         return None
     try:
         return int(kv["dram_bytes_per_launch"])
