@@ -225,7 +225,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Pairwise (tree) reductions over N compile-time-indexed values: depth log2 N
+// Pairwise (tree) maximum over N compile-time-indexed values: depth log2 N
 // instead of a chain of N - 1 dependent operations.
 template <int N>
 __device__ __forceinline__ float tree_max(const float* v) {
@@ -235,45 +235,56 @@ __device__ __forceinline__ float tree_max(const float* v) {
     return fmaxf(tree_max<N / 2>(v), tree_max<N / 2>(v + N / 2));
   }
 }
-template <int N>
-__device__ __forceinline__ float tree_sum(const float* v) {
-  if constexpr (N == 1) {
-    return v[0];
-  } else {
-    return tree_sum<N / 2>(v) + tree_sum<N / 2>(v + N / 2);
-  }
-}
 
 // Statistics of one group held by one thread: x[0..N) the semantic scores,
 // sr[0..N) the positional ones; on return e[] holds e_t = e^{s_t - m}.
 // m = max s_t, a = the lowest index attaining it, sra = sr_a, den = sum e_t,
 // num = sum e_t sc_t.
+// The elementwise work runs on packed fp32 pairs (two tokens per instruction).
 template <int N>
 __device__ __forceinline__ void group_stats(const float* x, const float* sr, float* e, float& m, int& a,
                                             float& sra, float& den, float& num) {
-  float s[N];
+  if constexpr (N == 1) {
+    m = x[0] + sr[0];
+    a = 0;
+    sra = sr[0];
+    e[0] = 1.f;
+    den = 1.f;
+    num = x[0];
+  } else {
+    float s[N];
 #pragma unroll
-  for (int t = 0; t < N; ++t) s[t] = x[t] + sr[t];
-  m = tree_max<N>(s);
-  // scanning down, the last hit is the lowest index attaining the maximum
-  a = 0;
-  sra = sr[0];
+    for (int t = 0; t < N; t += 2)
+      ptx::f32x2_split(ptx::add_f32x2(ptx::f32x2(x[t], x[t + 1]), ptx::f32x2(sr[t], sr[t + 1])), s[t], s[t + 1]);
+    m = tree_max<N>(s);
+    // scanning down, the last hit is the lowest index attaining the maximum
+    a = 0;
+    sra = sr[0];
 #pragma unroll
-  for (int t = N - 1; t >= 0; --t) {
-    const bool hit = s[t] == m;
-    a = hit ? t : a;
-    sra = hit ? sr[t] : sra;
+    for (int t = N - 1; t >= 0; --t) {
+      const bool hit = s[t] == m;
+      a = hit ? t : a;
+      sra = hit ? sr[t] : sra;
+    }
+    const float mb = -m * kLog2e;
+    const uint64_t l2e = ptx::f32x2(kLog2e, kLog2e), mb2 = ptx::f32x2(mb, mb);
+    uint64_t nacc = ptx::f32x2(0.f, 0.f), dacc = ptx::f32x2(0.f, 0.f);
+#pragma unroll
+    for (int t = 0; t < N; t += 2) {
+      float u0, u1;
+      ptx::f32x2_split(ptx::fma_f32x2(ptx::f32x2(s[t], s[t + 1]), l2e, mb2), u0, u1);
+      e[t] = ex2(u0);
+      e[t + 1] = ex2(u1);
+      const uint64_t ee = ptx::f32x2(e[t], e[t + 1]);
+      nacc = ptx::fma_f32x2(ee, ptx::f32x2(x[t], x[t + 1]), nacc);
+      dacc = ptx::add_f32x2(dacc, ee);
+    }
+    float n0, n1, d0, d1;
+    ptx::f32x2_split(nacc, n0, n1);
+    ptx::f32x2_split(dacc, d0, d1);
+    num = n0 + n1;
+    den = d0 + d1;
   }
-  const float mb = -m * kLog2e;
-  float n0 = 0.f, n1 = 0.f;
-#pragma unroll
-  for (int t = 0; t < N; ++t) {
-    e[t] = ex2(fmaf(s[t], kLog2e, mb));
-    if (t & 1) n1 = fmaf(e[t], x[t], n1);
-    else n0 = fmaf(e[t], x[t], n0);
-  }
-  den = tree_sum<N>(e);
-  num = n0 + n1;
 }
 
 template <int LOG2G>
@@ -647,7 +658,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         for (int j = 0; j < 8; ++j) {
           const int phys = (8 * k + j) ^ (ol & 15);
           const float4 v = *reinterpret_cast<const float4*>(rrow + 4 * phys);
-          x[4 * j] += v.x; x[4 * j + 1] += v.y; x[4 * j + 2] += v.z; x[4 * j + 3] += v.w;
+          ptx::f32x2_split(ptx::add_f32x2(ptx::f32x2(x[4 * j], x[4 * j + 1]), ptx::f32x2(v.x, v.y)), x[4 * j],
+                           x[4 * j + 1]);
+          ptx::f32x2_split(ptx::add_f32x2(ptx::f32x2(x[4 * j + 2], x[4 * j + 3]), ptx::f32x2(v.z, v.w)),
+                           x[4 * j + 2], x[4 * j + 3]);
         }
       }
       ptx::tc_fence_before();
@@ -789,22 +803,32 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           }
         }
         const float mb = -M * kLog2e;
+        if constexpr (kFast) {   // every token is grouped: one packed multiply per pair
 #pragma unroll
-        for (int t2 = 0; t2 < kHalfT / 2; ++t2) {
-          float pv[2];
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int t = 2 * t2 + e2;
-            float v;
-            if (kFast || grp[t / GW]) {
-              v = s[t] * f[t / GW];
-            } else {
-              v = tok0 + t < p.L ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
-              Z += v;
-            }
-            pv[e2] = v;
+          for (int t2 = 0; t2 < kHalfT / 2; ++t2) {
+            const float ff = f[(2 * t2) / GW];
+            float a0, a1;
+            ptx::f32x2_split(ptx::mul_f32x2(ptx::f32x2(s[2 * t2], s[2 * t2 + 1]), ptx::f32x2(ff, ff)), a0, a1);
+            pk[t2] = pack_bf16x2(a0, a1);
           }
-          pk[t2] = pack_bf16x2(pv[0], pv[1]);
+        } else {
+#pragma unroll
+          for (int t2 = 0; t2 < kHalfT / 2; ++t2) {
+            float pv[2];
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const int t = 2 * t2 + e2;
+              float v;
+              if (grp[t / GW]) {
+                v = s[t] * f[t / GW];
+              } else {
+                v = tok0 + t < p.L ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
+                Z += v;
+              }
+              pv[e2] = v;
+            }
+            pk[t2] = pack_bf16x2(pv[0], pv[1]);
+          }
         }
       };
       const bool fast = g > 1 && (tile + 1) * kT <= win0;   // warp-uniform
