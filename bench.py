@@ -417,6 +417,13 @@ class Runner:
         q_c, q_r, c_kv, k_r = self.dev[k % self.copies]
         self.plan.dense(q_c, q_r, c_kv, k_r, self.wl.L, self.out, self.stream)
 
+    def check_device(self) -> None:
+        """Raise, naming the workload and the wait site, if a kernel reported an error."""
+        st = self.plan.device_error()
+        if st != self.kvc.LCA_OK:
+            raise RuntimeError(f"device error {st} at site {self.plan.device_error_site():#x} on "
+                               f"{workload_desc(self.wl)}")
+
     def main_kernel_time(self, steps: int, g=None, w=None) -> list[float]:
         """Per-step duration of the main kernel alone: an event recorded on the
         launching stream before the step and, by the library, right after the
@@ -433,7 +440,7 @@ class Runner:
             self.step(k, g, w)
         torch.cuda.synchronize()
         self.plan.set_timing_event(None)
-        assert self.plan.device_error() == self.kvc.LCA_OK
+        self.check_device()
         return [ev_s[k].elapsed_time(ev_m[k]) * 1e-3 for k in range(steps)]
 
     def free(self) -> None:
@@ -503,7 +510,7 @@ def stored_leg(torch, kvc, r, K: int, peaks: dict, t_lca: float, t_mla: float) -
         for k in range(K):
             step(k)
         blocks.append(t.stop() / K)
-    assert r.plan.device_error() == kvc.LCA_OK
+    r.check_device()
     ts = statistics.median(blocks)
     alg = store_bytes + wl.B * wl.H * (wl.d_c + wl.d_r) * wl.elem_bytes + wl.B * wl.H * wl.d_c * 4
     del stores
@@ -588,7 +595,7 @@ def our_arm(args) -> None:
     for k in range(args.warmup):
         r.step(k)
     t_warm = tw.stop() / max(args.warmup, 1)
-    assert r.plan.device_error() == kvc.LCA_OK
+    r.check_device()
 
     K = args.steps
 
@@ -614,7 +621,7 @@ def our_arm(args) -> None:
     clocks = nvml.stop()
     block_s = [rank_max(t) for t in block_s]
     t_total = statistics.median(block_s)
-    assert r.plan.device_error() == kvc.LCA_OK
+    r.check_device()
 
     # The main kernel's own duration (its roofline): events on the launching stream
     # around each main-kernel launch, over a second pass of K steps.
@@ -628,7 +635,7 @@ def our_arm(args) -> None:
     barrier_sync()
     dense_s = [rank_max(t) for t in timed_blocks(torch, r, kd, 3, barrier_sync, fn=r.dense)]
     t_dense = statistics.median(dense_s)
-    assert r.plan.device_error() == kvc.LCA_OK
+    r.check_device()
 
     stored = None
     if not args.no_stored:

@@ -256,6 +256,16 @@ const char *lca_status_string(lca_status status);
 lca_status lca_get_device_error(lca_plan *plan, void *stream);
 
 /*
+ * The site of the last error that lca_get_device_error reported for this plan:
+ * a code naming the wait that ran out (or, in the range-checked build, the
+ * check that failed) inside the kernel, 0 if none was reported yet or for a
+ * NULL plan.  Codes are fixed per wait site in the kernel sources (for
+ * example 0x7xx for the O-MMA issuer of the two-CTA kernel).  Host only; no
+ * CUDA call.
+ */
+int lca_get_device_error_site(const lca_plan *plan);
+
+/*
  * Instrumentation for measuring the main kernel on its own: when `event` (a
  * cudaEvent_t) is non-NULL, each later lca_decode / mla_decode call records it
  * on the call's stream right after launching the main kernel and before

@@ -30,7 +30,7 @@ EXPORTS = ["lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", 
            "lca_decode_host", "lca_num_groups", "lca_status_string", "lca_get_device_error",
            "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
            "lca_stored_rows", "lca_build_stored", "lca_decode_stored", "lca_slice_groups",
-           "lca_decode_partial", "lca_merge_partials"]
+           "lca_decode_partial", "lca_merge_partials", "lca_get_device_error_site"]
 
 
 class LcaError(RuntimeError):
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lca_slice_groups.restype = i64
     lib.lca_decode_partial.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
     lib.lca_merge_partials.argtypes = [vp, i32, vp, vp, vp, vp]
+    lib.lca_get_device_error_site.argtypes = [vp]
+    lib.lca_get_device_error_site.restype = i32
     for name in ("lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
                  "lca_decode_host", "lca_get_device_error", "lca_plan_kernel",
                  "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
@@ -205,6 +207,10 @@ class Plan:
 
     def device_error(self, stream=None) -> int:
         return int(self._lib.lca_get_device_error(self._h, _stream_handle(stream)))
+
+    def device_error_site(self) -> int:
+        """Where (a per-wait-site code) the last error device_error reported arose."""
+        return int(self._lib.lca_get_device_error_site(self._h))
 
 
 def lca_decode(q_c, q_r, c_kv, k_r, g: int, w: int, plan: Plan | None = None, stream=None):

@@ -32,6 +32,7 @@ struct lca_plan {
   float* part_o;           // [ws_slots][H][d_c]
   float* part_mz;          // [ws_slots][H][2]
   int* err;                // [2]: flags, where
+  int last_site;           // where of the last error lca_get_device_error reported
   // options
   bool force_simt;
   int kernel_pref;         // 0: automatic, else the lca_plan_kernel code to use
@@ -741,9 +742,12 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
   if (cudaMemcpy(host, p->err, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess)
     return LCA_ERR_CUDA;
   if (host[0] != 0 && cudaMemset(p->err, 0, sizeof(host)) != cudaSuccess) return LCA_ERR_CUDA;
+  if (host[0] != 0) p->last_site = host[1];
   if (host[0] & lca::kErrCheck) return LCA_ERR_DEVICE_CHECK;
   return host[0] != 0 ? LCA_ERR_DEVICE_TIMEOUT : LCA_OK;
 }
+
+int lca_get_device_error_site(const lca_plan* p) { return p ? p->last_site : 0; }
 
 // For callers that may not allocate device memory when they decode -- a
 // server whose memory is all reserved up front by its own pool (a cudaMalloc

@@ -64,7 +64,8 @@ def run_lca(plan: kvc.Plan, d: DeviceInputs, g: int, w: int):
     anc = Guarded((wl.B, wl.H, max(nG, 1)), torch.int32, -7, ANC_SENTINEL)
     plan.decode(d.q_c, d.q_r, d.c_kv, d.k_r, wl.L, g, w, out.t, anc.t if nG > 0 else None)
     torch.cuda.synchronize()
-    assert plan.device_error() == kvc.LCA_OK
+    st = plan.device_error()
+    assert st == kvc.LCA_OK, f"device error {st} at wait site {plan.device_error_site():#x}"
     out.check()
     anc.check()
     return out.t.cpu().numpy().astype(np.float64), anc.t.cpu().numpy()[:, :, :nG]
