@@ -301,3 +301,47 @@ def merge(ms, zs, os_, lib: ctypes.CDLL | None = None) -> np.ndarray:
             lib.lca_oracle_merge(n, d_c, _ptr(m), _ptr(z), _ptr(o), _ptr(r))
             out[b, h] = r
     return out
+
+
+@dataclass
+class PagedResult:
+    out: np.ndarray            # [B, H, d_c] float64
+    anchor: list               # per sequence b: [H, n_G(b)] int32
+    tie_gap: list              # per sequence b: [H, n_G(b)] float64
+    max_abs_s: np.ndarray      # [B, H] float64
+
+
+def paged_rows(block_table, b: int, L: int, page_size: int) -> np.ndarray:
+    """Pool rows of tokens 0 .. L-1 of sequence b: token t sits in page
+    block_table[b, t // page_size], at offset t % page_size in it."""
+    t = np.arange(L, dtype=np.int64)
+    return block_table[b, t // page_size].astype(np.int64) * page_size + t % page_size
+
+
+def lca_paged(q_c, q_r, c_pool, k_pool, block_table, seq_lens, page_size: int, g: int, w: int,
+              nthreads: int = 0, lib: ctypes.CDLL | None = None) -> PagedResult:
+    """LCA decode over a paged cache with a length per sequence.
+
+    q_c [B,H,d_c], q_r [B,H,d_r]; c_pool [P*page_size, d_c], k_pool
+    [P*page_size, d_r]; block_table [B, max_pages] int; seq_lens [B].  Sequence
+    b is the contiguous context of its seq_lens[b] tokens gathered through its
+    block-table row (paged_rows), decoded exactly as ``lca`` decodes a
+    contiguous cache of that length: its own segmentation (n_G(b) groups,
+    section 2 step 1) and its own window.  No pool row outside those tokens
+    is read.
+    """
+    lib = lib or load()
+    B, H, d_c = q_c.shape
+    out = np.zeros((B, H, d_c), np.float64)
+    mx = np.zeros((B, H), np.float64)
+    anchors, gaps = [], []
+    for b in range(B):
+        L = int(seq_lens[b])
+        rows = paged_rows(block_table, b, L, page_size)
+        r = lca(q_c[b:b + 1], q_r[b:b + 1], c_pool[rows][None], k_pool[rows][None], g, w,
+                nthreads=nthreads, lib=lib)
+        out[b] = r.out[0]
+        mx[b] = r.max_abs_s[0]
+        anchors.append(r.anchor[0])
+        gaps.append(r.tie_gap[0])
+    return PagedResult(out, anchors, gaps, mx)

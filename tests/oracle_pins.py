@@ -29,6 +29,7 @@ import torch
 import torch.nn.functional as F
 
 from oracle import oracle as orc
+import workloads
 from workloads import bf16_bits_to_f32, f32_to_bf16_bits
 
 REL_TOL = 1e-10  # double vs double, different summation orders
@@ -448,9 +449,62 @@ def pin_stored_zero_query(lib):
         assert np.array_equal(ka[0, jj], widen(K[0, 5 * j]))
 
 
+# ----------------------------------------------------------------------------- paged cache
+def _paged_inputs(rng, dtype, B, L, d_c=16, d_r=8, H=2):
+    q_c, q_r, c_kv, k_r = rand_inputs(rng, B, H, L, d_c, d_r, dtype)
+    wl = workloads.small("paged_pin", B=B, H=H, L=L, g=8, w=20, d_c=d_c, d_r=d_r, dtype=dtype)
+    return workloads.Inputs(wl, q_c, q_r, c_kv, k_r)
+
+
+def _check_paged_against_prefix(lib, x, cache, g, w):
+    """Each sequence of the paged decode against the torch-built LCA of its own
+    contiguous tokens [0, L_b) (and, exactly, against the oracle's contiguous
+    decode of them)."""
+    res = orc.lca_paged(x.q_c, x.q_r, cache.c_pool, cache.k_pool, cache.block_table, cache.seq_lens,
+                        cache.page_size, g, w, lib=lib)
+    assert np.all(np.isfinite(res.out)), "a NaN row outside the sequences was read"
+    for b, L in enumerate(cache.seq_lens):
+        L = int(L)
+        C, K = x.c_kv[b:b + 1, :L], x.k_r[b:b + 1, :L]
+        ref, anc = torch_lca_seq(widen(x.q_c[b]), widen(x.q_r[b]), widen(C[0]), widen(K[0]), g, w)
+        assert rel_err(res.out[b], ref) < REL_TOL, (b, L)
+        assert np.array_equal(res.anchor[b], anc), (b, L)
+        whole = orc.lca(x.q_c[b:b + 1], x.q_r[b:b + 1], np.ascontiguousarray(C), np.ascontiguousarray(K),
+                        g, w, lib=lib)
+        assert np.array_equal(res.out[b], whole.out[0]) and np.array_equal(res.anchor[b], whole.anchor[0])
+
+
+def pin_paged_vs_prefix(lib):
+    """Paged, variable-length decode: sequence b gathered through its block
+    table is its own context of L_b tokens (lengths of one token, one page,
+    ragged, and longer than the window), for two page sizes and both element
+    types; every unowned pool row holds NaN."""
+    for dtype, ps, seed in (("f32", 64, 41), ("bf16", 64, 42), ("f32", 128, 43)):
+        rng = np.random.default_rng(seed)
+        x = _paged_inputs(rng, dtype, B=5, L=300)
+        cache = workloads.paged_layout(x, [300, 1, 130, 64, 21], ps, seed=seed)
+        _check_paged_against_prefix(lib, x, cache, 8, 20)
+
+
+def pin_paged_shared_prefix(lib):
+    """Two sequences sharing their first pages (a common prompt prefix): the
+    second sees the shared tokens as its own first tokens."""
+    rng = np.random.default_rng(44)
+    x = _paged_inputs(rng, "f32", B=3, L=400)
+    x.c_kv[1, :256] = x.c_kv[0, :256]
+    x.k_r[1, :256] = x.k_r[0, :256]
+    x.c_kv[2, :128] = x.c_kv[0, :128]
+    x.k_r[2, :128] = x.k_r[0, :128]
+    cache = workloads.paged_layout(x, [300, 400, 150], 64, seed=44, shared_prefix={1: (0, 4), 2: (0, 2)})
+    assert np.array_equal(cache.block_table[1, :4], cache.block_table[0, :4])
+    assert np.array_equal(cache.block_table[2, :2], cache.block_table[0, :2])
+    _check_paged_against_prefix(lib, x, cache, 8, 20)
+
+
 STORED_PINS = [pin_stored_brute_force, pin_stored_g1_dense, pin_stored_single_head,
                pin_stored_constant_groups, pin_stored_zero_query]
 
 ALL_PINS = [pin_segmentation, pin_dense_vs_torch, pin_g1_dense, pin_window_dense, pin_zero_query,
             pin_constant_groups, pin_brute_force, pin_near_tie_report, pin_ties, pin_formulations,
-            pin_permutation, pin_constant_rope] + STORED_PINS
+            pin_permutation, pin_constant_rope] + STORED_PINS + [pin_paged_vs_prefix,
+                                                                  pin_paged_shared_prefix]

@@ -53,3 +53,29 @@ def test_registry_shapes():
     assert (W["v2lite"].B, W["v2lite"].H, W["v2lite"].L, W["v2lite"].g, W["v2lite"].w) == (8, 16, 32768, 16, 1024)
     assert W["v2lite"].n_groups == 1984 and W["v2"].n_groups == 3968 and W["needle"].n_groups == 3968
     assert len(W["sweep"].sweep) == 10
+
+
+def test_paged_layout_places_every_token_once():
+    wl = workloads.small("paged", B=3, H=2, L=300, g=8, w=20, d_c=16, d_r=8, dtype="bf16", seed=5)
+    x = workloads.generate(wl, threads=1)
+    lens = [300, 65, 1]
+    cache = workloads.paged_layout(x, lens, 64, seed=5, spare_pages=2)
+    ps = cache.page_size
+    owned = np.zeros(cache.c_pool.shape[0], bool)
+    for b, L in enumerate(lens):
+        need = -(-L // ps)
+        pages = cache.block_table[b, :need]
+        assert np.all((pages >= 0) & (pages < cache.num_pages))
+        assert np.all(cache.block_table[b, need:] == -1)
+        for t in (0, L // 2, L - 1):
+            row = pages[t // ps] * ps + t % ps
+            assert np.array_equal(cache.c_pool[row], x.c_kv[b, t])
+            assert np.array_equal(cache.k_pool[row], x.k_r[b, t])
+        rows = pages[:, None].astype(np.int64) * ps + np.arange(ps)[None]
+        owned[rows.reshape(-1)[:L]] = True
+    assert cache.num_pages == (5 + 2 + 1) + 2
+    nan = workloads.nan_fill("bf16")
+    assert np.all(cache.c_pool[~owned] == nan) and np.all(cache.k_pool[~owned] == nan)
+    assert not np.any(cache.c_pool[owned] == nan)
+    again = workloads.paged_layout(x, lens, 64, seed=5, spare_pages=2)
+    assert np.array_equal(again.block_table, cache.block_table)

@@ -35,7 +35,7 @@ from dataclasses import dataclass, field, replace
 
 import numpy as np
 
-TENSOR_ID = {"q_c": 1, "q_r": 2, "c_kv": 3, "k_r": 4, "needle_pos": 5}
+TENSOR_ID = {"q_c": 1, "q_r": 2, "c_kv": 3, "k_r": 4, "needle_pos": 5, "page_order": 6}
 NEEDLES_PER_SEQ = 64
 
 
@@ -178,3 +178,71 @@ def small(name: str, B: int, H: int, L: int, g: int, w: int, d_c: int = 512, d_r
         return Workload(name, B, H, d_c, d_r, L, g, w, "f32", s, s, needles, seed)
     return Workload(name, B, H, d_c, d_r, L, g, w, "bf16", 1.0 / math.sqrt(d_c + d_r), 1.0,
                     needles, seed)
+
+
+@dataclass
+class PagedCache:
+    """A batch's caches laid out in pages of a shared pool (input layout only)."""
+    c_pool: np.ndarray        # [num_pages * page_size, d_c]
+    k_pool: np.ndarray        # [num_pages * page_size, d_r]
+    block_table: np.ndarray   # [B, max_pages] int32
+    seq_lens: np.ndarray      # [B] int32
+    page_size: int
+
+    @property
+    def num_pages(self) -> int:
+        return self.c_pool.shape[0] // self.page_size
+
+
+def nan_fill(dtype: str):
+    """The value planted in pool rows that no sequence owns: a quiet NaN."""
+    return np.uint16(0x7FC0) if dtype == "bf16" else np.float32(np.nan)
+
+
+def paged_layout(x: Inputs, seq_lens, page_size: int, seed: int = 0, spare_pages: int = 3,
+                 shared_prefix: dict | None = None, unused_entry: int = -1) -> PagedCache:
+    """Scatter tokens [0, seq_lens[b]) of each sequence of ``x`` into pages of a
+    pool, in a seeded random page order (rng tensor "page_order").
+
+    Every pool row that holds none of those tokens -- the spare pages, and the
+    rows past a sequence's last token in its last page -- holds NaN, so that a
+    kernel that reads one shows it.  Block-table entries past a sequence's last
+    page hold ``unused_entry`` (-1 by default: not a page).  ``shared_prefix``
+    maps a sequence b to (a, n) with a < b: b's block table starts with a's
+    first n pages (prefix sharing; both sequences must own them whole), and
+    b's tokens over those pages must equal a's (the caller arranges the inputs
+    so).
+    """
+    wl = x.wl
+    seq_lens = np.asarray(seq_lens, np.int32)
+    B = wl.B
+    assert seq_lens.shape == (B,) and np.all(seq_lens >= 1) and np.all(seq_lens <= wl.L)
+    need = [-(-int(n) // page_size) for n in seq_lens]
+    shared_prefix = dict(shared_prefix or {})
+    own = list(need)
+    for b, (a, n) in shared_prefix.items():
+        assert a < b and n * page_size <= min(int(seq_lens[a]), int(seq_lens[b]))
+        own[b] -= n
+    num_pages = sum(own) + spare_pages
+    order = np.random.default_rng([seed, TENSOR_ID["page_order"], 0]).permutation(num_pages)
+    max_pages = max(need)
+    table = np.full((B, max_pages), unused_entry, np.int32)
+    fill = nan_fill(wl.dtype)
+    c_pool = np.full((num_pages * page_size, wl.d_c), fill, x.c_kv.dtype)
+    k_pool = np.full((num_pages * page_size, wl.d_r), fill, x.k_r.dtype)
+    nxt = 0
+    for b in range(B):
+        first = 0
+        if b in shared_prefix:
+            a, first = shared_prefix[b]
+            table[b, :first] = table[a, :first]
+        for j in range(first, need[b]):
+            table[b, j] = order[nxt]
+            nxt += 1
+        L = int(seq_lens[b])
+        for j in range(first, need[b]):
+            t0, t1 = j * page_size, min(L, (j + 1) * page_size)
+            r0 = int(table[b, j]) * page_size
+            c_pool[r0:r0 + t1 - t0] = x.c_kv[b, t0:t1]
+            k_pool[r0:r0 + t1 - t0] = x.k_r[b, t0:t1]
+    return PagedCache(c_pool, k_pool, table, seq_lens, page_size)
