@@ -47,8 +47,10 @@ typedef enum {
     LCA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait inside a kernel ran out (see lca_get_device_error) */
     LCA_ERR_PLAN_MISMATCH = 6,   /* the plan was made for another shape / dtype / device */
     LCA_ERR_NO_MEMORY = 7,       /* device or host allocation failed */
-    LCA_ERR_DEVICE_CHECK = 8     /* debug build only: a kernel index failed its range check and the
+    LCA_ERR_DEVICE_CHECK = 8,    /* debug build only: a kernel index failed its range check and the
                                     access was skipped (see lca_get_device_error) */
+    LCA_ERR_DEVICE_INPUT = 9     /* lca_decode_paged: a length or block-table entry read on the
+                                    device was out of range (see lca_get_device_error) */
 } lca_status;
 
 typedef enum { LCA_F32 = 0, LCA_BF16 = 1 } lca_dtype;
@@ -250,8 +252,9 @@ const char *lca_status_string(lca_status status);
  * Returns LCA_OK, LCA_ERR_DEVICE_CHECK when (in the range-checked debug build,
  * liblca_checked.so) a kernel index failed its check, LCA_ERR_DEVICE_TIMEOUT
  * when an in-kernel wait ran out (the kernel then skipped its remaining work
- * and left outputs undefined), or LCA_ERR_CUDA when the synchronisation
- * itself failed.
+ * and left outputs undefined), LCA_ERR_DEVICE_INPUT when lca_decode_paged read
+ * a length or block-table entry out of range, or LCA_ERR_CUDA when the
+ * synchronisation itself failed.
  */
 lca_status lca_get_device_error(lca_plan *plan, void *stream);
 
@@ -278,6 +281,46 @@ lca_status lca_plan_set_timing_event(lca_plan *plan, void *event);
  * (16 heads per CTA), 3 = tcgen05 two-CTA (128 heads per cluster of two CTAs that split the
  * latent width; H a multiple of 128, g <= 64). */
 int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
+
+/*
+ * LCA decode of a paged, variable-length batch: the caches of the B sequences
+ * sit in pages of one pool, each sequence has its own length, and each is
+ * decoded exactly as lca_decode decodes a contiguous cache of that length --
+ * its own n_G(b) = floor((L_b - w) / g) groups (0 when L_b <= w) and its own
+ * window (section 2, "O Algoritmo LCA", steps 1-3).  The page has no paged
+ * layout: this is the serving form of the same step (several sequences of
+ * different lengths in one call, caches grown a page at a time, pages shared
+ * between sequences with a common prefix).
+ *   q_c, q_r     device [B][H][d_c], [B][H][d_r] (the plan's B, H, dtype)
+ *   c_pool       device [num_pages * page_size][d_c]; k_pool [.. ][d_r]
+ *   page_size    rows per page, a positive multiple of 64
+ *   block_table  device int32 [B][max_pages]: sequence b's token t is row
+ *                block_table[b max_pages + t / page_size] page_size + t % page_size
+ *                of the pools.  Entries past a sequence's last page are never read.
+ *   seq_lens     device int32 [B]: L_b, 1 <= L_b <= min(max_L, max_pages page_size)
+ *   out          device fp32 [B][H][d_c]
+ *   anchor       device int32 [B][H][anchor_stride], a_j of (b, h) at
+ *                (b H + h) anchor_stride + j for j < n_G(b); may be NULL only when no
+ *                length up to min(max_L, max_pages page_size) has a group
+ * Lengths and table entries stay on the device (no host synchronisation; the
+ * call can be captured in a CUDA graph).  A length outside its range, or with
+ * n_G(b) > anchor_stride, leaves that sequence's output NaN and its anchors
+ * unwritten; a used table entry outside [0, num_pages) is read as page 0.
+ * Either raises LCA_ERR_DEVICE_INPUT from the next lca_get_device_error.
+ * Pool rows that hold no token of a sequence may hold anything, NaN included.
+ * The kernels and their precision are lca_decode's for the plan's shape.
+ * Errors (synchronous): LCA_ERR_INVALID_ARG (null pointers, page_size not a
+ * positive multiple of 64, num_pages or max_pages < 1, g < 1, w < 0, a NULL
+ * anchor where groups are possible), LCA_ERR_UNSUPPORTED (num_pages page_size
+ * > 2^31 - 1, or no kernel), LCA_ERR_ALIGNMENT (q, pools, out, anchor not
+ * 16-byte aligned; table or lengths not 4-byte aligned), LCA_ERR_PLAN_MISMATCH,
+ * LCA_ERR_CUDA.
+ */
+lca_status lca_decode_paged(lca_plan *plan, const void *q_c, const void *q_r, const void *c_pool,
+                            const void *k_pool, int64_t num_pages, int page_size,
+                            const int32_t *block_table, int64_t max_pages, const int32_t *seq_lens,
+                            int g, int w, float *out, int32_t *anchor, int64_t anchor_stride,
+                            void *stream);
 
 /*
  * lca_decode without a plan and without any allocation.  The page has no

@@ -20,7 +20,8 @@ LCA_ERR_UNSUPPORTED = 2
 LCA_ERR_DEVICE_TIMEOUT = 5
 STATUS = {0: "LCA_OK", 1: "LCA_ERR_INVALID_ARG", 2: "LCA_ERR_UNSUPPORTED", 3: "LCA_ERR_ALIGNMENT",
           4: "LCA_ERR_CUDA", 5: "LCA_ERR_DEVICE_TIMEOUT", 6: "LCA_ERR_PLAN_MISMATCH",
-          7: "LCA_ERR_NO_MEMORY", 8: "LCA_ERR_DEVICE_CHECK"}
+          7: "LCA_ERR_NO_MEMORY", 8: "LCA_ERR_DEVICE_CHECK", 9: "LCA_ERR_DEVICE_INPUT"}
+LCA_ERR_DEVICE_INPUT = 9
 LCA_F32, LCA_BF16 = 0, 1
 OPT_FORCE_SIMT, OPT_NUM_CTAS, OPT_WAIT_TIMEOUT_NS, OPT_DEBUG_SKIP_LOAD, OPT_KERNEL = 1, 2, 3, 4, 5
 KERNEL_NAMES = {0: "none", 1: "simt", 2: "tcgen05", 3: "tcgen05_pair"}
@@ -30,7 +31,7 @@ EXPORTS = ["lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", 
            "lca_decode_host", "lca_num_groups", "lca_status_string", "lca_get_device_error",
            "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
            "lca_stored_rows", "lca_build_stored", "lca_decode_stored", "lca_slice_groups",
-           "lca_decode_partial", "lca_merge_partials", "lca_get_device_error_site"]
+           "lca_decode_partial", "lca_merge_partials", "lca_get_device_error_site", "lca_decode_paged"]
 
 
 class LcaError(RuntimeError):
@@ -77,10 +78,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lca_merge_partials.argtypes = [vp, i32, vp, vp, vp, vp]
     lib.lca_get_device_error_site.argtypes = [vp]
     lib.lca_get_device_error_site.restype = i32
+    lib.lca_decode_paged.argtypes = [vp, vp, vp, vp, vp, i64, i32, vp, i64, vp, i32, i32, vp, vp, i64, vp]
     for name in ("lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
                  "lca_decode_host", "lca_get_device_error", "lca_plan_kernel",
                  "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
-                 "lca_build_stored", "lca_decode_stored", "lca_decode_partial", "lca_merge_partials"):
+                 "lca_build_stored", "lca_decode_stored", "lca_decode_partial", "lca_merge_partials",
+                 "lca_decode_paged"):
         getattr(lib, name).restype = i32
     if path == LIB_PATH:
         _lib = lib
@@ -204,6 +207,17 @@ class Plan:
         """lca_merge_partials: out from n_parts stacked partials."""
         _check(self._lib.lca_merge_partials(self._h, n_parts, _ptr(part_mz), _ptr(part_o), _ptr(out),
                                             _stream_handle(stream)), "lca_merge_partials")
+
+    def decode_paged(self, q_c, q_r, c_pool, k_pool, page_size: int, block_table, seq_lens, g: int, w: int,
+                     out, anchor, stream=None) -> None:
+        """lca_decode_paged: pools [num_pages * page_size, d], block_table [B, max_pages] and
+        seq_lens [B] int32 CUDA tensors; anchor [B, H, anchor_stride] int32 or None."""
+        num_pages = c_pool.shape[0] // page_size
+        stride = 0 if anchor is None else anchor.shape[2]
+        _check(self._lib.lca_decode_paged(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_pool), _ptr(k_pool), num_pages,
+                                          page_size, _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
+                                          g, w, _ptr(out), _ptr(anchor), stride, _stream_handle(stream)),
+               "lca_decode_paged")
 
     def device_error(self, stream=None) -> int:
         return int(self._lib.lca_get_device_error(self._h, _stream_handle(stream)))

@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include "checks.cuh"
+#include "paged_kernel.cuh"
 #include "ptx.cuh"
 
 namespace lca {
@@ -24,11 +25,15 @@ struct CombineParams {
   //           partial of sequence b into slot b + c.
   //   mode 2: slots b, B + b, 2B + b, ... (n_split of them): partials stacked
   //           by part, merged across parts (lca_merge_partials)
+  //   mode 3: as mode 1 over sequences of their own lengths: U, G and the
+  //           first tile and tile count of each sequence from the paged
+  //           metadata (a sequence without tiles has no partial: NaN out)
   int mode;
   int n_split;
   int64_t tiles_per_seq;
   int64_t G;
   int wait_prior;        // 1: launched as a programmatic dependent of the producer grid
+  const int* meta;       // mode 3: the paged metadata
   float* out_mz;         // non-null: write the merged (M, Z) to out_mz [B][H][2] and the
                          // unnormalised sum O to out (a partial for a later merge)
   int64_t n_slots;       // slots readable in part_o / part_mz (range checks)
@@ -62,6 +67,17 @@ __global__ void __launch_bounds__(kCombineThreads) lca_combine_kernel(const Comb
     first = b;
     count = p.n_split;
     slot_step = p.B;
+  } else if (p.mode == 3) {
+    const int64_t U = p.meta[0], G = p.meta[1];
+    const int4 rec = meta_seq(p.meta)[b];
+    first = b;
+    count = 0;
+    if (rec.w > 0 && G > 0) {
+      const int64_t c0 = range_owner(rec.y, U, G);
+      const int64_t c1 = range_owner((int64_t)rec.y + rec.w - 1, U, G);
+      first = b + c0;
+      count = c1 - c0 + 1;
+    }
   } else {
     const int64_t U = (int64_t)p.B * p.tiles_per_seq;
     const int64_t c0 = range_owner((int64_t)b * p.tiles_per_seq, U, p.G);

@@ -15,6 +15,7 @@
 #include "checks.cuh"
 #include "combine_kernel.cuh"
 #include "condense_kernel.cuh"
+#include "paged_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "simt_kernel.cuh"
 #include "tc_kernel.cuh"
@@ -31,6 +32,7 @@ struct lca_plan {
   int64_t ws_slots;
   float* part_o;           // [ws_slots][H][d_c]
   float* part_mz;          // [ws_slots][H][2]
+  int* meta;               // paged-decode metadata, lca::meta_ints(B, ws_slots) ints
   int* err;                // [2]: flags, where
   int last_site;           // where of the last error lca_get_device_error reported
   // options
@@ -124,6 +126,37 @@ struct Slice {
   float* out_mz;
 };
 
+// A paged, variable-length batch (lca_decode_paged): the pools' pages, the
+// block table and the device lengths; cap bounds every length.
+struct Paged {
+  const int32_t* block_table;
+  int64_t max_pages;
+  int page_size;
+  int64_t num_pages;
+  const int32_t* seq_lens;
+  int64_t cap;
+  int64_t anchor_stride;
+  int g, w;     // the segmentation every sequence's n_G(b) follows
+};
+
+// The metadata of a paged call (lengths checked, tiles of kT tokens, G ranges)
+// into the plan's metadata buffer; stream-ordered before the decode kernel.
+lca_status launch_meta(const lca_plan* p, const Paged& pg, int kT, int64_t G, cudaStream_t stream) {
+  lca::MetaParams mp = {};
+  mp.seq_lens = pg.seq_lens;
+  mp.B = p->B;
+  mp.cap = pg.cap;
+  mp.g = pg.g;
+  mp.w = pg.w;
+  mp.anchor_stride = pg.anchor_stride;
+  mp.kT = kT;
+  mp.G = G;
+  mp.meta = p->meta;
+  mp.err = p->err;
+  lca::lca_paged_meta_kernel<<<1, lca::kMetaThreads, 0, stream>>>(mp);
+  return cudaGetLastError() == cudaSuccess ? LCA_OK : LCA_ERR_CUDA;
+}
+
 bool tc_group_ok(int64_t nG, int g, int gmax) { return nG == 0 || (is_pow2(g) && g <= gmax); }
 
 // The kernel for (n_G, g): the two-CTA tcgen05 kernel where H is a multiple of
@@ -171,21 +204,33 @@ lca_status launch_combine(const lca_plan* p, const lca::CombineParams& cp_in, cu
 
 lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                     const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
-                    cudaStream_t stream, const Slice& sl) {
+                    cudaStream_t stream, const Slice& sl, const Paged* pg = nullptr) {
   const int ge = nG > 0 ? g : 1;
   const int tile = ge * std::max(1, 256 / ge);
+  // a paged batch: every sequence is cut into the same number of splits of
+  // its own length (in the kernel); lengths are known only on the device
   int64_t split_len = ceil_div(L, simt_target_splits(p));
   split_len = ceil_div(split_len, ge) * ge;
-  const int64_t n_split = ceil_div(L, split_len);
+  const int64_t n_split = pg ? simt_target_splits(p) : ceil_div(L, split_len);
   if ((int64_t)p->B * n_split > p->ws_slots) return LCA_ERR_UNSUPPORTED;
-  lca::SimtParams sp;
+  if (pg) {
+    const lca_status st = launch_meta(p, *pg, 0, 0, stream);
+    if (st != LCA_OK) return st;
+  }
+  lca::SimtParams sp = {};
   sp.q_c = q_c; sp.q_r = q_r; sp.c_kv = c_kv; sp.k_r = k_r;
   sp.B = p->B; sp.H = p->H; sp.d_c = p->d_c; sp.d_r = p->d_r;
   sp.L = L; sp.g = ge; sp.nG = nG; sp.split_len = split_len; sp.tile = tile;
   sp.n_split = (int)n_split; sp.anchor = anchor; sp.part_o = p->part_o; sp.part_mz = p->part_mz;
   sp.bias_rows = p->bias_rows; sp.bias = p->bias; sp.win0 = sl.win0; sp.pos0 = sl.pos0;
   sp.ws_slots = p->ws_slots; sp.err = p->err;
-  const size_t smem = (size_t)(p->d_c + p->d_r + 4 * lca::kSimtTileMax + lca::kSimtWarps) * 4;
+  sp.anchor_stride = pg ? pg->anchor_stride : nG;
+  if (pg) {
+    sp.meta = p->meta; sp.block_table = pg->block_table; sp.max_pages = pg->max_pages;
+    sp.page_size = pg->page_size; sp.num_pages = pg->num_pages;
+  }
+  const size_t smem = (size_t)(p->d_c + p->d_r + 4 * lca::kSimtTileMax + lca::kSimtWarps) * 4 +
+                      (size_t)lca::kSimtTileMax * sizeof(int64_t);
   dim3 grid((unsigned)n_split, (unsigned)p->H, (unsigned)p->B);
   if (p->dt == LCA_F32)
     lca::lca_simt_kernel<float><<<grid, lca::kSimtThreads, smem, stream>>>(sp);
@@ -212,11 +257,11 @@ void device_flag_mark(std::atomic<uint64_t>& flags, int device) {
     flags.fetch_or(uint64_t(1) << device, std::memory_order_acq_rel);
 }
 
-template <int LOG2G>
+template <int LOG2G, bool kPaged>
 cudaError_t launch_tc(const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream, int device) {
   static std::atomic<uint64_t> configured{0};
   if (!device_flag_set(configured, device)) {
-    cudaError_t e = cudaFuncSetAttribute(lca::tc::lca_tc_kernel<LOG2G>,
+    cudaError_t e = cudaFuncSetAttribute(lca::tc::lca_tc_kernel<LOG2G, kPaged>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          lca::tc::kSmemAlloc);
     if (e != cudaSuccess) return e;
@@ -235,63 +280,82 @@ cudaError_t launch_tc(const lca::tc::TcParams& tp, unsigned grid, cudaStream_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, lca::tc::lca_tc_kernel<LOG2G>, tp);
+  return cudaLaunchKernelEx(&cfg, lca::tc::lca_tc_kernel<LOG2G, kPaged>, tp);
 }
 
-cudaError_t launch_tc_g(int g, const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream,
-                        int device) {
+template <bool kPaged>
+cudaError_t launch_tc_gp(int g, const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream,
+                         int device) {
   switch (g) {
-    case 1: return launch_tc<0>(tp, grid, stream, device);
-    case 2: return launch_tc<1>(tp, grid, stream, device);
-    case 4: return launch_tc<2>(tp, grid, stream, device);
-    case 8: return launch_tc<3>(tp, grid, stream, device);
-    case 16: return launch_tc<4>(tp, grid, stream, device);
-    case 32: return launch_tc<5>(tp, grid, stream, device);
-    case 64: return launch_tc<6>(tp, grid, stream, device);
-    case 128: return launch_tc<7>(tp, grid, stream, device);
+    case 1: return launch_tc<0, kPaged>(tp, grid, stream, device);
+    case 2: return launch_tc<1, kPaged>(tp, grid, stream, device);
+    case 4: return launch_tc<2, kPaged>(tp, grid, stream, device);
+    case 8: return launch_tc<3, kPaged>(tp, grid, stream, device);
+    case 16: return launch_tc<4, kPaged>(tp, grid, stream, device);
+    case 32: return launch_tc<5, kPaged>(tp, grid, stream, device);
+    case 64: return launch_tc<6, kPaged>(tp, grid, stream, device);
+    case 128: return launch_tc<7, kPaged>(tp, grid, stream, device);
   }
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_tc_g(int g, const lca::tc::TcParams& tp, unsigned grid, cudaStream_t stream,
+                        int device) {
+  return tp.meta ? launch_tc_gp<true>(g, tp, grid, stream, device) : launch_tc_gp<false>(g, tp, grid, stream, device);
+}
+
 lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                   const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
-                  cudaStream_t stream, const Slice& sl) {
+                  cudaStream_t stream, const Slice& sl, const Paged* pg = nullptr) {
   lca::tc::TcParams tp;
   std::memset(&tp, 0, sizeof(tp));
-  const uint64_t rows = (uint64_t)p->B * (uint64_t)L;
+  const uint64_t rows = pg ? (uint64_t)pg->num_pages * (uint64_t)pg->page_size : (uint64_t)p->B * (uint64_t)L;
   if (rows > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
   const uint64_t qrows = (uint64_t)p->B * (uint64_t)p->H;
-  if (!make_map(&tp.tm_c, c_kv, 512, rows, 128) || !make_map(&tp.tm_k, k_r, 64, rows, 128) ||
+  // a paged tile's two 64-token halves may sit in two pages: 64-row boxes
+  const uint32_t box = pg ? lca::tc::kT / 2 : lca::tc::kT;
+  if (!make_map(&tp.tm_c, c_kv, 512, rows, box) || !make_map(&tp.tm_k, k_r, 64, rows, box) ||
       !make_map(&tp.tm_qc, q_c, 512, qrows, 16) || !make_map(&tp.tm_qr, q_r, 64, qrows, 16))
     return LCA_ERR_CUDA;
   const int n_hb = p->H / lca::tc::kHC;
-  const int64_t tps = ceil_div(L, lca::tc::kT);
+  const int64_t tps = pg ? 0 : ceil_div(L, lca::tc::kT);
   const int64_t U = (int64_t)p->B * tps;
   const int ctas = p->num_ctas > 0 ? p->num_ctas : p->num_sms;
-  int64_t G = std::max<int64_t>(1, std::min<int64_t>(ctas / n_hb, U));
+  // a paged batch's tile count is known on the device only: it uses
+  // min(G, U) of these ranges (the metadata)
+  int64_t G = std::max<int64_t>(1, pg ? ctas / n_hb : std::min<int64_t>(ctas / n_hb, U));
   G = std::min<int64_t>(G, p->ws_slots - p->B + 1);    // range c writes slot b + c
   if (G < 1) return LCA_ERR_UNSUPPORTED;
+  if (pg) {
+    const lca_status st = launch_meta(p, *pg, lca::tc::kT, G, stream);
+    if (st != LCA_OK) return st;
+  }
   tp.B = p->B; tp.H = p->H; tp.L = L; tp.nG = nG;
-  tp.tiles_per_seq = tps; tp.U = U; tp.G = G; tp.n_hb = n_hb;
+  tp.tiles_per_seq = pg ? 1 : tps; tp.U = U; tp.G = G; tp.n_hb = n_hb;
   tp.anchor = anchor; tp.part_o = p->part_o; tp.part_mz = p->part_mz; tp.err = p->err;
   tp.timeout_ns = p->timeout_ns; tp.debug_skip_load = p->debug_skip_load;
   tp.bias_rows = p->bias_rows; tp.bias = p->bias; tp.win0 = sl.win0; tp.pos0 = sl.pos0;
   tp.ws_slots = p->ws_slots;
+  tp.anchor_stride = pg ? pg->anchor_stride : nG;
+  if (pg) {
+    tp.meta = p->meta; tp.block_table = pg->block_table; tp.max_pages = pg->max_pages;
+    tp.page_size = pg->page_size; tp.num_pages = pg->num_pages;
+  }
   const unsigned grid = (unsigned)(G * n_hb);
   if (launch_tc_g(nG > 0 ? g : 1, tp, grid, stream, p->device) != cudaSuccess) return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
   lca::CombineParams cp = {};
   cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;
-  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 1; cp.tiles_per_seq = tps; cp.G = G;
-  cp.wait_prior = 1; cp.out_mz = sl.out_mz;
+  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = pg ? 3 : 1; cp.tiles_per_seq = tps; cp.G = G;
+  cp.wait_prior = 1; cp.out_mz = sl.out_mz; cp.meta = p->meta;
   return launch_combine(p, cp, stream, true);
 }
 
-template <int LOG2G>
+template <int LOG2G, bool kPaged>
 cudaError_t launch_pair(const lca::pair::PairParams& pp, unsigned clusters, cudaStream_t stream, int device) {
   static std::atomic<uint64_t> configured{0};
   if (!device_flag_set(configured, device)) {
-    cudaError_t e = cudaFuncSetAttribute(lca::pair::lca_pair_kernel<LOG2G>,
+    cudaError_t e = cudaFuncSetAttribute(lca::pair::lca_pair_kernel<LOG2G, kPaged>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          lca::pair::kSmemAlloc);
     if (e != cudaSuccess) return e;
@@ -313,27 +377,34 @@ cudaError_t launch_pair(const lca::pair::PairParams& pp, unsigned clusters, cuda
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, lca::pair::lca_pair_kernel<LOG2G>, pp);
+  return cudaLaunchKernelEx(&cfg, lca::pair::lca_pair_kernel<LOG2G, kPaged>, pp);
+}
+
+template <bool kPaged>
+cudaError_t launch_pair_gp(int g, const lca::pair::PairParams& pp, unsigned clusters, cudaStream_t stream,
+                           int device) {
+  switch (g) {
+    case 1: return launch_pair<0, kPaged>(pp, clusters, stream, device);
+    case 2: return launch_pair<1, kPaged>(pp, clusters, stream, device);
+    case 4: return launch_pair<2, kPaged>(pp, clusters, stream, device);
+    case 8: return launch_pair<3, kPaged>(pp, clusters, stream, device);
+    case 16: return launch_pair<4, kPaged>(pp, clusters, stream, device);
+    case 32: return launch_pair<5, kPaged>(pp, clusters, stream, device);
+    case 64: return launch_pair<6, kPaged>(pp, clusters, stream, device);
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_pair_g(int g, const lca::pair::PairParams& pp, unsigned clusters, cudaStream_t stream,
                           int device) {
-  switch (g) {
-    case 1: return launch_pair<0>(pp, clusters, stream, device);
-    case 2: return launch_pair<1>(pp, clusters, stream, device);
-    case 4: return launch_pair<2>(pp, clusters, stream, device);
-    case 8: return launch_pair<3>(pp, clusters, stream, device);
-    case 16: return launch_pair<4>(pp, clusters, stream, device);
-    case 32: return launch_pair<5>(pp, clusters, stream, device);
-    case 64: return launch_pair<6>(pp, clusters, stream, device);
-  }
-  return cudaErrorInvalidValue;
+  return pp.meta ? launch_pair_gp<true>(g, pp, clusters, stream, device)
+                 : launch_pair_gp<false>(g, pp, clusters, stream, device);
 }
 
 // Two-CTA clusters of the pair kernel that fit on the device at once (one
 // wave); 0 when the query fails.
 int pair_cluster_capacity(int num_sms) {
-  cudaError_t e = cudaFuncSetAttribute(lca::pair::lca_pair_kernel<4>,
+  cudaError_t e = cudaFuncSetAttribute(lca::pair::lca_pair_kernel<4, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        lca::pair::kSmemAlloc);
   if (e != cudaSuccess) { cudaGetLastError(); return num_sms / 2; }
@@ -349,7 +420,7 @@ int pair_cluster_capacity(int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, lca::pair::lca_pair_kernel<4>, &cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, lca::pair::lca_pair_kernel<4, false>, &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     return num_sms / 2;
   }
@@ -358,10 +429,10 @@ int pair_cluster_capacity(int num_sms) {
 
 lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c_kv,
                     const void* k_r, int64_t L, int g, int64_t nG, float* out, int32_t* anchor,
-                    cudaStream_t stream, const Slice& sl) {
+                    cudaStream_t stream, const Slice& sl, const Paged* pg = nullptr) {
   lca::pair::PairParams pp;
   std::memset(&pp, 0, sizeof(pp));
-  const uint64_t rows = (uint64_t)p->B * (uint64_t)L;
+  const uint64_t rows = pg ? (uint64_t)pg->num_pages * (uint64_t)pg->page_size : (uint64_t)p->B * (uint64_t)L;
   if (rows > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
   const uint64_t qrows = (uint64_t)p->B * (uint64_t)p->H;
   if (!make_map(&pp.tm_c, c_kv, 512, rows, lca::pair::kT) ||
@@ -370,25 +441,36 @@ lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c
     return LCA_ERR_CUDA;
   pp.q_r = static_cast<const __nv_bfloat16*>(q_r);
   const int n_hb = p->H / lca::pair::kHeads;
-  const int64_t tps = ceil_div(L, lca::pair::kT);
+  const int64_t tps = pg ? 0 : ceil_div(L, lca::pair::kT);
   const int64_t U = (int64_t)p->B * tps;
   const int64_t clusters = p->num_ctas > 0 ? std::max(1, p->num_ctas / 2) : p->pair_clusters;
-  int64_t G = std::max<int64_t>(1, std::min<int64_t>(clusters / n_hb, U));
+  // a paged batch's tile count is known on the device only: it uses
+  // min(G, U) of these ranges (the metadata)
+  int64_t G = std::max<int64_t>(1, pg ? clusters / n_hb : std::min<int64_t>(clusters / n_hb, U));
   G = std::min<int64_t>(G, p->ws_slots - p->B + 1);    // range c writes slot b + c
   if (G < 1) return LCA_ERR_UNSUPPORTED;
+  if (pg) {
+    const lca_status st = launch_meta(p, *pg, lca::pair::kT, G, stream);
+    if (st != LCA_OK) return st;
+  }
   pp.B = p->B; pp.H = p->H; pp.L = L; pp.nG = nG;
-  pp.tiles_per_seq = tps; pp.U = U; pp.G = G; pp.n_hb = n_hb;
+  pp.tiles_per_seq = pg ? 1 : tps; pp.U = U; pp.G = G; pp.n_hb = n_hb;
   pp.anchor = anchor; pp.part_o = p->part_o; pp.part_mz = p->part_mz; pp.err = p->err;
   pp.timeout_ns = p->timeout_ns; pp.debug_skip_load = p->debug_skip_load;
   pp.bias_rows = p->bias_rows; pp.bias = p->bias; pp.win0 = sl.win0; pp.pos0 = sl.pos0;
   pp.ws_slots = p->ws_slots;
+  pp.anchor_stride = pg ? pg->anchor_stride : nG;
+  if (pg) {
+    pp.meta = p->meta; pp.block_table = pg->block_table; pp.max_pages = pg->max_pages;
+    pp.page_size = pg->page_size; pp.num_pages = pg->num_pages;
+  }
   if (launch_pair_g(nG > 0 ? g : 1, pp, (unsigned)(G * n_hb), stream, p->device) != cudaSuccess)
     return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
   lca::CombineParams cp = {};
   cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;
-  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 1; cp.tiles_per_seq = tps; cp.G = G;
-  cp.wait_prior = 1; cp.out_mz = sl.out_mz;
+  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = pg ? 3 : 1; cp.tiles_per_seq = tps; cp.G = G;
+  cp.wait_prior = 1; cp.out_mz = sl.out_mz; cp.meta = p->meta;
   return launch_combine(p, cp, stream, true);
 }
 
@@ -490,6 +572,7 @@ const char* lca_status_string(lca_status s) {
     case LCA_ERR_PLAN_MISMATCH: return "plan made for another shape or device";
     case LCA_ERR_NO_MEMORY: return "out of memory";
     case LCA_ERR_DEVICE_CHECK: return "a kernel index failed its range check (debug build)";
+    case LCA_ERR_DEVICE_INPUT: return "a sequence length or block-table entry on the device was out of range";
   }
   return "unknown status";
 }
@@ -520,11 +603,13 @@ lca_status lca_plan_create(int B, int H, int d_c, int d_r, lca_dtype dt, int64_t
   p->ws_slots = std::max(simt_slots, tc_slots);
   const size_t o_bytes = (size_t)p->ws_slots * H * d_c * sizeof(float);
   const size_t mz_bytes = (size_t)p->ws_slots * H * 2 * sizeof(float);
+  const size_t meta_bytes = (size_t)lca::meta_ints(B, p->ws_slots) * sizeof(int);
   if (cudaMalloc(&p->part_o, o_bytes) != cudaSuccess ||
       cudaMalloc(&p->part_mz, mz_bytes) != cudaSuccess ||
+      cudaMalloc(&p->meta, meta_bytes) != cudaSuccess ||
       cudaMalloc(&p->err, 2 * sizeof(int)) != cudaSuccess ||
       cudaMemset(p->err, 0, 2 * sizeof(int)) != cudaSuccess) {
-    cudaFree(p->part_o); cudaFree(p->part_mz); cudaFree(p->err);
+    cudaFree(p->part_o); cudaFree(p->part_mz); cudaFree(p->meta); cudaFree(p->err);
     cudaGetLastError();
     delete p;
     return LCA_ERR_NO_MEMORY;
@@ -535,7 +620,7 @@ lca_status lca_plan_create(int B, int H, int d_c, int d_r, lca_dtype dt, int64_t
 
 lca_status lca_plan_destroy(lca_plan* p) {
   if (!p) return LCA_OK;
-  cudaFree(p->part_o); cudaFree(p->part_mz); cudaFree(p->err);
+  cudaFree(p->part_o); cudaFree(p->part_mz); cudaFree(p->meta); cudaFree(p->err);
   free_staging(p);
   delete p;
   return LCA_OK;
@@ -744,10 +829,46 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
   if (host[0] != 0 && cudaMemset(p->err, 0, sizeof(host)) != cudaSuccess) return LCA_ERR_CUDA;
   if (host[0] != 0) p->last_site = host[1];
   if (host[0] & lca::kErrCheck) return LCA_ERR_DEVICE_CHECK;
+  if (host[0] & lca::kErrInput) return LCA_ERR_DEVICE_INPUT;
   return host[0] != 0 ? LCA_ERR_DEVICE_TIMEOUT : LCA_OK;
 }
 
 int lca_get_device_error_site(const lca_plan* p) { return p ? p->last_site : 0; }
+
+lca_status lca_decode_paged(lca_plan* p, const void* q_c, const void* q_r, const void* c_pool,
+                            const void* k_pool, int64_t num_pages, int page_size,
+                            const int32_t* block_table, int64_t max_pages, const int32_t* seq_lens,
+                            int g, int w, float* out, int32_t* anchor, int64_t anchor_stride,
+                            void* stream) {
+  if (!p || !q_c || !q_r || !c_pool || !k_pool || !block_table || !seq_lens || !out)
+    return LCA_ERR_INVALID_ARG;
+  if (num_pages < 1 || page_size < 64 || (page_size % 64) != 0 || max_pages < 1 || g < 1 || w < 0 ||
+      anchor_stride < 0)
+    return LCA_ERR_INVALID_ARG;
+  if ((uint64_t)num_pages * (uint64_t)page_size > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
+  if (dev != p->device) return LCA_ERR_PLAN_MISMATCH;
+  Paged pg;
+  pg.block_table = block_table; pg.max_pages = max_pages; pg.page_size = page_size;
+  pg.num_pages = num_pages; pg.seq_lens = seq_lens; pg.g = g; pg.w = w;
+  pg.cap = std::min<int64_t>(p->max_L, max_pages * (int64_t)page_size);
+  const int64_t nG_cap = lca_num_groups(pg.cap, g, w);
+  if (nG_cap > 0 && !anchor) return LCA_ERR_INVALID_ARG;
+  pg.anchor_stride = anchor ? anchor_stride : INT64_MAX;
+  const Kernel k = choose(p, nG_cap, g);
+  if (k == kNone) return LCA_ERR_UNSUPPORTED;
+  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(c_pool) || !aligned16(k_pool) || !aligned16(out) ||
+      (anchor && !aligned16(anchor)) || (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0)
+    return LCA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Slice whole = {0, 0, nullptr};
+  const int ge = nG_cap > 0 ? g : 1;
+  if (k == kPair) return run_pair(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+  if (k == kTc) return run_tc(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+  return run_simt(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+}
 
 // For callers that may not allocate device memory when they decode -- a
 // server whose memory is all reserved up front by its own pool (a cudaMalloc

@@ -63,6 +63,7 @@
 #include <type_traits>
 
 #include "checks.cuh"
+#include "paged_kernel.cuh"
 #include "ptx.cuh"
 
 namespace lca {
@@ -144,6 +145,17 @@ struct PairParams {
   int64_t pos0;        // position of row 0 in the context (a slice's offset): anchors are
                        // written as pos0 + row, and groups start at rows that are multiples of g
   int64_t ws_slots;    // slots of part_o / part_mz (range checks)
+  int64_t anchor_stride;   // anchors of (b, h) start at (b H + h) anchor_stride
+  // Paged, variable-length decode (meta != null): tm_c / tm_k cover the pools,
+  // [num_pages * page_size rows]; sequence b's token t is row
+  // block_table[b max_pages + t / page_size] page_size + t % page_size, and its
+  // length, groups, tiles and the ranges come from the metadata (L, nG, U, G,
+  // tiles_per_seq, win0 above are then unused; page_size is a multiple of 64).
+  const int* meta;
+  const int32_t* block_table;
+  int64_t max_pages;
+  int page_size;
+  int64_t num_pages;
 };
 
 struct Bars {
@@ -287,7 +299,7 @@ __device__ __forceinline__ void group_stats(const float* x, const float* sr, flo
   }
 }
 
-template <int LOG2G>
+template <int LOG2G, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_constant__ PairParams p) {
   constexpr int g = 1 << LOG2G;
   static_assert(g <= kT, "a group must fit in one tile");
@@ -338,17 +350,42 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   const int hb = (int)(cl % p.n_hb);
   const int64_t c = cl / p.n_hb;
   const int h0 = hb * kHeads;
-  const int64_t u0 = c * p.U / p.G;
-  const int64_t u1 = (c + 1) * p.U / p.G;
-  const int64_t n_tiles = u1 - u0;
-  const int64_t win0 = p.win0;
-  const int64_t seq0 = u0 / p.tiles_per_seq;
-  const int64_t tile0 = u0 - seq0 * p.tiles_per_seq;
-  auto step = [&](int64_t& seq, int64_t& tile) {
-    if (++tile == p.tiles_per_seq) { tile = 0; ++seq; }
+  constexpr bool paged = kPaged;   // a separate instantiation: the contiguous loops stay as they were
+  // The cluster's range of tiles, for sequences of tiles_per_seq tiles each; a
+  // paged batch takes its range from the metadata once the previous kernel in
+  // the stream is done (below).
+  int64_t u0 = c * p.U / p.G;
+  int64_t n_tiles = (c + 1) * p.U / p.G - u0;
+  int64_t seq0 = u0 / p.tiles_per_seq;
+  int64_t tile0 = u0 - seq0 * p.tiles_per_seq;
+  auto seq_tiles = [&](int64_t b) -> int64_t {
+    if constexpr (kPaged) return (int64_t)meta_seq(p.meta)[b].w;
+    else return p.tiles_per_seq;
   };
-  auto last_of_part = [&](int64_t i, int64_t tile) {
-    return i + 1 == n_tiles || tile + 1 == p.tiles_per_seq;
+  // the next (sequence, tile) of the range; a paged batch's sequences without
+  // tiles are passed over (tps: tiles of the current sequence)
+  auto step = [&](int64_t& seq, int64_t& tile, int64_t& tps) {
+    if constexpr (kPaged) {
+      if (++tile == tps) {
+        tile = 0;
+        do {
+          ++seq;
+          tps = seq < p.B ? seq_tiles(seq) : 1;
+        } while (tps == 0);
+      }
+    } else {
+      if (++tile == p.tiles_per_seq) { tile = 0; ++seq; }
+    }
+  };
+  auto last_of_part = [&](int64_t i, int64_t tile, int64_t tps) {
+    if constexpr (kPaged) return i + 1 == n_tiles || tile + 1 == tps;
+    else return i + 1 == n_tiles || tile + 1 == p.tiles_per_seq;
+  };
+  // first row of a tile's 64 tokens in the C_KV / K_R tensor maps
+  auto tile_row = [&](int64_t b, int64_t tile) -> int32_t {
+    if constexpr (!kPaged) return (int32_t)(b * p.L + tile * kT);
+    else return (int32_t)paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b, tile * kT, p.err,
+                                   0xA03);
   };
 
   if (tid == 0) {
@@ -400,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   // Programmatic dependent launch: nothing below touches global memory before
   // the previous kernel in the stream has completed; its first tile and query
   // block are only prefetched into L2 (no data reaches this CTA).
-  if (tid == 0) {
+  if (tid == 0 && !paged) {
     const int32_t frow = (int32_t)(seq0 * p.L + tile0 * kT);
     for (int a = 0; a < kAtoms; ++a) ptx::tma_prefetch_l2_2d(&p.tm_c, kDim * r + 64 * a, frow);
     ptx::tma_prefetch_l2_2d(&p.tm_k, 0, frow);
@@ -409,6 +446,21 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   }
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
+  if constexpr (kPaged) {
+    const int64_t U = p.meta[0], Ge = p.meta[1];
+    u0 = 0;
+    n_tiles = 0;
+    seq0 = 0;
+    tile0 = 0;
+    if (c < Ge) {
+      u0 = c * U / Ge;
+      n_tiles = (c + 1) * U / Ge - u0;
+      const int2 rg = meta_range(p.meta, p.B)[c];
+      seq0 = rg.x;
+      tile0 = rg.y;
+    }
+  }
+  const int64_t tps0 = n_tiles > 0 ? seq_tiles(seq0) : 1;
 
   if (warp == 0 && lane == 0) {
     // ===================================================== TMA producer
@@ -426,8 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     int issued_q = -1, seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
-    int64_t pseq = seq0, ptile = tile0;
-    for (int64_t i = 0; i < n_tiles && ok; ++i, step(pseq, ptile)) {
+    int64_t pseq = seq0, ptile = tile0, ptps = tps0;
+    // each tile's row is looked up a tile ahead (a paged batch reads its block
+    // table), so that the lookup's latency passes during the waits
+    int32_t row_next = (kPaged && n_tiles > 0) ? tile_row(pseq, ptile) : 0;
+    for (int64_t i = 0; i < n_tiles && ok; ++i) {
       const int64_t b = pseq;
       if (b != cur_b) {
         cur_b = b;
@@ -440,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           ptx::tma_load_2d(smem + kOffQc + a * kQcAtom, &p.tm_qc, kDim * r + 64 * a, qrow, bb.q_full);
         issued_q = seg;
       }
-      const int32_t row = (int32_t)(b * p.L + ptile * kT);
+      const int32_t row = kPaged ? row_next : tile_row(b, ptile);
       {
         const int ks = (int)(i % kNKr);
         const int kk = (int)(i / kNKr);
@@ -458,7 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         const int ck = (int)(i / kNS);
         if (ck >= 1) ok = bounded_wait(&bb.c_empty[cs], (ck - 1) & 1, abort_flag, p, 0x502, true);
         if (!ok) break;
-        if (!LCA_CHECK(p.err, cs < kNS && (int64_t)row < (int64_t)p.B * p.L, 0xE01)) { ok = false; break; }
+        if (!LCA_CHECK(p.err, cs < kNS && (int64_t)row < (paged ? p.num_pages * p.page_size : (int64_t)p.B * p.L),
+                       0xE01)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bb.c_full[cs], kStage);
         uint8_t* dst = smem + kOffC + cs * kStage;
         for (int a = 0; a < kAtoms; ++a)
@@ -466,6 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
 #pragma unroll
         for (int q = 0; q < kNS; ++q) if (q == cs) issued_c[q] = ck;
       }
+      step(pseq, ptile, ptps);
+      if (kPaged && i + 1 < n_tiles) row_next = tile_row(pseq, ptile);
     }
     // Let every copy this thread started land before the CTA can exit.
 #pragma unroll
@@ -488,10 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
-    int64_t sseq = seq0, stile = tile0;
-    for (int64_t t = 0; t < n_tiles && ok; ++t, step(sseq, stile)) {
+    int64_t sseq = seq0, stile = tile0, stps = tps0;
+    for (int64_t t = 0; t < n_tiles && ok; ++t, step(sseq, stile, stps)) {
       const int64_t b = sseq;
-      const bool last_in_seg = last_of_part(t, stile);
+      const bool last_in_seg = last_of_part(t, stile, stps);
       const int buf = (int)(t & 1);
       bool new_seg = false;
       if (b != cur_b) {
@@ -550,8 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     const uint64_t d_p = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_cb = ptx::smem_desc(ptx::smem_u32(smem + kOffC), kCAtom, 1024, ptx::kSwizzle128B);
     int n_resc = 0;
-    int64_t oseq = seq0, otile = tile0;
-    for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile)) {
+    int64_t oseq = seq0, otile = tile0, otps = tps0;
+    for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile, otps)) {
       const int buf = (int)(j & 1);
       if (!bounded_wait(bb.p_local, (uint32_t)j & 1, abort_flag, p, 0x700, true)) break;
       bool ok = true;
@@ -594,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
                          k > 0 ? 1u : acc0);
       ptx::mma_commit(&bb.c_empty[cs]);
       ptx::mma_commit_multicast(&bb.p_free[2 * r + buf], (uint16_t)0x3);
-      if (last_of_part(j, otile)) ptx::mma_commit(bb.part_done);
+      if (last_of_part(j, otile, otps)) ptx::mma_commit(bb.part_done);
     }
     ptx::mma_commit(&bb.drain[1]);
     bounded_wait(&bb.drain[1], 0, abort_flag, p, 0x7F0, false);
@@ -638,12 +696,27 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       return true;
     };
     float M = -INFINITY, Z = 0.f;
-    int64_t cseq = seq0, ctile = tile0;
+    int64_t cseq = seq0, ctile = tile0, ctps = tps0;
+    // the current sequence's length, groups and first window token
+    int64_t sL = 0, snG = 0, swin0 = 0, s_of = -1;
     int seg = 0;
     int64_t i = 0;
     bool ok = n_tiles > 0 ? load_qr(seq0, 0) : true;
-    for (; i < n_tiles && ok; ++i, step(cseq, ctile)) {
+    for (; i < n_tiles && ok; ++i, step(cseq, ctile, ctps)) {
       const int64_t b = cseq, tile = ctile;
+      if constexpr (kPaged) {
+        if (b != s_of) {
+          s_of = b;
+          const int4 rec = meta_seq(p.meta)[b];
+          sL = rec.x;
+          snG = rec.z;
+          swin0 = snG * g;
+        }
+      } else {
+        sL = p.L;
+        snG = p.nG;
+        swin0 = p.win0;
+      }
       const int buf = (int)(i & 1);
       if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x800)) break;
       if (!warp_wait(&bb.recv_full[q], (uint32_t)i & 1, abort_flag, p, 0x801)) break;
@@ -675,13 +748,16 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ptx::mbar_arrive_remote(peer_recv_free);
       }
       // the next sequence's q_r, for the sr MMA of the tile after this one
-      if (last_of_part(i, tile) && i + 1 < n_tiles) {
+      if (last_of_part(i, tile, ctps) && i + 1 < n_tiles) {
         ++seg;
-        if (!load_qr(b + 1, seg)) break;
+        int64_t nb = b + 1;
+        if constexpr (kPaged)
+          while (nb + 1 < p.B && seq_tiles(nb) == 0) ++nb;
+        if (!load_qr(nb, seg)) break;
       }
 
       const int64_t tok0 = tile * kT + kHalfT * k;
-      int32_t* anc = p.anchor + ((int64_t)b * p.H + h) * p.nG;
+      int32_t* anc = p.anchor + ((int64_t)b * p.H + h) * p.anchor_stride;
       const bool first = i == 0 || tile == 0;
       float alpha = 1.f;
       uint32_t pk[kHalfT / 2];
@@ -695,16 +771,16 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         // multiple of g, which may fall inside the thread's 32 tokens, so the
         // choice is made per group (grp[]).  For g = 64 a group is the whole
         // tile, and the choice is the same for both threads of a head.
-        const bool half_groups = kFast || ((g > 1) && (tok0 < win0));
+        const bool half_groups = kFast || ((g > 1) && (tok0 < swin0));
         bool grp[NGT];
 #pragma unroll
-        for (int gi = 0; gi < NGT; ++gi) grp[gi] = kFast || (half_groups && (tok0 + gi * GW < win0));
+        for (int gi = 0; gi < NGT; ++gi) grp[gi] = kFast || (half_groups && (tok0 + gi * GW < swin0));
 
         float f[NGT], Sg[NGT], deng[NGT], own_den[NGT], ent = -INFINITY;
         if constexpr (!kFast && g == 1) {
 #pragma unroll
           for (int t = 0; t < kHalfT; ++t)
-            if (tok0 + t < win0 && LCA_CHECK(p.err, tok0 + t < p.nG, 0xE05))
+            if (tok0 + t < swin0 && LCA_CHECK(p.err, tok0 + t < snG, 0xE05))
               anc[tok0 + t] = (int32_t)(p.pos0 + tok0 + t);
         }
         if (half_groups) {
@@ -749,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
 #pragma unroll
             for (int gi = 0; gi < NGT; ++gi) {
               const int64_t jg = (tile * kT + (g <= kHalfT ? kHalfT * k + gi * GW : 0)) / g;
-              if (grp[gi] && LCA_CHECK(p.err, jg >= 0 && jg < p.nG && ag[gi] >= 0 && ag[gi] < kT, 0xE04))
+              if (grp[gi] && LCA_CHECK(p.err, jg >= 0 && jg < snG && ag[gi] >= 0 && ag[gi] < kT, 0xE04))
                 anc[jg] = (int32_t)(p.pos0 + tile * kT + ag[gi]);
             }
           }
@@ -760,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
 #pragma unroll
                 for (int t = 0; t < GW; ++t) {
                   s[gi * GW + t] = x[gi * GW + t] + sr[gi * GW + t];
-                  if (tok0 + gi * GW + t < p.L) ent = fmaxf(ent, s[gi * GW + t]);
+                  if (tok0 + gi * GW + t < sL) ent = fmaxf(ent, s[gi * GW + t]);
                 }
               }
             }
@@ -769,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
 #pragma unroll
           for (int t = 0; t < kHalfT; ++t) {
             s[t] = x[t] + sr[t] + (tok0 + t < p.bias_rows ? p.bias : 0.f);
-            if (tok0 + t < p.L) ent = fmaxf(ent, s[t]);
+            if (tok0 + t < sL) ent = fmaxf(ent, s[t]);
           }
         }
 
@@ -822,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
               if (grp[t / GW]) {
                 v = s[t] * f[t / GW];
               } else {
-                v = tok0 + t < p.L ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
+                v = tok0 + t < sL ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
                 Z += v;
               }
               pv[e2] = v;
@@ -831,7 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           }
         }
       };
-      const bool fast = g > 1 && (tile + 1) * kT <= win0;   // warp-uniform
+      const bool fast = g > 1 && (tile + 1) * kT <= swin0;   // warp-uniform
       if (fast) tile_math(std::true_type{});
       else tile_math(std::false_type{});
       if (*abort_flag) break;
@@ -855,6 +931,20 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
+      }
+      // A paged sequence's last tile: its stage rows past the last token hold
+      // whatever the pool has there.  Their weights are 0, but 0 x NaN is not,
+      // so the four softmax warps clear those rows before O reads the stage
+      // (the score MMAs are done with it; the fence below orders the stores).
+      if (kPaged && (tile + 1) * kT > sL) {
+        const int n_valid = (int)(sL - tile * kT);
+        uint8_t* st = smem + kOffC + (int)(i % kNS) * kStage;
+        for (int idx = (warp - 3) * 32 + lane; idx < kAtoms * kT * 8; idx += 128) {
+          const int row = (idx >> 3) & (kT - 1);   // 8 chunks of 16 bytes a row, in every atom
+          if (row >= n_valid)
+            *reinterpret_cast<uint4*>(st + (idx >> 9) * kCAtom + row * 128 + (idx & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       // ---- this head's P row and factor into this CTA's P buffer (free once
       // its O of tile i - 2 is done; the previous copy out of it has read it)
@@ -890,7 +980,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ptx::mbar_arrive(bb.p_local);
       }
 
-      if (last_of_part(i, tile)) {
+      if (last_of_part(i, tile, ctps)) {
         // the partial of the range's part of sequence b: this head's O row over
         // this CTA's dims, and (owner) its (M, Z).  O of tile i is done when
         // buffer i & 1 is released (this warp saw its previous release above).
@@ -960,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       return true;
     };
     // what O of tile j needed of these heads' rows, done after O of tile j
-    auto behind = [&](int64_t j, int64_t b, int64_t tile) -> bool {
+    auto behind = [&](int64_t j, int64_t b, int64_t tile, int64_t tps) -> bool {
       if (!warp_wait(&bb.dec[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x902)) return false;
       if (dec_flag[j & 1]) {
         // every O before tile j is done (one phase per request, seen in order)
@@ -983,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bb.resc_done);
       }
-      if (last_of_part(j, tile)) {
+      if (last_of_part(j, tile, tps)) {
         const int64_t slot = b + c;
         if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xE08)) return false;
         // the last O of the part is done (one phase per part, seen in order)
@@ -1005,19 +1095,19 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       return true;
     };
     bool ok = n_tiles > 0 ? ship(0) : true;
-    int64_t bseq = seq0, btile = tile0;          // (sequence, tile) of tile i - 1
+    int64_t bseq = seq0, btile = tile0, btps = tps0;   // (sequence, tile) of tile i - 1
     int64_t i = 0;
     for (; i < n_tiles && ok; ++i) {
       if (i + 1 < n_tiles && !(ok = ship(i + 1))) break;
       if (i >= 1) {
-        if (!(ok = behind(i - 1, bseq, btile))) break;
-        step(bseq, btile);
+        if (!(ok = behind(i - 1, bseq, btile, btps))) break;
+        step(bseq, btile, btps);
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bb.lanes_ready);
     }
     if (ok && i == n_tiles && n_tiles > 0) {
-      behind(n_tiles - 1, bseq, btile);
+      behind(n_tiles - 1, bseq, btile, btps);
       // the peer's release of the last partial scores has landed here before this CTA exits
       if (lane == 0)
         bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true);

@@ -19,6 +19,7 @@
 #include <cstdint>
 
 #include "checks.cuh"
+#include "paged_kernel.cuh"
 
 namespace lca {
 
@@ -57,6 +58,15 @@ struct SimtParams {
   int64_t pos0;      // position of row 0 in the context: anchors are written as pos0 + row
   int64_t ws_slots;  // slots of part_o / part_mz (range checks)
   int* err;          // device error word (range checks)
+  int64_t anchor_stride;     // anchors of (b, h) start at (b H + h) anchor_stride
+  // paged, variable-length decode (meta != null): c_kv / k_r are the pools,
+  // sequence b has meta_seq(meta)[b].x tokens, token t in row
+  // block_table[b max_pages + t / page_size] page_size + t % page_size
+  const int* meta;
+  const int32_t* block_table;
+  int64_t max_pages;
+  int page_size;
+  int64_t num_pages;
 };
 
 constexpr int kSimtTileMax = 1024;
@@ -99,17 +109,28 @@ lca_simt_kernel(const SimtParams p) {
   float* pw = sr + kSimtTileMax;       // [tile] per-token attention weight
   float* glog = pw + kSimtTileMax;     // [tile] condensed logit of the group starting here
   float* red = glog + kSimtTileMax;    // [kSimtWarps]
+  int64_t* rowix = reinterpret_cast<int64_t*>(red + kSimtWarps);   // [tile] pool row (paged)
 
   const T* qc_g = static_cast<const T*>(p.q_c) + ((int64_t)b * p.H + h) * p.d_c;
   const T* qr_g = static_cast<const T*>(p.q_r) + ((int64_t)b * p.H + h) * p.d_r;
-  const T* c_g = static_cast<const T*>(p.c_kv) + (int64_t)b * p.L * p.d_c;
-  const T* k_g = static_cast<const T*>(p.k_r) + (int64_t)b * p.L * p.d_r;
+  const bool paged = p.meta != nullptr;
+  const T* c_g = static_cast<const T*>(p.c_kv) + (paged ? 0 : (int64_t)b * p.L * p.d_c);
+  const T* k_g = static_cast<const T*>(p.k_r) + (paged ? 0 : (int64_t)b * p.L * p.d_r);
   for (int i = tid; i < p.d_c; i += kSimtThreads) qc[i] = load_elem(qc_g + i);
   for (int i = tid; i < p.d_r; i += kSimtThreads) qr[i] = load_elem(qr_g + i);
 
-  const int64_t win0 = p.win0;      // first uncompressed (window) token
-  const int64_t s0 = (int64_t)split * p.split_len;
-  const int64_t s1 = (p.L < s0 + p.split_len) ? p.L : s0 + p.split_len;
+  // this sequence's length, groups and split (paged: its own, from the metadata)
+  int64_t L = p.L, nG = p.nG, win0 = p.win0, split_len = p.split_len;
+  if (paged) {
+    const int4 rec = meta_seq(p.meta)[b];
+    L = rec.x;
+    nG = rec.z;
+    win0 = nG * p.g;
+    split_len = (L + p.n_split - 1) / p.n_split;
+    split_len = (split_len + p.g - 1) / p.g * p.g;
+  }
+  const int64_t s0 = (int64_t)split * split_len;
+  const int64_t s1 = (L < s0 + split_len) ? L : s0 + split_len;
 
   constexpr int kDPerThread = kSimtMaxDc / kSimtThreads;
   float o[kDPerThread];
@@ -120,10 +141,17 @@ lca_simt_kernel(const SimtParams p) {
 
   for (int64_t t0 = s0; t0 < s1; t0 += p.tile) {
     const int n = (int)((int64_t)p.tile < s1 - t0 ? (int64_t)p.tile : s1 - t0);
+    // ---- the rows of this tile's tokens
+    for (int tt = tid; tt < n; tt += kSimtThreads)
+      if (LCA_CHECK(p.err, tt < kSimtTileMax, 0xC05))
+        rowix[tt] = paged ? paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b, t0 + tt,
+                                      p.err, 0xA02)
+                          : t0 + tt;
+    __syncthreads();
     // ---- scores, one warp per token
     for (int tt = warp; tt < n; tt += kSimtWarps) {
-      const T* crow = c_g + (t0 + tt) * p.d_c;
-      const T* krow = k_g + (t0 + tt) * p.d_r;
+      const T* crow = c_g + rowix[tt] * p.d_c;
+      const T* krow = k_g + rowix[tt] * p.d_r;
       float a = 0.f, r = 0.f;
       for (int d = lane; d < p.d_c; d += 32) a = fmaf(qc[d], load_elem(crow + d), a);
       for (int d = lane; d < p.d_r; d += 32) r = fmaf(qr[d], load_elem(krow + d), r);
@@ -152,8 +180,8 @@ lca_simt_kernel(const SimtParams p) {
         glog[tt] = num / den + sr[amax];
         const float inv = 1.f / den;
         for (int u = tt; u < tt + p.g; ++u) pw[u] = expf(sc[u] + sr[u] - m) * inv;  // w_t
-        if (LCA_CHECK(p.err, t / p.g < p.nG, 0xC03))
-          p.anchor[((int64_t)b * p.H + h) * p.nG + t / p.g] = (int32_t)(p.pos0 + t0 + amax);
+        if (LCA_CHECK(p.err, t / p.g < nG, 0xC03))
+          p.anchor[((int64_t)b * p.H + h) * p.anchor_stride + t / p.g] = (int32_t)(p.pos0 + t0 + amax);
       }
     }
     __syncthreads();
@@ -192,7 +220,7 @@ lca_simt_kernel(const SimtParams p) {
     for (int k = 0; k < kDPerThread; ++k) o[k] *= alpha;
     for (int tt = 0; tt < n; ++tt) {
       const float w = pw[tt];
-      const T* crow = c_g + (t0 + tt) * p.d_c;
+      const T* crow = c_g + rowix[tt] * p.d_c;
 #pragma unroll
       for (int k = 0; k < kDPerThread; ++k) {
         const int d = tid + k * kSimtThreads;

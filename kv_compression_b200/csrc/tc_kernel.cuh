@@ -48,6 +48,7 @@
 #include <cstdint>
 
 #include "checks.cuh"
+#include "paged_kernel.cuh"
 #include "ptx.cuh"
 
 namespace lca {
@@ -127,6 +128,18 @@ struct TcParams {
   int64_t pos0;        // position of row 0 in the context (a slice's offset): anchors are
                        // written as pos0 + row, and groups start at rows that are multiples of g
   int64_t ws_slots;    // slots of part_o / part_mz (range checks)
+  int64_t anchor_stride;   // anchors of (b, h) start at (b H + h) anchor_stride
+  // Paged, variable-length decode (meta != null): tm_c / tm_k cover the pools
+  // with a 64-row box, and a tile's two 64-token halves are loaded from their
+  // own pages; sequence b's token t is row
+  // block_table[b max_pages + t / page_size] page_size + t % page_size, and its
+  // length, groups, tiles and the ranges come from the metadata (L, nG, U, G,
+  // tiles_per_seq, win0 above are then unused; page_size is a multiple of 64).
+  const int* meta;
+  const int32_t* block_table;
+  int64_t max_pages;
+  int page_size;
+  int64_t num_pages;
 };
 
 struct Bars {
@@ -243,7 +256,7 @@ __device__ __forceinline__ void group_stats(const float (&s)[kHH], const float (
   for (int h = 0; h < kHH; ++h) sra[h] = __shfl_sync(0xffffffffu, sr[h], a[h]);
 }
 
-template <int LOG2G>
+template <int LOG2G, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr int g = 1 << LOG2G;
   static_assert(g <= kT, "a group must fit in one tile");
@@ -275,16 +288,51 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   const int hb = blockIdx.x % p.n_hb;
   const int64_t c = blockIdx.x / p.n_hb;
   const int h0 = hb * kHC;
-  const int64_t u0 = c * p.U / p.G;
-  const int64_t u1 = (c + 1) * p.U / p.G;
-  const int64_t n_tiles = u1 - u0;
-  const int64_t win0 = p.win0;
+  constexpr bool paged = kPaged;   // a separate instantiation: the contiguous loops stay as they were
+  // The CTA's range of tiles, for sequences of tiles_per_seq tiles each; a
+  // paged batch takes its range from the metadata once the previous kernel in
+  // the stream is done (below).
+  int64_t u0 = c * p.U / p.G;
+  int64_t n_tiles = (c + 1) * p.U / p.G - u0;
   // (sequence, tile within it) of the range's first tile; each role then steps
   // its own copy once per tile rather than dividing
-  const int64_t seq0 = u0 / p.tiles_per_seq;
-  const int64_t tile0 = u0 - seq0 * p.tiles_per_seq;
-  auto step = [&](int64_t& seq, int64_t& tile) {
-    if (++tile == p.tiles_per_seq) { tile = 0; ++seq; }
+  int64_t seq0 = u0 / p.tiles_per_seq;
+  int64_t tile0 = u0 - seq0 * p.tiles_per_seq;
+  auto seq_tiles = [&](int64_t b) -> int64_t {
+    if constexpr (kPaged) return (int64_t)meta_seq(p.meta)[b].w;
+    else return p.tiles_per_seq;
+  };
+  // the next (sequence, tile); a paged batch's sequences without tiles are
+  // passed over (tps: tiles of the current sequence)
+  auto step = [&](int64_t& seq, int64_t& tile, int64_t& tps) {
+    if constexpr (kPaged) {
+      if (++tile == tps) {
+        tile = 0;
+        do {
+          ++seq;
+          tps = seq < p.B ? seq_tiles(seq) : 1;
+        } while (tps == 0);
+      }
+    } else {
+      if (++tile == p.tiles_per_seq) { tile = 0; ++seq; }
+    }
+  };
+  // first rows of a tile's two 64-token halves in the C_KV / K_R tensor maps
+  // (contiguous: one 128-row box from the first).  A paged half that starts at
+  // or past the sequence's end reads the first half's rows again: they are
+  // cleared before use, and no table entry past the sequence's end is read.
+  auto tile_rows = [&](int64_t b, int64_t tile, int32_t& ra, int32_t& rb) {
+    if constexpr (!kPaged) {
+      ra = (int32_t)(b * p.L + tile * kT);
+      rb = ra + kT / 2;
+      return;
+    }
+    const int64_t Lb = meta_seq(p.meta)[b].x;
+    const int64_t tok = tile * kT;
+    ra = (int32_t)paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b, tok, p.err, 0xA04);
+    rb = tok + kT / 2 < Lb ? (int32_t)paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b,
+                                                 tok + kT / 2, p.err, 0xA04)
+                           : ra;
   };
 
   if (tid == 0) {
@@ -323,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   // previous kernel may still run: an L2 prefetch returns no data to this CTA,
   // and L2 holds every later write to those lines, so nothing read after the
   // wait below can be stale.  (One tile: prefetching two measured no better.)
-  if (tid == 0) {
+  if (tid == 0 && !paged) {
     const int32_t frow = (int32_t)(seq0 * p.L + tile0 * kT);
     for (int cc = 0; cc < 8; ++cc) ptx::tma_prefetch_l2_2d(&p.tm_c, 64 * cc, frow);
     ptx::tma_prefetch_l2_2d(&p.tm_k, 0, frow);
@@ -333,6 +381,21 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
   }
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
+  if constexpr (kPaged) {
+    const int64_t U = p.meta[0], Ge = p.meta[1];
+    u0 = 0;
+    n_tiles = 0;
+    seq0 = 0;
+    tile0 = 0;
+    if (c < Ge) {
+      u0 = c * U / Ge;
+      n_tiles = (c + 1) * U / Ge - u0;
+      const int2 rg = meta_range(p.meta, p.B)[c];
+      seq0 = rg.x;
+      tile0 = rg.y;
+    }
+  }
+  const int64_t tps0 = n_tiles > 0 ? seq_tiles(seq0) : 1;
 
   if (warp == 0 && lane == 0) {
     // ===================================================== TMA producer
@@ -367,20 +430,28 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     int64_t cur_b = -1;
     bool ok = true;
     const int64_t T = n_tiles;
-    auto issue = [&](uint64_t* full, int slot, int32_t row, int pr, uint64_t policy) {
+    auto issue = [&](uint64_t* full, int slot, int32_t row, int32_t row_b, int pr, uint64_t policy) {
       if (!LCA_CHECK(p.err, slot >= 0 && slot < kNPair && pr >= 0 && pr < kPairsPerTile, 0xD01)) return;
       ptx::mbar_arrive_expect_tx(full, kPairBytes);
       uint8_t* dst = smem + kOffPair + slot * kPairBytes;
-      ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, full, policy);
-      ptx::tma_load_2d_hint(dst + kChunk, &p.tm_c, 128 * pr + 64, row, full, policy);
+      if constexpr (!kPaged) {
+        ptx::tma_load_2d_hint(dst, &p.tm_c, 128 * pr, row, full, policy);
+        ptx::tma_load_2d_hint(dst + kChunk, &p.tm_c, 128 * pr + 64, row, full, policy);
+      } else {   // 64-row boxes: the second half lands 8 KB (eight swizzle atoms) further on
+        for (int ch = 0; ch < 2; ++ch) {
+          ptx::tma_load_2d_hint(dst + ch * kChunk, &p.tm_c, 128 * pr + 64 * ch, row, full, policy);
+          ptx::tma_load_2d_hint(dst + ch * kChunk + kChunk / 2, &p.tm_c, 128 * pr + 64 * ch, row_b, full,
+                                policy);
+        }
+      }
     };
     // ring A, pair pr (slot pr) of tile i for its scores.  The slot's previous content:
     // nothing (i = 0), the scores load of tile 0 (i = 1), else the reload of i-2.
-    auto load_scores_a = [&](int64_t i, int32_t row, int pr) -> bool {
+    auto load_scores_a = [&](int64_t i, int32_t row, int32_t row_b, int pr) -> bool {
       if (i == 1 && !bounded_wait(&bb.empty_as[pr], 0, abort_flag, p, 0x102, true)) return false;
       if (i >= 2 && !bounded_wait(&bb.empty_ar[pr], (uint32_t)(i - 2) & 1, abort_flag, p, 0x102, true))
         return false;
-      issue(&bb.full_as[pr], pr, row, pr, keep);
+      issue(&bb.full_as[pr], pr, row, row_b, pr, keep);
 #pragma unroll
       for (int q = 0; q < kNA; ++q) if (q == pr) issued_as[q] = (int)i;
       return true;
@@ -388,31 +459,36 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     // ring A, pair pr of tile j again for O.  The slot's previous content: the
     // scores load of tile j+1, or for the last tile the reload of j-1 (the
     // scores load of tile 0 when it is the only tile).
-    auto load_reload_a = [&](int64_t j, int32_t row, int pr) -> bool {
+    auto load_reload_a = [&](int64_t j, int32_t row, int32_t row_b, int pr) -> bool {
       bool w;
       if (j + 1 < T) w = bounded_wait(&bb.empty_as[pr], (uint32_t)(j + 1) & 1, abort_flag, p, 0x103, true);
       else if (j >= 1) w = bounded_wait(&bb.empty_ar[pr], (uint32_t)(j - 1) & 1, abort_flag, p, 0x103, true);
       else w = bounded_wait(&bb.empty_as[pr], 0, abort_flag, p, 0x103, true);
       if (!w) return false;
-      issue(&bb.full_ar[pr], pr, row, pr, once);
+      issue(&bb.full_ar[pr], pr, row, row_b, pr, once);
 #pragma unroll
       for (int q = 0; q < kNA; ++q) if (q == pr) issued_ar[q] = (int)j;
       return true;
     };
     // ring B: the next slot, after O of the tile two back that held it
-    auto load_b = [&](int32_t row, int pr) -> bool {
+    auto load_b = [&](int32_t row, int32_t row_b, int pr) -> bool {
       const int cs = (int)(nb % kNB);
       const int ck = (int)(nb / kNB);
       if (ck >= 1 && !bounded_wait(&bb.empty_b[cs], (ck - 1) & 1, abort_flag, p, 0x104, true)) return false;
-      issue(&bb.full_b[cs], kNA + cs, row, pr, once);
+      issue(&bb.full_b[cs], kNA + cs, row, row_b, pr, once);
 #pragma unroll
       for (int q = 0; q < kNB; ++q) if (q == cs) issued_b[q] = ck;
       ++nb;
       return true;
     };
     int64_t pseq = seq0, ptile = tile0;
-    int32_t prev_row = 0;             // first row of the previous tile
-    for (int64_t u = u0; u < u1 && ok; ++u, step(pseq, ptile)) {
+    int64_t ptps = tps0;
+    int32_t prev_row = 0, prev_row_b = 0;   // first rows of the previous tile's halves
+    // each tile's rows are looked up a tile ahead (a paged batch reads its
+    // block table), so that the lookup's latency passes during the waits
+    int32_t next_row = 0, next_row_b = 0;
+    if (kPaged && n_tiles > 0) tile_rows(pseq, ptile, next_row, next_row_b);
+    for (int64_t i = 0; i < n_tiles && ok; ++i) {
       const int64_t b = pseq;
       if (b != cur_b) {
         cur_b = b;
@@ -426,7 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         ptx::tma_load_2d(smem + kOffQ + 8 * kQChunk, &p.tm_qr, 0, qrow, bb.q_full);
         issued_q = seg;
       }
-      const int32_t row = (int32_t)(b * p.L + ptile * kT);
+      int32_t row = next_row, row_b = next_row_b;
+      if constexpr (!kPaged) tile_rows(b, ptile, row, row_b);
       {
         const int ks = (int)(nk % kNKr);
         const int kk = (int)(nk / kNKr);
@@ -435,18 +512,24 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         if (!(p.debug_skip_load && nk == 0)) {
           ptx::mbar_arrive_expect_tx(&bb.full_k[ks], kChunk);
           ptx::tma_load_2d_hint(smem + kOffKr + ks * kChunk, &p.tm_k, 0, row, &bb.full_k[ks], once);
+          if constexpr (kPaged)
+            ptx::tma_load_2d_hint(smem + kOffKr + ks * kChunk + kChunk / 2, &p.tm_k, 0, row_b, &bb.full_k[ks],
+                                  once);
 #pragma unroll
           for (int q = 0; q < kNKr; ++q) if (q == ks) issued_k[q] = kk;
         }
         ++nk;
       }
-      const int64_t i = u - u0;
-      for (int pr = 0; pr < kNA && ok; ++pr) ok = load_scores_a(i, row, pr);
-      for (int pr = kNA; pr < kPairsPerTile && ok; ++pr) ok = load_b(row, pr);
-      for (int pr = 0; pr < kNA && ok && i >= 1; ++pr) ok = load_reload_a(i - 1, prev_row, pr);
+      for (int pr = 0; pr < kNA && ok; ++pr) ok = load_scores_a(i, row, row_b, pr);
+      for (int pr = kNA; pr < kPairsPerTile && ok; ++pr) ok = load_b(row, row_b, pr);
+      for (int pr = 0; pr < kNA && ok && i >= 1; ++pr) ok = load_reload_a(i - 1, prev_row, prev_row_b, pr);
       prev_row = row;
+      prev_row_b = row_b;
+      step(pseq, ptile, ptps);
+      if (kPaged && i + 1 < n_tiles) tile_rows(pseq, ptile, next_row, next_row_b);
     }
-    for (int pr = 0; pr < kNA && ok && T > 0; ++pr) ok = load_reload_a(T - 1, prev_row, pr);   // the last tile
+    for (int pr = 0; pr < kNA && ok && T > 0; ++pr)
+      ok = load_reload_a(T - 1, prev_row, prev_row_b, pr);   // the last tile
     // Let every copy this thread started land before the CTA can exit.
 #pragma unroll
     for (int i = 0; i < kNA; ++i) {
@@ -474,10 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     int seg = -1;
     int64_t cur_b = -1;
     bool ok = true;
-    int64_t sseq = seq0, stile = tile0;
-    for (int64_t t = 0; t < n_tiles && ok; ++t, step(sseq, stile)) {
+    int64_t sseq = seq0, stile = tile0, stps = tps0;
+    for (int64_t t = 0; t < n_tiles && ok; ++t, step(sseq, stile, stps)) {
       const int64_t b = sseq;
-      const bool last_in_seg = t + 1 == n_tiles || stile + 1 == p.tiles_per_seq;
+      const bool last_in_seg = t + 1 == n_tiles || stile + 1 == (kPaged ? stps : p.tiles_per_seq);
       const int buf = (int)(t & 1);
       if (b != cur_b) {
         cur_b = b;
@@ -536,8 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     const uint64_t d_ct = ptx::smem_desc(ptx::smem_u32(smem + kOffPair), kChunk, 1024, ptx::kSwizzle128B);
     // B = P^T, N = 16 heads (8-head core blocks 2 KB apart), K = 16 tokens
     const uint64_t d_pt = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 128, 2048, ptx::kSwizzleNone);
-    int64_t oseq = seq0, otile = tile0;
-    for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile)) {
+    int64_t oseq = seq0, otile = tile0, otps = tps0;
+    for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile, otps)) {
       const int buf = (int)(j & 1);
       if (!bounded_wait(&bb.p_full[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x204, true)) break;
       ptx::tc_fence_after();
@@ -584,10 +667,25 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 #pragma unroll
     for (int h = 0; h < kHH; ++h) { Zt[h] = 0.f; Mh[h] = -INFINITY; }
 
-    int64_t cseq = seq0, ctile = tile0;
-    for (int64_t i = 0; i < n_tiles; ++i, step(cseq, ctile)) {
+    int64_t cseq = seq0, ctile = tile0, ctps = tps0;
+    // the current sequence's length, groups and first window token
+    int64_t sL = 0, snG = 0, swin0 = 0, s_of = -1;
+    for (int64_t i = 0; i < n_tiles; ++i, step(cseq, ctile, ctps)) {
       const int64_t b = cseq, tile = ctile;
-      const bool last_in_seg = i + 1 == n_tiles || tile + 1 == p.tiles_per_seq;
+      const bool last_in_seg = i + 1 == n_tiles || tile + 1 == (kPaged ? ctps : p.tiles_per_seq);
+      if constexpr (kPaged) {
+        if (b != s_of) {
+          s_of = b;
+          const int4 rec = meta_seq(p.meta)[b];
+          sL = rec.x;
+          snG = rec.z;
+          swin0 = snG * g;
+        }
+      } else {
+        sL = p.L;
+        snG = p.nG;
+        swin0 = p.win0;
+      }
       const int buf = (int)(i & 1);
       const int kb = (int)(i >> 1);
       warp_wait(&bb.s_full[buf], kb & 1, abort_flag, p, 0x300);
@@ -604,14 +702,14 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
 
       const int64_t tok0 = tile * kT;
       const int64_t t = tok0 + row;
-      const bool valid = t < p.L;
-      const bool grouped = t < win0;
+      const bool valid = t < sL;
+      const bool grouped = t < swin0;
       if (t < p.bias_rows) {
 #pragma unroll
         for (int h = 0; h < kHH; ++h) s[h] += p.bias;
       }
-      const bool tile_groups = (g > 1) && (tok0 < win0);   // tile-uniform
-      int32_t* anc = p.anchor + ((int64_t)b * p.H + h0 + kHH * hh) * p.nG;
+      const bool tile_groups = (g > 1) && (tok0 < swin0);   // tile-uniform
+      int32_t* anc = p.anchor + ((int64_t)b * p.H + h0 + kHH * hh) * p.anchor_stride;
 
       // ---- step 2: condense; ent = the softmax entry this token stands for
       float kj[kHH], ent[kHH];
@@ -620,8 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
       if (g == 1 && grouped) {
 #pragma unroll
         for (int h = 0; h < kHH; ++h)
-          if (LCA_CHECK(p.err, t < p.nG && h0 + kHH * hh + h < p.H, 0xD04))
-            anc[(int64_t)h * p.nG + t] = (int32_t)(p.pos0 + t);
+          if (LCA_CHECK(p.err, t < snG && h0 + kHH * hh + h < p.H, 0xD04))
+            anc[(int64_t)h * p.anchor_stride + t] = (int32_t)(p.pos0 + t);
       }
       if (tile_groups) {
         const int64_t jg = t / g;                 // this token's group (if grouped)
@@ -671,8 +769,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
           if (writer) {
 #pragma unroll
             for (int h = 0; h < kHH; ++h)
-              if (LCA_CHECK(p.err, jg < p.nG && a[h] >= 0 && a[h] < kT, 0xD05))
-                anc[(int64_t)h * p.nG + jg] = (int32_t)(p.pos0 + tok0 + a[h]);
+              if (LCA_CHECK(p.err, jg < snG && a[h] >= 0 && a[h] < kT, 0xD05))
+                anc[(int64_t)h * p.anchor_stride + jg] = (int32_t)(p.pos0 + tok0 + a[h]);
           }
         }
       }
@@ -744,6 +842,25 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pk[h2]);
         Zt[2 * h2] += __low2float(v);          // Z from the rounded P
         Zt[2 * h2 + 1] += __high2float(v);
+      }
+      // A paged sequence's last tile: the rows past its last token, in the four
+      // pair slots O reads (pair 3 held in ring B, pairs 0-2 reloaded into ring
+      // A), hold whatever the pool has there.  Their weights are 0, but 0 x NaN
+      // is not, so the softmax warps clear them before P is released.  The
+      // reload cannot be overtaken: the slot's next load waits for O of this
+      // tile, which waits for P.
+      if (kPaged && (tile + 1) * kT > sL) {
+        const int n_valid = (int)(sL - tile * kT);
+        for (int pr = 0; pr < kNA; ++pr) warp_wait(&bb.full_ar[pr], (uint32_t)i & 1, abort_flag, p, 0x306);
+        const int held = kNA + (int)((kHeld * i) % kNB);
+        for (int idx = (warp - 2) * 32 + lane; idx < 4 * 2 * kT * 8; idx += kSoftmaxThreads) {
+          const int row = (idx >> 3) & (kT - 1);    // 8 chunks of 16 bytes a row
+          const int sl = idx >> 11;                 // slot 0-2 (ring A) or 3 (ring B)
+          const int slot = sl < kNA ? sl : held;
+          if (row >= n_valid)
+            *reinterpret_cast<uint4*>(smem + kOffPair + slot * kPairBytes + ((idx >> 10) & 1) * kChunk +
+                                      row * 128 + (idx & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       // the P buffer is free once O of the tile two back is done
       if (i >= 2) warp_wait(&bb.o_full[buf], (uint32_t)((i - 2) >> 1) & 1, abort_flag, p, 0x305);
