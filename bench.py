@@ -525,6 +525,80 @@ def stored_leg(torch, kvc, r, K: int, peaks: dict, t_lca: float, t_mla: float) -
                     "lca_decode_stored over [stored || window] per step, no bias"}
 
 
+def paged_leg(torch, kvc, r, K: int, peaks: dict, t_lca: float) -> dict:
+    """The same batch through lca_decode_paged: its cache cut into 64-token
+    pages placed in a seeded random order in one pool, first at the batch's
+    own length (the cost of the block-table path against lca_decode), then
+    with lengths drawn uniformly from [L/4, L] per sequence (variable-length
+    batch; bytes counted per sequence)."""
+    wl = r.wl
+    ps = 64
+    pages = -(-wl.L // ps)
+    q_c, q_r, c_kv, k_r = r.dev[0]
+    gen = torch.Generator().manual_seed(1234)
+    perm = torch.randperm(wl.B * pages, generator=gen).cuda()
+    table = perm.view(wl.B, pages).to(torch.int32).contiguous()
+    tdt = c_kv.dtype
+
+    def pool_of(t):
+        d = t.shape[-1]
+        src = torch.zeros(wl.B, pages * ps, d, dtype=tdt, device="cuda")
+        src[:, :wl.L] = t
+        pool = torch.empty(wl.B * pages, ps, d, dtype=tdt, device="cuda")
+        pool.index_copy_(0, perm, src.view(wl.B * pages, ps, d))
+        return pool.view(-1, d)
+
+    c_pool, k_pool = pool_of(c_kv), pool_of(k_r)
+    nG_max = wl.n_groups
+    out = torch.empty(wl.B, wl.H, wl.d_c, dtype=torch.float32, device="cuda")
+    anc = torch.empty(wl.B, wl.H, max(nG_max, 1), dtype=torch.int32, device="cuda")
+    full = torch.full((wl.B,), wl.L, dtype=torch.int32, device="cuda")
+    lo = max(1, wl.L // 4)
+    var_host = torch.randint(lo, wl.L + 1, (wl.B,), generator=gen, dtype=torch.int32)
+    var = var_host.cuda()
+
+    def run(lens, steps: int, event=None) -> float:
+        t = Timer(torch, r.stream)
+        t.start()
+        for _ in range(steps):
+            r.plan.decode_paged(q_c, q_r, c_pool, k_pool, ps, table, lens, wl.g, wl.w, out,
+                                anc if nG_max > 0 else None, r.stream)
+        return t.stop() / steps
+
+    res = {}
+    for name, lens, toks in (("same_lengths", full, wl.B * wl.L),
+                             ("variable_lengths", var, int(var_host.sum()))):
+        run(lens, 3)
+        torch.cuda.synchronize()
+        ts = statistics.median([run(lens, K) for _ in range(5)])
+        ev_s = torch.cuda.Event(enable_timing=True)
+        ev_m = torch.cuda.Event(enable_timing=True)
+        mains = []
+        for _ in range(5):
+            ev_s.record(r.stream)
+            r.plan.set_timing_event(ev_m)
+            run(lens, 1)
+            torch.cuda.synchronize()
+            mains.append(ev_s.elapsed_time(ev_m) * 1e-3)
+        r.plan.set_timing_event(None)
+        r.check_device()
+        alg = toks * (wl.d_c + wl.d_r) * wl.elem_bytes + wl.B * wl.H * (wl.d_c + wl.d_r) * wl.elem_bytes + \
+            wl.B * wl.H * wl.d_c * 4
+        tm = statistics.mean(mains)
+        res[name] = {"ms_per_step": ts * 1e3, "main_kernel_ms": tm * 1e3,
+                     "context_tokens_per_s": toks / ts, "context_tokens_per_step": toks,
+                     "hbm_frac_whole_step": alg / ts / 1e9 / peaks["hbm_gbs"],
+                     "hbm_frac_main_kernel": alg / tm / 1e9 / peaks["hbm_gbs"]}
+    res["same_lengths"]["time_vs_lca_decode"] = res["same_lengths"]["ms_per_step"] / (t_lca * 1e3)
+    res.update({"page_size": ps, "pages_per_seq": pages, "kernel": r.kernel(), "unit": UNIT,
+                "variable_lengths_range": [lo, wl.L],
+                "note": "lca_decode_paged over a pool of 64-token pages in random order; the main-kernel "
+                        "time includes the metadata kernel before it"})
+    del c_pool, k_pool
+    torch.cuda.empty_cache()
+    return res
+
+
 def workload_fractions(wl, t_step: float, t_main: float, peaks: dict) -> dict:
     alg = algorithmic_bytes(wl)
     flops = algorithmic_flops(wl)
@@ -643,6 +717,11 @@ def our_arm(args) -> None:
         stored = stored_leg(torch, kvc, r, max(5, min(K, 200)), measured_peaks()[0], t_total / K,
                             t_dense / kd)
 
+    paged = None
+    if not args.no_paged and rank == 0 and world == 1:
+        barrier_sync()
+        paged = paged_leg(torch, kvc, r, max(5, min(K, 50)), measured_peaks()[0], t_total / K)
+
     tokens_per_step = world * wl.B * wl.L
     value = whole_job_rate(world, wl, K, t_total * 1.0)
     peaks, peak_kind = measured_peaks()
@@ -732,6 +811,7 @@ def our_arm(args) -> None:
                        "hbm_frac": alg / (t_dense / kd) / 1e9 / peaks["hbm_gbs"],
                        "note": "dense MLA decode over the same cache (same bytes), same kernels with n_G = 0"},
         "stored_cache": stored,
+        "paged": paged,
         "per_config": pc,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -764,6 +844,7 @@ def main() -> None:
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--no-stored", action="store_true")
+    ap.add_argument("--no-paged", action="store_true")
     args = ap.parse_args()
     rc = spawn_ranks(args)
     if rc is not None:
