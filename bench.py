@@ -47,9 +47,9 @@ L2_BYTES = 126 * 1024 * 1024
 _CSRC = "kv_compression_b200/csrc/"
 TRAFFIC_FILES = {
     "v2lite": ("profiles/lca_tc_kernel_v2lite_traffic.txt",
-               [_CSRC + "tc_kernel.cuh", _CSRC + "ptx.cuh", _CSRC + "checks.cuh"]),
+               [_CSRC + "tc_kernel.cuh", _CSRC + "ptx.cuh", _CSRC + "checks.cuh", _CSRC + "paged_kernel.cuh"]),
     "v2": ("profiles/lca_pair_kernel_v2_traffic.txt",
-           [_CSRC + "pair_kernel.cuh", _CSRC + "ptx.cuh", _CSRC + "checks.cuh"]),
+           [_CSRC + "pair_kernel.cuh", _CSRC + "ptx.cuh", _CSRC + "checks.cuh", _CSRC + "paged_kernel.cuh"]),
 }
 MAIN_KERNEL_NAMES = {"tcgen05": "lca_tc_kernel", "tcgen05_pair": "lca_pair_kernel", "simt": "lca_simt_kernel"}
 
@@ -573,6 +573,8 @@ def paged_leg(torch, kvc, r, K: int, peaks: dict, t_lca: float) -> dict:
         ts = statistics.median([run(lens, K) for _ in range(5)])
         ev_s = torch.cuda.Event(enable_timing=True)
         ev_m = torch.cuda.Event(enable_timing=True)
+        ev_m.record(r.stream)          # torch creates the event at its first record
+        torch.cuda.synchronize()
         mains = []
         for _ in range(5):
             ev_s.record(r.stream)

@@ -105,7 +105,7 @@ constexpr int kOffRecv = kOffP + 2 * kPBytes;
 constexpr int kOffAlpha = kOffRecv + kRecvBytes;           // [2][128] float: the rescale factor per head
 constexpr int kOffFlag = kOffAlpha + 2 * kHeads * 4;       // int [2]: peer rows need a rescale
 constexpr int kOffBar = kOffFlag + 16;
-constexpr int kNumBars = 52;
+constexpr int kNumBars = 53;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -173,7 +173,8 @@ struct Bars {
   uint64_t* sr_empty;    // the softmax warps have read sr
   uint64_t* recv_full;   // [4] quarter q of the peer's partial scores landed (transaction bytes)
   uint64_t* recv_free;   // [4] the peer's quarter q has read the partial scores sent to it
-  uint64_t* p_local;     // the own rows of P buffer i & 1 are written
+  uint64_t* p_local;     // [2] the own rows of P buffer b are written (one barrier per buffer: a
+                         // single one could run two phases ahead of the O issuer's wait)
   uint64_t* p_remote;    // [2 x 4] quarter q of the peer's rows of P buffer b landed (transaction bytes)
   uint64_t* p_free;      // [2 x 2] index 2 c + b: O of CTA c done with P buffer b (and every O before)
   uint64_t* lanes_ready; // the shippers finished what precedes O of a tile (the tile before's rows)
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.recv_full = bb.sr_empty + 1;
   bb.recv_free = bb.recv_full + 4;
   bb.p_local = bb.recv_free + 4;
-  bb.p_remote = bb.p_local + 1;
+  bb.p_remote = bb.p_local + 2;
   bb.p_free = bb.p_remote + 8;
   bb.lanes_ready = bb.p_free + 4;
   bb.dec = bb.lanes_ready + 1;
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.resc_done = bb.resc_go + 1;
   bb.part_done = bb.resc_done + 1;
   bb.drain = bb.part_done + 1;
-  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 1 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 ==
+  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 ==
                     kNumBars,
                 "barrier count");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -410,7 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       ptx::mbar_init(&bb.p_remote[q], 1);         // armed with its transaction bytes
       ptx::mbar_init(&bb.p_remote[4 + q], 1);
     }
-    ptx::mbar_init(bb.p_local, 4);                // the 4 softmax warps
+    ptx::mbar_init(&bb.p_local[0], 4);            // the 4 softmax warps
+    ptx::mbar_init(&bb.p_local[1], 4);
     ptx::mbar_init(bb.lanes_ready, 4);            // the 4 shipper warps
     ptx::mbar_init(bb.resc_go, 1);
     ptx::mbar_init(bb.resc_done, 4);
@@ -611,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     int64_t oseq = seq0, otile = tile0, otps = tps0;
     for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile, otps)) {
       const int buf = (int)(j & 1);
-      if (!bounded_wait(bb.p_local, (uint32_t)j & 1, abort_flag, p, 0x700, true)) break;
+      if (!bounded_wait(&bb.p_local[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x700, true)) break;
       bool ok = true;
       for (int q = 0; q < 4 && ok; ++q)
         ok = bounded_wait(&bb.p_remote[4 * buf + q], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x701, true);
@@ -698,7 +700,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     float M = -INFINITY, Z = 0.f;
     int64_t cseq = seq0, ctile = tile0, ctps = tps0;
     // the current sequence's length, groups and first window token
-    int64_t sL = 0, snG = 0, swin0 = 0, s_of = -1;
+    // (32-bit in the paged kernel: the registers are short there)
+    using SeqInt = std::conditional_t<kPaged, int32_t, int64_t>;
+    SeqInt sL = 0, snG = 0, swin0 = 0;
+    int64_t s_of = -1;
     int seg = 0;
     int64_t i = 0;
     bool ok = n_tiles > 0 ? load_qr(seq0, 0) : true;
@@ -977,7 +982,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ptx::bulk_copy_to_peer(ptx::mapa(ptx::smem_u32(fac), peer), fac, 16 * 4, bar);
         ptx::bulk_commit_group();
         copy_pending = true;
-        ptx::mbar_arrive(bb.p_local);
+        ptx::mbar_arrive(&bb.p_local[buf]);
       }
 
       if (last_of_part(i, tile, ctps)) {
