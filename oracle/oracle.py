@@ -345,3 +345,18 @@ def lca_paged(q_c, q_r, c_pool, k_pool, block_table, seq_lens, page_size: int, g
         anchors.append(r.anchor[0])
         gaps.append(r.tie_gap[0])
     return PagedResult(out, anchors, gaps, mx)
+
+
+def lca_prefill(q_c, q_r, c_pool, k_pool, table_row, pos0: int, page_size: int, g: int, w: int,
+                nthreads: int = 0, lib: ctypes.CDLL | None = None) -> PagedResult:
+    """LCA prefill of a chunk of n queries of one sequence: query i sits at
+    position pos0 + i and attends causally to tokens [0, pos0 + i], which it
+    condenses itself (its own n_G = floor((pos0 + i + 1 - w) / g) groups and
+    its own window).  The sequence's tokens are paged through the one block-
+    table row ``table_row``.  Each query is the decode of its own causal prefix,
+    so this is ``lca_paged`` with the row shared by every query and lengths
+    pos0 + 1 .. pos0 + n."""
+    n = q_c.shape[0]
+    table = np.repeat(np.asarray(table_row, np.int32)[None, :], n, axis=0)
+    lens = np.arange(pos0 + 1, pos0 + n + 1, dtype=np.int32)
+    return lca_paged(q_c, q_r, c_pool, k_pool, table, lens, page_size, g, w, nthreads=nthreads, lib=lib)

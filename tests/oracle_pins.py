@@ -501,10 +501,38 @@ def pin_paged_shared_prefix(lib):
     _check_paged_against_prefix(lib, x, cache, 8, 20)
 
 
+def pin_prefill_causal_prefixes(lib):
+    """Prefill of a chunk of queries at positions pos0 .. pos0 + n - 1 of one
+    paged sequence: query i equals the torch-built LCA of tokens [0, pos0 + i]
+    with its own segmentation (groups complete and appear as the position
+    grows), and tokens after a query's position never change its output."""
+    rng = np.random.default_rng(45)
+    for dtype, ps in (("f32", 64), ("bf16", 128)):
+        n, pos0, g, w = 6, 57, 4, 10
+        x = _paged_inputs(rng, dtype, B=1, L=pos0 + n)
+        qc, qr, _, _ = rand_inputs(rng, n, 2, 1, 16, 8, dtype)
+        cache = workloads.paged_layout(x, [pos0 + n], ps, seed=45)
+        res = orc.lca_prefill(qc, qr, cache.c_pool, cache.k_pool, cache.block_table[0], pos0, ps, g, w, lib=lib)
+        for i in range(n):
+            L = pos0 + i + 1
+            ref, anc = torch_lca_seq(widen(qc[i]), widen(qr[i]), widen(x.c_kv[0, :L]), widen(x.k_r[0, :L]), g, w)
+            assert rel_err(res.out[i], ref) < REL_TOL, (dtype, i)
+            assert np.array_equal(res.anchor[i], anc)
+            assert res.anchor[i].shape[1] == max(0, (L - w) // g)
+        # causality: overwrite the last token; every earlier query is unchanged
+        pool2 = cache.c_pool.copy()
+        last = pos0 + n - 1
+        pool2[cache.block_table[0, last // ps] * ps + last % ps] = cache.c_pool[0]
+        res2 = orc.lca_prefill(qc, qr, pool2, cache.k_pool, cache.block_table[0], pos0, ps, g, w, lib=lib)
+        assert np.array_equal(res2.out[:n - 1], res.out[:n - 1])
+        assert not np.array_equal(res2.out[n - 1], res.out[n - 1])
+
+
 STORED_PINS = [pin_stored_brute_force, pin_stored_g1_dense, pin_stored_single_head,
                pin_stored_constant_groups, pin_stored_zero_query]
 
 ALL_PINS = [pin_segmentation, pin_dense_vs_torch, pin_g1_dense, pin_window_dense, pin_zero_query,
             pin_constant_groups, pin_brute_force, pin_near_tie_report, pin_ties, pin_formulations,
             pin_permutation, pin_constant_rope] + STORED_PINS + [pin_paged_vs_prefix,
-                                                                  pin_paged_shared_prefix]
+                                                                  pin_paged_shared_prefix,
+                                                                  pin_prefill_causal_prefixes]
