@@ -601,6 +601,53 @@ def paged_leg(torch, kvc, r, K: int, peaks: dict, t_lca: float) -> dict:
     return res
 
 
+def prefill_leg(torch, kvc, r, K: int, n: int = 64) -> dict:
+    """LCA prefill of the last chunk of one sequence of the batch: n queries at
+    positions L - n .. L - 1, each condensing its own causal prefix
+    (lca_prefill_paged over the sequence's cache as 64-token pages), beside the
+    same chunk with nothing condensed (w = L: dense causal attention over each
+    prefix, the same kernels).  Queries are seeded N(0, 1) scaled like the
+    workload's."""
+    wl = r.wl
+    ps = 64
+    pages = -(-wl.L // ps)
+    q_c0, q_r0, c_kv, k_r = r.dev[0]
+    c_pool = c_kv[0].contiguous()                 # sequence 0's rows, pages in order
+    k_pool = k_r[0].contiguous()
+    row = torch.arange(pages, dtype=torch.int32, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    tdt = q_c0.dtype
+    q_c = (torch.randn(n, wl.H, wl.d_c, generator=gen, device="cuda") * wl.q_scale).to(tdt)
+    q_r = (torch.randn(n, wl.H, wl.d_r, generator=gen, device="cuda") * wl.q_scale).to(tdt)
+    plan = kvc.Plan(n, wl.H, wl.d_c, wl.d_r, wl.dtype, wl.L)
+    out = torch.empty(n, wl.H, wl.d_c, dtype=torch.float32, device="cuda")
+    anc = torch.empty(n, wl.H, max(wl.n_groups, 1), dtype=torch.int32, device="cuda")
+    pos0 = wl.L - n
+    tokens = n * pos0 + n * (n + 1) // 2          # sum of the queries' prefix lengths
+    res = {"queries": n, "pos0": pos0, "context_tokens_per_chunk": tokens, "page_size": ps,
+           "kernel": plan.kernel(wl.L, wl.g, wl.w), "unit": UNIT}
+    for name, w in (("lca", wl.w), ("dense", wl.L)):
+        def run(steps: int) -> float:
+            t = Timer(torch, r.stream)
+            t.start()
+            for _ in range(steps):
+                plan.prefill_paged(q_c, q_r, c_pool, k_pool, ps, row, pos0, wl.g, w, out,
+                                   anc if w < wl.L else None, r.stream)
+            return t.stop() / steps
+        run(2)
+        torch.cuda.synchronize()
+        ts = statistics.median([run(K) for _ in range(3)])
+        st = plan.device_error()
+        if st != kvc.LCA_OK:
+            raise RuntimeError(f"device error {st} at site {plan.device_error_site():#x} in the prefill leg")
+        res[name] = {"ms_per_chunk": ts * 1e3, "queries_per_s": n / ts, "context_tokens_per_s": tokens / ts}
+    res["note"] = ("each query is the decode of its own causal prefix (lengths pos0 + 1 .. L), every query "
+                   "reading the sequence's pages; the sequence's cache (" +
+                   f"{wl.L * (wl.d_c + wl.d_r) * wl.elem_bytes / 1e6:.0f} MB) is read from L2 after the first query")
+    plan.close()
+    return res
+
+
 def workload_fractions(wl, t_step: float, t_main: float, peaks: dict) -> dict:
     alg = algorithmic_bytes(wl)
     flops = algorithmic_flops(wl)
@@ -723,6 +770,10 @@ def our_arm(args) -> None:
     if not args.no_paged and rank == 0 and world == 1:
         barrier_sync()
         paged = paged_leg(torch, kvc, r, max(5, min(K, 50)), measured_peaks()[0], t_total / K)
+    prefill = None
+    if not args.no_prefill and rank == 0 and world == 1:
+        barrier_sync()
+        prefill = prefill_leg(torch, kvc, r, max(3, min(K, 20)))
 
     tokens_per_step = world * wl.B * wl.L
     value = whole_job_rate(world, wl, K, t_total * 1.0)
@@ -814,6 +865,7 @@ def our_arm(args) -> None:
                        "note": "dense MLA decode over the same cache (same bytes), same kernels with n_G = 0"},
         "stored_cache": stored,
         "paged": paged,
+        "prefill": prefill,
         "per_config": pc,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -847,6 +899,7 @@ def main() -> None:
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--no-stored", action="store_true")
     ap.add_argument("--no-paged", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args()
     rc = spawn_ranks(args)
     if rc is not None:

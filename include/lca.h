@@ -323,6 +323,35 @@ lca_status lca_decode_paged(lca_plan *plan, const void *q_c, const void *q_r, co
                             void *stream);
 
 /*
+ * LCA prefill of a chunk of queries of one sequence, each with per-query
+ * condensation: the plan's B queries sit at positions pos0, pos0 + 1, ...,
+ * pos0 + B - 1 of one sequence whose cache is paged through one block-table
+ * row, and query i attends causally to tokens [0, pos0 + i] -- its own
+ * n_G = floor((pos0 + i + 1 - w) / g) groups and its own window (section 2,
+ * "O Algoritmo LCA", steps 1-3, applied at every position of the prompt; the
+ * summary's prefill figures in section 4 speak of the same condensed
+ * attention during the prefill).  The tokens of the chunk itself must already
+ * be in the cache.  Query i's result is lca_decode_paged's for a sequence of
+ * length pos0 + i + 1 with that block-table row, which is how it runs: the
+ * same kernels, the lengths formed on the device from pos0, every query
+ * reading the one row.
+ *   q_c, q_r         device [B][H][d_c], [B][H][d_r]: query i of the chunk in row i
+ *   c_pool, k_pool,
+ *   num_pages,
+ *   page_size        as for lca_decode_paged
+ *   block_table_row  device int32 [max_pages]: the sequence's pages
+ *   pos0             position of the chunk's first query; 0 <= pos0 and
+ *                    pos0 + B <= min(max_L, max_pages page_size)
+ *   out, anchor      as for lca_decode_paged ([B][H][d_c] and [B][H][anchor_stride])
+ * Errors: LCA_ERR_INVALID_ARG (pos0 out of range, and as for lca_decode_paged);
+ * the rest as for lca_decode_paged.
+ */
+lca_status lca_prefill_paged(lca_plan *plan, const void *q_c, const void *q_r, const void *c_pool,
+                             const void *k_pool, int64_t num_pages, int page_size,
+                             const int32_t *block_table_row, int64_t max_pages, int64_t pos0, int g,
+                             int w, float *out, int32_t *anchor, int64_t anchor_stride, void *stream);
+
+/*
  * lca_decode without a plan and without any allocation.  The page has no
  * counterpart: this is a deployment variant of lca_decode for callers that may
  * not allocate device memory when they decode (a server whose memory is all

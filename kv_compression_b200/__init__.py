@@ -31,7 +31,8 @@ EXPORTS = ["lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", 
            "lca_decode_host", "lca_num_groups", "lca_status_string", "lca_get_device_error",
            "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
            "lca_stored_rows", "lca_build_stored", "lca_decode_stored", "lca_slice_groups",
-           "lca_decode_partial", "lca_merge_partials", "lca_get_device_error_site", "lca_decode_paged"]
+           "lca_decode_partial", "lca_merge_partials", "lca_get_device_error_site", "lca_decode_paged",
+           "lca_prefill_paged"]
 
 
 class LcaError(RuntimeError):
@@ -79,11 +80,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lca_get_device_error_site.argtypes = [vp]
     lib.lca_get_device_error_site.restype = i32
     lib.lca_decode_paged.argtypes = [vp, vp, vp, vp, vp, i64, i32, vp, i64, vp, i32, i32, vp, vp, i64, vp]
+    lib.lca_prefill_paged.argtypes = [vp, vp, vp, vp, vp, i64, i32, vp, i64, i64, i32, i32, vp, vp, i64, vp]
     for name in ("lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
                  "lca_decode_host", "lca_get_device_error", "lca_plan_kernel",
                  "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
                  "lca_build_stored", "lca_decode_stored", "lca_decode_partial", "lca_merge_partials",
-                 "lca_decode_paged"):
+                 "lca_decode_paged", "lca_prefill_paged"):
         getattr(lib, name).restype = i32
     if path == LIB_PATH:
         _lib = lib
@@ -218,6 +220,16 @@ class Plan:
                                           page_size, _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
                                           g, w, _ptr(out), _ptr(anchor), stride, _stream_handle(stream)),
                "lca_decode_paged")
+
+    def prefill_paged(self, q_c, q_r, c_pool, k_pool, page_size: int, table_row, pos0: int, g: int, w: int,
+                      out, anchor, stream=None) -> None:
+        """lca_prefill_paged: the plan's B queries at positions pos0 .. pos0 + B - 1 of the one
+        sequence paged through table_row [max_pages] int32; anchor [B, H, stride] or None."""
+        num_pages = c_pool.shape[0] // page_size
+        stride = 0 if anchor is None else anchor.shape[2]
+        _check(self._lib.lca_prefill_paged(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_pool), _ptr(k_pool), num_pages,
+                                           page_size, _ptr(table_row), table_row.shape[0], pos0, g, w, _ptr(out),
+                                           _ptr(anchor), stride, _stream_handle(stream)), "lca_prefill_paged")
 
     def device_error(self, stream=None) -> int:
         return int(self._lib.lca_get_device_error(self._h, _stream_handle(stream)))

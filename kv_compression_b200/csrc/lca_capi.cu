@@ -130,10 +130,12 @@ struct Slice {
 // block table and the device lengths; cap bounds every length.
 struct Paged {
   const int32_t* block_table;
-  int64_t max_pages;
+  int64_t max_pages;        // pages a sequence may have (bounds every length)
+  int64_t table_stride;     // entries from one sequence's table row to the next (0: one shared row)
   int page_size;
   int64_t num_pages;
-  const int32_t* seq_lens;
+  const int32_t* seq_lens;  // null: a prefill chunk, query b's length pos0 + b + 1
+  int64_t pos0;
   int64_t cap;
   int64_t anchor_stride;
   int g, w;     // the segmentation every sequence's n_G(b) follows
@@ -144,6 +146,7 @@ struct Paged {
 lca_status launch_meta(const lca_plan* p, const Paged& pg, int kT, int64_t G, cudaStream_t stream) {
   lca::MetaParams mp = {};
   mp.seq_lens = pg.seq_lens;
+  mp.pos0 = pg.pos0;
   mp.B = p->B;
   mp.cap = pg.cap;
   mp.g = pg.g;
@@ -226,7 +229,7 @@ lca_status run_simt(lca_plan* p, const void* q_c, const void* q_r, const void* c
   sp.ws_slots = p->ws_slots; sp.err = p->err;
   sp.anchor_stride = pg ? pg->anchor_stride : nG;
   if (pg) {
-    sp.meta = p->meta; sp.block_table = pg->block_table; sp.max_pages = pg->max_pages;
+    sp.meta = p->meta; sp.block_table = pg->block_table; sp.table_stride = pg->table_stride;
     sp.page_size = pg->page_size; sp.num_pages = pg->num_pages;
   }
   const size_t smem = (size_t)(p->d_c + p->d_r + 4 * lca::kSimtTileMax + lca::kSimtWarps) * 4 +
@@ -338,7 +341,7 @@ lca_status run_tc(lca_plan* p, const void* q_c, const void* q_r, const void* c_k
   tp.ws_slots = p->ws_slots;
   tp.anchor_stride = pg ? pg->anchor_stride : nG;
   if (pg) {
-    tp.meta = p->meta; tp.block_table = pg->block_table; tp.max_pages = pg->max_pages;
+    tp.meta = p->meta; tp.block_table = pg->block_table; tp.table_stride = pg->table_stride;
     tp.page_size = pg->page_size; tp.num_pages = pg->num_pages;
   }
   const unsigned grid = (unsigned)(G * n_hb);
@@ -461,7 +464,7 @@ lca_status run_pair(lca_plan* p, const void* q_c, const void* q_r, const void* c
   pp.ws_slots = p->ws_slots;
   pp.anchor_stride = pg ? pg->anchor_stride : nG;
   if (pg) {
-    pp.meta = p->meta; pp.block_table = pg->block_table; pp.max_pages = pg->max_pages;
+    pp.meta = p->meta; pp.block_table = pg->block_table; pp.table_stride = pg->table_stride;
     pp.page_size = pg->page_size; pp.num_pages = pg->num_pages;
   }
   if (launch_pair_g(nG > 0 ? g : 1, pp, (unsigned)(G * n_hb), stream, p->device) != cudaSuccess)
@@ -552,6 +555,42 @@ void free_staging(lca_plan* p) {
   p->st_anc = nullptr;
 }
 
+
+// lca_decode_paged and lca_prefill_paged: argument checks, kernel choice, and
+// the three launches (metadata, decode, combine).
+lca_status paged_impl(lca_plan* p, const void* q_c, const void* q_r, const void* c_pool, const void* k_pool,
+                      int64_t num_pages, int page_size, const int32_t* block_table, int64_t max_pages,
+                      int64_t table_stride, const int32_t* seq_lens, int64_t pos0, int g, int w, float* out,
+                      int32_t* anchor, int64_t anchor_stride, void* stream) {
+  if (!p || !q_c || !q_r || !c_pool || !k_pool || !block_table || !out) return LCA_ERR_INVALID_ARG;
+  if (num_pages < 1 || page_size < 64 || (page_size % 64) != 0 || max_pages < 1 || g < 1 || w < 0 ||
+      anchor_stride < 0)
+    return LCA_ERR_INVALID_ARG;
+  if ((uint64_t)num_pages * (uint64_t)page_size > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
+  if (dev != p->device) return LCA_ERR_PLAN_MISMATCH;
+  Paged pg;
+  pg.block_table = block_table; pg.max_pages = max_pages; pg.table_stride = table_stride;
+  pg.page_size = page_size; pg.num_pages = num_pages; pg.seq_lens = seq_lens; pg.pos0 = pos0;
+  pg.g = g; pg.w = w;
+  pg.cap = std::min<int64_t>(p->max_L, max_pages * (int64_t)page_size);
+  const int64_t nG_cap = lca_num_groups(pg.cap, g, w);
+  if (nG_cap > 0 && !anchor) return LCA_ERR_INVALID_ARG;
+  pg.anchor_stride = anchor ? anchor_stride : INT64_MAX;
+  const Kernel k = choose(p, nG_cap, g);
+  if (k == kNone) return LCA_ERR_UNSUPPORTED;
+  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(c_pool) || !aligned16(k_pool) || !aligned16(out) ||
+      (anchor && !aligned16(anchor)) || (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0)
+    return LCA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Slice whole = {0, 0, nullptr};
+  const int ge = nG_cap > 0 ? g : 1;
+  if (k == kPair) return run_pair(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+  if (k == kTc) return run_tc(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+  return run_simt(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+}
 }  // namespace
 
 extern "C" {
@@ -840,34 +879,19 @@ lca_status lca_decode_paged(lca_plan* p, const void* q_c, const void* q_r, const
                             const int32_t* block_table, int64_t max_pages, const int32_t* seq_lens,
                             int g, int w, float* out, int32_t* anchor, int64_t anchor_stride,
                             void* stream) {
-  if (!p || !q_c || !q_r || !c_pool || !k_pool || !block_table || !seq_lens || !out)
+  if (!seq_lens) return LCA_ERR_INVALID_ARG;
+  return paged_impl(p, q_c, q_r, c_pool, k_pool, num_pages, page_size, block_table, max_pages, max_pages,
+                    seq_lens, 0, g, w, out, anchor, anchor_stride, stream);
+}
+
+lca_status lca_prefill_paged(lca_plan* p, const void* q_c, const void* q_r, const void* c_pool,
+                             const void* k_pool, int64_t num_pages, int page_size,
+                             const int32_t* block_table_row, int64_t max_pages, int64_t pos0, int g, int w,
+                             float* out, int32_t* anchor, int64_t anchor_stride, void* stream) {
+  if (!p || pos0 < 0 || pos0 + p->B > std::min<int64_t>(p->max_L, max_pages * (int64_t)page_size))
     return LCA_ERR_INVALID_ARG;
-  if (num_pages < 1 || page_size < 64 || (page_size % 64) != 0 || max_pages < 1 || g < 1 || w < 0 ||
-      anchor_stride < 0)
-    return LCA_ERR_INVALID_ARG;
-  if ((uint64_t)num_pages * (uint64_t)page_size > (uint64_t)INT32_MAX) return LCA_ERR_UNSUPPORTED;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
-  if (dev != p->device) return LCA_ERR_PLAN_MISMATCH;
-  Paged pg;
-  pg.block_table = block_table; pg.max_pages = max_pages; pg.page_size = page_size;
-  pg.num_pages = num_pages; pg.seq_lens = seq_lens; pg.g = g; pg.w = w;
-  pg.cap = std::min<int64_t>(p->max_L, max_pages * (int64_t)page_size);
-  const int64_t nG_cap = lca_num_groups(pg.cap, g, w);
-  if (nG_cap > 0 && !anchor) return LCA_ERR_INVALID_ARG;
-  pg.anchor_stride = anchor ? anchor_stride : INT64_MAX;
-  const Kernel k = choose(p, nG_cap, g);
-  if (k == kNone) return LCA_ERR_UNSUPPORTED;
-  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(c_pool) || !aligned16(k_pool) || !aligned16(out) ||
-      (anchor && !aligned16(anchor)) || (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
-      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0)
-    return LCA_ERR_ALIGNMENT;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const Slice whole = {0, 0, nullptr};
-  const int ge = nG_cap > 0 ? g : 1;
-  if (k == kPair) return run_pair(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
-  if (k == kTc) return run_tc(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
-  return run_simt(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
+  return paged_impl(p, q_c, q_r, c_pool, k_pool, num_pages, page_size, block_table_row, max_pages, 0,
+                    nullptr, pos0, g, w, out, anchor, anchor_stride, stream);
 }
 
 // For callers that may not allocate device memory when they decode -- a

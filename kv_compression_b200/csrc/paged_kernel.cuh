@@ -8,8 +8,12 @@
 // section 2, "O Algoritmo LCA", step 1).  The lengths stay on the device, so
 // one call needs no host round trip and can be captured in a CUDA graph.
 //
-// lca_paged_meta_kernel (one CTA) reads the lengths and writes, for the
-// decode kernels and the combine:
+// A prefill chunk is the same batch for n queries of one sequence: query b
+// sits at position pos0 + b and condenses its own causal prefix, so its length
+// is pos0 + b + 1 and every query reads the one block-table row (row stride 0).
+//
+// lca_paged_meta_kernel (one CTA) reads the lengths (or forms them from pos0)
+// and writes, for the decode kernels and the combine:
 //
 //   meta[0] U        tiles of all sequences (tile = kT tokens of the chosen kernel)
 //   meta[1] G_eff    tile ranges used: min(G, U); range c = [c U / G_eff, (c+1) U / G_eff)
@@ -48,13 +52,13 @@ __device__ __forceinline__ void input_error(int* err, int where) {
 // The pool row of token `tok` of sequence b: its page from the block table,
 // checked against the pool (an entry outside [0, num_pages) raises the device
 // input bit, and page 0 is read instead, so no access leaves the pool).
-__device__ __forceinline__ int64_t paged_row(const int32_t* table, int64_t max_pages, int page_size,
+__device__ __forceinline__ int64_t paged_row(const int32_t* table, int64_t row_stride, int page_size,
                                              int64_t num_pages, int64_t b, int64_t tok, int* err,
                                              int where) {
   const uint32_t ps = (uint32_t)page_size;
   const uint32_t t = (uint32_t)tok;
   const uint32_t j = t / ps;
-  int64_t page = table[b * max_pages + j];
+  int64_t page = table[b * row_stride + j];
   if (page < 0 || page >= num_pages) {
     input_error(err, where);
     page = 0;
@@ -63,7 +67,8 @@ __device__ __forceinline__ int64_t paged_row(const int32_t* table, int64_t max_p
 }
 
 struct MetaParams {
-  const int32_t* seq_lens;   // [B] device
+  const int32_t* seq_lens;   // [B] device; null: a prefill chunk, length pos0 + b + 1
+  int64_t pos0;
   int B;
   int64_t cap;               // the longest valid length: min(max_L, max_pages * page_size)
   int g, w;
@@ -87,7 +92,7 @@ __global__ void __launch_bounds__(kMetaThreads) lca_paged_meta_kernel(const Meta
   int64_t local = 0;
   bool bad = false;
   for (int b = b0; b < b1; ++b) {
-    const int64_t L = p.seq_lens[b];
+    const int64_t L = p.seq_lens ? (int64_t)p.seq_lens[b] : p.pos0 + b + 1;
     const int64_t nG = L > p.w ? (L - p.w) / p.g : 0;
     const bool ok = L >= 1 && L <= p.cap && nG <= p.anchor_stride;
     bad = bad || !ok;
@@ -108,7 +113,7 @@ __global__ void __launch_bounds__(kMetaThreads) lca_paged_meta_kernel(const Meta
   int64_t start = before + incl - local;
   int4* seq = meta_seq(p.meta);
   for (int b = b0; b < b1; ++b) {
-    int64_t L = p.seq_lens[b];
+    int64_t L = p.seq_lens ? (int64_t)p.seq_lens[b] : p.pos0 + b + 1;
     int64_t nG = L > p.w ? (L - p.w) / p.g : 0;
     if (!(L >= 1 && L <= p.cap && nG <= p.anchor_stride)) L = 0, nG = 0;
     const int64_t tiles = p.kT > 0 ? (L + p.kT - 1) / p.kT : 0;

@@ -148,12 +148,12 @@ struct PairParams {
   int64_t anchor_stride;   // anchors of (b, h) start at (b H + h) anchor_stride
   // Paged, variable-length decode (meta != null): tm_c / tm_k cover the pools,
   // [num_pages * page_size rows]; sequence b's token t is row
-  // block_table[b max_pages + t / page_size] page_size + t % page_size, and its
+  // block_table[b table_stride + t / page_size] page_size + t % page_size, and its
   // length, groups, tiles and the ranges come from the metadata (L, nG, U, G,
   // tiles_per_seq, win0 above are then unused; page_size is a multiple of 64).
   const int* meta;
   const int32_t* block_table;
-  int64_t max_pages;
+  int64_t table_stride;   // block-table entries from one sequence's row to the next (0: one shared row)
   int page_size;
   int64_t num_pages;
 };
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   // first row of a tile's 64 tokens in the C_KV / K_R tensor maps
   auto tile_row = [&](int64_t b, int64_t tile) -> int32_t {
     if constexpr (!kPaged) return (int32_t)(b * p.L + tile * kT);
-    else return (int32_t)paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b, tile * kT, p.err,
+    else return (int32_t)paged_row(p.block_table, p.table_stride, p.page_size, p.num_pages, b, tile * kT, p.err,
                                    0xA03);
   };
 

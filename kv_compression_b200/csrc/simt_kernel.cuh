@@ -61,10 +61,10 @@ struct SimtParams {
   int64_t anchor_stride;     // anchors of (b, h) start at (b H + h) anchor_stride
   // paged, variable-length decode (meta != null): c_kv / k_r are the pools,
   // sequence b has meta_seq(meta)[b].x tokens, token t in row
-  // block_table[b max_pages + t / page_size] page_size + t % page_size
+  // block_table[b table_stride + t / page_size] page_size + t % page_size
   const int* meta;
   const int32_t* block_table;
-  int64_t max_pages;
+  int64_t table_stride;   // block-table entries from one sequence's row to the next (0: one shared row)
   int page_size;
   int64_t num_pages;
 };
@@ -144,7 +144,7 @@ lca_simt_kernel(const SimtParams p) {
     // ---- the rows of this tile's tokens
     for (int tt = tid; tt < n; tt += kSimtThreads)
       if (LCA_CHECK(p.err, tt < kSimtTileMax, 0xC05))
-        rowix[tt] = paged ? paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b, t0 + tt,
+        rowix[tt] = paged ? paged_row(p.block_table, p.table_stride, p.page_size, p.num_pages, b, t0 + tt,
                                       p.err, 0xA02)
                           : t0 + tt;
     __syncthreads();

@@ -132,12 +132,12 @@ struct TcParams {
   // Paged, variable-length decode (meta != null): tm_c / tm_k cover the pools
   // with a 64-row box, and a tile's two 64-token halves are loaded from their
   // own pages; sequence b's token t is row
-  // block_table[b max_pages + t / page_size] page_size + t % page_size, and its
+  // block_table[b table_stride + t / page_size] page_size + t % page_size, and its
   // length, groups, tiles and the ranges come from the metadata (L, nG, U, G,
   // tiles_per_seq, win0 above are then unused; page_size is a multiple of 64).
   const int* meta;
   const int32_t* block_table;
-  int64_t max_pages;
+  int64_t table_stride;   // block-table entries from one sequence's row to the next (0: one shared row)
   int page_size;
   int64_t num_pages;
 };
@@ -329,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_tc_kernel(const __grid_consta
     }
     const int64_t Lb = meta_seq(p.meta)[b].x;
     const int64_t tok = tile * kT;
-    ra = (int32_t)paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b, tok, p.err, 0xA04);
-    rb = tok + kT / 2 < Lb ? (int32_t)paged_row(p.block_table, p.max_pages, p.page_size, p.num_pages, b,
+    ra = (int32_t)paged_row(p.block_table, p.table_stride, p.page_size, p.num_pages, b, tok, p.err, 0xA04);
+    rb = tok + kT / 2 < Lb ? (int32_t)paged_row(p.block_table, p.table_stride, p.page_size, p.num_pages, b,
                                                  tok + kT / 2, p.err, 0xA04)
                            : ra;
   };
