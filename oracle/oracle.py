@@ -360,3 +360,69 @@ def lca_prefill(q_c, q_r, c_pool, k_pool, table_row, pos0: int, page_size: int, 
     table = np.repeat(np.asarray(table_row, np.int32)[None, :], n, axis=0)
     lens = np.arange(pos0 + 1, pos0 + n + 1, dtype=np.int32)
     return lca_paged(q_c, q_r, c_pool, k_pool, table, lens, page_size, g, w, nthreads=nthreads, lib=lib)
+
+
+def _wide(a: np.ndarray) -> np.ndarray:
+    """Stored elements widened exactly to float64 (bf16 carried as uint16 bits)."""
+    if a.dtype == np.uint16:
+        return (np.ascontiguousarray(a).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def lca_gqa(q, k_cache, v_cache, g: int, w: int, rows=None, lib: ctypes.CDLL | None = None) -> OracleResult:
+    """LCA decode for grouped-query attention (GQA), one query token per sequence.
+
+    q [B,H,d_k]; k_cache [B,L,H_kv,d_k] (keys with RoPE applied); v_cache
+    [B,L,H_kv,d_v]; query head h reads KV head h // (H / H_kv).
+
+    The LCA page's dual path ("Latent-Condensed Transformer for Efficient Long
+    Context Modeling", section 2, "Condensacao Dual-Path"; section 3, item 3
+    extends it to GQA) pools the semantic component with the query-aware group
+    softmax and keeps the positional (RoPE) component of the top-scoring token.
+    In a GQA cache the key carries the position and the value the content, so
+    for each query head and each group G_j of the section-2 segmentation:
+      scores   s_t = q . k_t
+      weights  w_t = softmax over t in G_j of s_t
+      anchor   a_j = the lowest index in G_j with the largest s_t
+      entry    key k_{a_j}, value v_bar_j = sum_t w_t v_t, logit q . k_{a_j} = s_{a_j}
+    and the window tokens stand for themselves; the output is the softmax
+    attention over [condensed || window].  Plain float64 numpy, step by step.
+    """
+    B, H, d_k = q.shape
+    L, H_kv = k_cache.shape[1], k_cache.shape[2]
+    d_v = v_cache.shape[3]
+    assert H % H_kv == 0 and k_cache.shape[3] == d_k and v_cache.shape[:3] == (B, L, H_kv)
+    r = H // H_kv
+    rows = list(range(B)) if rows is None else list(rows)
+    nG = num_groups(L, g, w, lib)
+    win0 = max(nG, 0) * g
+    out = np.zeros((len(rows), H, d_v))
+    anc = np.zeros((len(rows), H, max(nG, 0)), np.int32)
+    gap = np.zeros((len(rows), H, max(nG, 0)))
+    mx = np.zeros((len(rows), H))
+    t0 = time.perf_counter()
+    for i, b in enumerate(rows):
+        for h in range(H):
+            kv = h // r
+            K = _wide(k_cache[b, :, kv])            # [L, d_k]
+            V = _wide(v_cache[b, :, kv])            # [L, d_v]
+            s = K @ _wide(q[b, h])                  # [L]
+            mx[i, h] = np.abs(s).max()
+            logits, values = [], []
+            for j in range(nG):
+                sg = s[j * g:(j + 1) * g]
+                a = int(np.argmax(sg))               # first maximum: the lowest index
+                e = np.exp(sg - sg[a])
+                wt = e / e.sum()
+                values.append(wt @ V[j * g:(j + 1) * g])
+                logits.append(sg[a])
+                anc[i, h, j] = j * g + a
+                srt = np.sort(sg)
+                gap[i, h, j] = srt[-1] - srt[-2] if g >= 2 else np.inf
+            for t in range(win0, L):
+                logits.append(s[t])
+                values.append(V[t])
+            lg = np.asarray(logits)
+            p = np.exp(lg - lg.max())
+            out[i, h] = (p / p.sum()) @ np.asarray(values)
+    return OracleResult(out, anc, gap, mx, rows, time.perf_counter() - t0, 1)

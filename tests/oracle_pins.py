@@ -528,6 +528,118 @@ def pin_prefill_causal_prefixes(lib):
         assert not np.array_equal(res2.out[n - 1], res.out[n - 1])
 
 
+# ----------------------------------------------------------------------------- GQA
+def _gqa_inputs(rng, B, H, H_kv, L, d_k, d_v, dtype="f32"):
+    s = 1.0 / math.sqrt(d_k)
+    q = (rng.standard_normal((B, H, d_k)) * s).astype(np.float32)
+    k = rng.standard_normal((B, L, H_kv, d_k)).astype(np.float32)
+    v = rng.standard_normal((B, L, H_kv, d_v)).astype(np.float32)
+    if dtype == "bf16":
+        return tuple(f32_to_bf16_bits(a) for a in (q, k, v))
+    return q, k, v
+
+
+def torch_gqa_seq(q, K, V, g, w):
+    """GQA LCA for one (sequence, query head) from library routines: the
+    condensed set (anchor key, softmax-pooled value) then torch SDPA."""
+    groups, window = partition(K.shape[0], g, w)
+    Kt, Vt, qt = torch.from_numpy(K), torch.from_numpy(V), torch.from_numpy(q)
+    s = Kt @ qt
+    keys, vals, anc = [], [], []
+    for G in groups:
+        idx = torch.tensor(G)
+        a = G[int(torch.argmax(s[idx]))]
+        vals.append(torch.softmax(s[idx], dim=0) @ Vt[idx])
+        keys.append(Kt[a])
+        anc.append(a)
+    for t in window:
+        keys.append(Kt[t])
+        vals.append(Vt[t])
+    o = torch_attention(q[None], torch.stack(keys).numpy(), torch.stack(vals).numpy())[0]
+    return o, anc
+
+
+def pin_gqa_brute_force(lib):
+    """Every (g, w) on short sequences, both element types, 3 query heads per KV
+    head: the oracle's GQA LCA against the torch-built condensed set."""
+    rng = np.random.default_rng(51)
+    for dtype in ("f32", "bf16"):
+        q, k, v = _gqa_inputs(rng, 2, 6, 2, 13, 8, 6, dtype)
+        for g in (1, 2, 3, 5):
+            for w in (0, 1, 4, 13):
+                res = orc.lca_gqa(q, k, v, g, w, lib=lib)
+                for b in range(2):
+                    for h in range(6):
+                        o, anc = torch_gqa_seq(widen(q[b, h]), widen(k[b, :, h // 3]), widen(v[b, :, h // 3]), g, w)
+                        assert rel_err(res.out[b, h], o) < REL_TOL, (dtype, g, w, b, h)
+                        assert list(res.anchor[b, h]) == anc
+
+
+def pin_gqa_is_mla_lca_with_zero_semantic_query(lib):
+    """The reading restated in MLA terms: per KV head, GQA LCA is the MLA LCA
+    of that head's query heads with q_c = 0, C_KV = V (pooled) and K_R = K
+    (anchored) -- against the pinned MLA oracle."""
+    rng = np.random.default_rng(52)
+    q, k, v = _gqa_inputs(rng, 2, 8, 2, 300, 16, 12)
+    res = orc.lca_gqa(q, k, v, 8, 40, lib=lib)
+    for kv in range(2):
+        hs = slice(4 * kv, 4 * kv + 4)
+        ref = orc.lca(np.zeros((2, 4, 12), np.float32), np.ascontiguousarray(q[:, hs]),
+                      np.ascontiguousarray(v[:, :, kv]), np.ascontiguousarray(k[:, :, kv]), 8, 40, lib=lib)
+        assert rel_err(res.out[:, hs], ref.out) < REL_TOL
+        assert np.array_equal(res.anchor[:, hs], ref.anchor)
+
+
+def pin_gqa_dense_limits(lib):
+    """g = 1 and w >= L: nothing is condensed, so GQA LCA is dense GQA softmax
+    attention (torch SDPA over the head's K and V)."""
+    rng = np.random.default_rng(53)
+    q, k, v = _gqa_inputs(rng, 1, 4, 2, 50, 8, 8)
+    for g, w in ((1, 0), (4, 50), (3, 64)):
+        res = orc.lca_gqa(q, k, v, g, w, lib=lib)
+        for h in range(4):
+            o = torch_attention(widen(q[0, h])[None], widen(k[0, :, h // 2]), widen(v[0, :, h // 2]))[0]
+            assert rel_err(res.out[0, h], o) < REL_TOL
+
+
+def pin_gqa_kv_head_sharing(lib):
+    """A query head reads only its own KV head: changing another KV head's
+    cache leaves it unchanged, and two equal query heads of one KV head agree."""
+    rng = np.random.default_rng(54)
+    q, k, v = _gqa_inputs(rng, 1, 6, 3, 90, 8, 8)
+    q[0, 1] = q[0, 0]
+    res = orc.lca_gqa(q, k, v, 4, 10, lib=lib)
+    assert np.array_equal(res.out[0, 0], res.out[0, 1])
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 2] += 1.0
+    v2[:, :, 2] *= -1.0
+    res2 = orc.lca_gqa(q, k2, v2, 4, 10, lib=lib)
+    assert np.array_equal(res2.out[0, :4], res.out[0, :4])
+    assert not np.allclose(res2.out[0, 4:], res.out[0, 4:])
+
+
+def pin_gqa_ties(lib):
+    """Groups whose keys are identical: every score ties, so the anchor is the
+    group's first token and the pooled value is the plain mean of its values."""
+    rng = np.random.default_rng(55)
+    q, k, v = _gqa_inputs(rng, 1, 2, 1, 40, 8, 8)
+    g, w = 5, 10
+    for j in range(6):
+        k[0, j * g:(j + 1) * g] = k[0, j * g]
+    res = orc.lca_gqa(q, k, v, g, w, lib=lib)
+    assert np.array_equal(res.anchor[0], np.tile(np.arange(6) * g, (2, 1)))
+    assert np.all(res.tie_gap[0] == 0)
+    for h in range(2):
+        keys = np.concatenate([widen(k[0, 0:30:g, 0]), widen(k[0, 30:, 0])])
+        vals = np.concatenate([widen(v[0, :30, 0]).reshape(6, g, 8).mean(axis=1), widen(v[0, 30:, 0])])
+        o = torch_attention(widen(q[0, h])[None], keys, vals)[0]
+        assert rel_err(res.out[0, h], o) < REL_TOL
+
+
+GQA_PINS = [pin_gqa_brute_force, pin_gqa_is_mla_lca_with_zero_semantic_query, pin_gqa_dense_limits,
+            pin_gqa_kv_head_sharing, pin_gqa_ties]
+
+
 STORED_PINS = [pin_stored_brute_force, pin_stored_g1_dense, pin_stored_single_head,
                pin_stored_constant_groups, pin_stored_zero_query]
 
@@ -535,4 +647,4 @@ ALL_PINS = [pin_segmentation, pin_dense_vs_torch, pin_g1_dense, pin_window_dense
             pin_constant_groups, pin_brute_force, pin_near_tie_report, pin_ties, pin_formulations,
             pin_permutation, pin_constant_rope] + STORED_PINS + [pin_paged_vs_prefix,
                                                                   pin_paged_shared_prefix,
-                                                                  pin_prefill_causal_prefixes]
+                                                                  pin_prefill_causal_prefixes] + GQA_PINS

@@ -104,3 +104,43 @@ def test_unmutated_copy_passes(oracle_src, tmp_path):
     for pin in pins.ALL_PINS:
         pin(lib)
     assert os.path.exists(lib_path)
+
+
+# Plausible mistakes in the GQA oracle (numpy, in oracle.py): each is planted in a
+# copy of the function's source, and one of the GQA pins must fail.
+GQA_MUTANTS = {
+    # query head h read KV head h % H_kv instead of h // (H / H_kv)
+    "kv_head_interleaved": ("kv = h // r", "kv = h % H_kv"),
+    # pooled key instead of the anchor's key (the positional component mixed)
+    "pooled_key_logit": ("logits.append(sg[a])", "logits.append(wt @ sg)"),
+    # values not pooled: the anchor's value stands for the group
+    "anchor_value": ("values.append(wt @ V[j * g:(j + 1) * g])", "values.append(V[j * g + a])"),
+    # uniform pooling weights
+    "mean_pooling": ("wt = e / e.sum()", "wt = np.full(len(sg), 1.0 / len(sg))"),
+    # tie-break on the highest index
+    "tie_break_highest": ("a = int(np.argmax(sg))", "a = len(sg) - 1 - int(np.argmax(sg[::-1]))"),
+    # window without its first leftover token
+    "window_off_by_one": ("for t in range(win0, L):", "for t in range(win0 + 1, L):"),
+}
+
+
+@pytest.fixture(scope="module")
+def gqa_src():
+    import inspect
+    return inspect.getsource(orc.lca_gqa)
+
+
+@pytest.mark.parametrize("name", sorted(GQA_MUTANTS))
+def test_gqa_mutant_is_caught(name, gqa_src, oracle_lib, monkeypatch):
+    old, new = GQA_MUTANTS[name]
+    assert gqa_src.count(old) == 1, f"mutant anchor text not found: {name}"
+    ns = dict(vars(orc))
+    exec(compile(gqa_src.replace(old, new), "<gqa mutant>", "exec"), ns)
+    monkeypatch.setattr(orc, "lca_gqa", ns["lca_gqa"])
+    failures = []
+    for pin in pins.GQA_PINS:
+        try:
+            pin(oracle_lib)
+        except AssertionError:
+            failures.append(pin.__name__)
+    assert failures, f"GQA mutant {name} passed every pin"
