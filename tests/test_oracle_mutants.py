@@ -90,7 +90,9 @@ def test_mutant_is_caught(name, oracle_src, tmp_path):
     for pin in pins.ALL_PINS:
         try:
             pin(lib)
-        except (AssertionError, RuntimeError):   # a wrong value, or the oracle refusing its own output
+        except (AssertionError, RuntimeError, IndexError, ValueError):
+            # a wrong value, the oracle refusing its own output, or an oracle built on the
+            # mutant's segmentation failing on it
             failures.append(pin.__name__)
     assert failures, f"mutant {name} passed every pin"
 
