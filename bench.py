@@ -648,6 +648,61 @@ def prefill_leg(torch, kvc, r, K: int, n: int = 64) -> dict:
     return res
 
 
+def gqa_leg(torch, kvc, stream, K: int, peaks: dict) -> dict:
+    """GQA LCA decode (lca_decode_gqa) on a Distill-Qwen-7B-shaped batch: B=8,
+    28 query heads over 4 KV heads of 128 (keys and values), L=32768, g=16,
+    w=1024, bf16 caches N(0, 1) and queries N(0, 1)/sqrt(128) drawn on the device
+    (seeded); beside it the same kernels with nothing condensed (w = L)."""
+    B, H, H_kv, d, L, g, w = 8, 28, 4, 128, 32768, 16, 1024
+    gen = torch.Generator(device="cuda").manual_seed(4242)
+    k = torch.randn(B, L, H_kv, d, generator=gen, device="cuda").to(torch.bfloat16)
+    v = torch.randn(B, L, H_kv, d, generator=gen, device="cuda").to(torch.bfloat16)
+    q = (torch.randn(B, H, d, generator=gen, device="cuda") / math.sqrt(d)).to(torch.bfloat16)
+    plan = kvc.Plan(B, H, d, d, "bf16", L)
+    nG = kvc.num_groups(L, g, w)
+    out = torch.empty(B, H, d, dtype=torch.float32, device="cuda")
+    anc = torch.empty(B, H, nG, dtype=torch.int32, device="cuda")
+    alg = B * L * H_kv * 2 * d * 2 + B * H * d * 2 + B * H * d * 4
+    res = {"workload": f"GQA (Distill-Qwen-7B-shaped): B={B} H={H} H_kv={H_kv} d_k=d_v={d} L={L} g={g} w={w} "
+                       "bf16, q*0.0884", "bytes_per_step": alg, "unit": UNIT, "kernel": "lca_gqa_kernel (CUDA cores)"}
+    for name, ww in (("lca", w), ("dense", L)):
+        def step() -> None:
+            plan.decode_gqa(q, k, v, L, H_kv, g, ww, out, anc if ww < L else None, stream)
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        t = Timer(torch, stream)
+        blocks = []
+        for _ in range(5):
+            t.start()
+            for _ in range(K):
+                step()
+            blocks.append(t.stop() / K)
+        ev_s = torch.cuda.Event(enable_timing=True)
+        ev_m = torch.cuda.Event(enable_timing=True)
+        ev_m.record(stream)
+        torch.cuda.synchronize()
+        mains = []
+        for _ in range(5):
+            ev_s.record(stream)
+            plan.set_timing_event(ev_m)
+            step()
+            torch.cuda.synchronize()
+            mains.append(ev_s.elapsed_time(ev_m) * 1e-3)
+        plan.set_timing_event(None)
+        st = plan.device_error()
+        if st != kvc.LCA_OK:
+            raise RuntimeError(f"device error {st} in the GQA leg")
+        ts, tm = statistics.median(blocks), statistics.mean(mains)
+        res[name] = {"ms_per_step": ts * 1e3, "main_kernel_ms": tm * 1e3, "context_tokens_per_s": B * L / ts,
+                     "hbm_frac_whole_step": alg / ts / 1e9 / peaks["hbm_gbs"],
+                     "hbm_frac_main_kernel": alg / tm / 1e9 / peaks["hbm_gbs"]}
+    plan.close()
+    del k, v, q
+    torch.cuda.empty_cache()
+    return res
+
+
 def workload_fractions(wl, t_step: float, t_main: float, peaks: dict) -> dict:
     alg = algorithmic_bytes(wl)
     flops = algorithmic_flops(wl)
@@ -830,6 +885,9 @@ def our_arm(args) -> None:
     if rank == 0 and world == 1 and not args.no_per_config:
         others = [n for n in ("v2lite", "v2", "needle", "sweep", "tiny_f32") if n != args.workload]
         pc = per_config(torch, kvc, stream, others, peaks, max(5, min(K, 50)))
+    gqa = None
+    if rank == 0 and world == 1 and not args.no_gqa:
+        gqa = gqa_leg(torch, kvc, stream, max(5, min(K, 50)), peaks)
 
     if dist is not None:
         dist.destroy_process_group()
@@ -866,6 +924,7 @@ def our_arm(args) -> None:
         "stored_cache": stored,
         "paged": paged,
         "prefill": prefill,
+        "gqa": gqa,
         "per_config": pc,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -900,6 +959,7 @@ def main() -> None:
     ap.add_argument("--no-stored", action="store_true")
     ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-gqa", action="store_true")
     args = ap.parse_args()
     rc = spawn_ranks(args)
     if rc is not None:

@@ -283,6 +283,37 @@ lca_status lca_plan_set_timing_event(lca_plan *plan, void *event);
 int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
 
 /*
+ * LCA decode for grouped-query attention (GQA): one query token per sequence,
+ * H query heads sharing n_kv_heads key/value heads (query head h reads KV head
+ * h / (H / n_kv_heads)).  Section 2 ("Condensacao Dual-Path") pools the
+ * semantic component and anchors the positional (RoPE) one; section 3, item 3
+ * extends the method to GQA.  In a GQA cache the key carries the position and
+ * the value the content, so per query head and per group G_j (the section-2
+ * segmentation, n_G = floor((L - w) / g)):
+ *   s_t = q . k_t;  w_t = softmax over G_j of s_t;  a_j = lowest-index argmax;
+ *   condensed entry: key k_{a_j} (logit s_{a_j}), value sum_t w_t v_t;
+ * window tokens stand for themselves; out = softmax attention over
+ * [condensed || window].  This equals lca_decode's operation with q_c = 0,
+ * C_KV = V and K_R = K per KV head.
+ * The plan is made with B, H = query heads, d_c = d_v (value width) and
+ * d_r = d_k (key width), max_L >= L.
+ *   q        device [B][H][d_k]; k_cache device [B][L][n_kv_heads][d_k] (keys with
+ *            RoPE applied); v_cache device [B][L][n_kv_heads][d_v]
+ *   out      device fp32 [B][H][d_v];  anchor device int32 [B][H][n_G] (NULL allowed
+ *            only when n_G = 0)
+ * Runs a CUDA-core kernel with fp32 accumulation (one CTA per context split, KV
+ * head and sequence, serving the KV head's query heads).  Needs
+ * H / n_kv_heads <= 16 and d_k, d_v <= 256 (LCA_ERR_UNSUPPORTED otherwise).
+ * Errors: LCA_ERR_INVALID_ARG (null pointers, L outside [1, max_L], g < 1, w < 0,
+ * n_kv_heads < 1 or not dividing H, NULL anchor with groups), LCA_ERR_ALIGNMENT
+ * (q, caches, out or anchor not 16-byte aligned), LCA_ERR_PLAN_MISMATCH,
+ * LCA_ERR_UNSUPPORTED, LCA_ERR_CUDA.
+ */
+lca_status lca_decode_gqa(lca_plan *plan, const void *q, const void *k_cache, const void *v_cache,
+                          int64_t L, int n_kv_heads, int g, int w, float *out, int32_t *anchor,
+                          void *stream);
+
+/*
  * LCA decode of a paged, variable-length batch: the caches of the B sequences
  * sit in pages of one pool, each sequence has its own length, and each is
  * decoded exactly as lca_decode decodes a contiguous cache of that length --

@@ -32,7 +32,7 @@ EXPORTS = ["lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", 
            "lca_plan_kernel", "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
            "lca_stored_rows", "lca_build_stored", "lca_decode_stored", "lca_slice_groups",
            "lca_decode_partial", "lca_merge_partials", "lca_get_device_error_site", "lca_decode_paged",
-           "lca_prefill_paged"]
+           "lca_prefill_paged", "lca_decode_gqa"]
 
 
 class LcaError(RuntimeError):
@@ -81,11 +81,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lca_get_device_error_site.restype = i32
     lib.lca_decode_paged.argtypes = [vp, vp, vp, vp, vp, i64, i32, vp, i64, vp, i32, i32, vp, vp, i64, vp]
     lib.lca_prefill_paged.argtypes = [vp, vp, vp, vp, vp, i64, i32, vp, i64, i64, i32, i32, vp, vp, i64, vp]
+    lib.lca_decode_gqa.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp]
     for name in ("lca_plan_create", "lca_plan_destroy", "lca_plan_set", "lca_decode", "mla_decode",
                  "lca_decode_host", "lca_get_device_error", "lca_plan_kernel",
                  "lca_plan_set_timing_event", "lca_decode_noalloc", "lca_condense",
                  "lca_build_stored", "lca_decode_stored", "lca_decode_partial", "lca_merge_partials",
-                 "lca_decode_paged", "lca_prefill_paged"):
+                 "lca_decode_paged", "lca_prefill_paged", "lca_decode_gqa"):
         getattr(lib, name).restype = i32
     if path == LIB_PATH:
         _lib = lib
@@ -230,6 +231,12 @@ class Plan:
         _check(self._lib.lca_prefill_paged(self._h, _ptr(q_c), _ptr(q_r), _ptr(c_pool), _ptr(k_pool), num_pages,
                                            page_size, _ptr(table_row), table_row.shape[0], pos0, g, w, _ptr(out),
                                            _ptr(anchor), stride, _stream_handle(stream)), "lca_prefill_paged")
+
+    def decode_gqa(self, q, k_cache, v_cache, L: int, n_kv_heads: int, g: int, w: int, out, anchor,
+                   stream=None) -> None:
+        """lca_decode_gqa: q [B,H,d_k], k_cache [B,L,H_kv,d_k], v_cache [B,L,H_kv,d_v] CUDA tensors."""
+        _check(self._lib.lca_decode_gqa(self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), L, n_kv_heads, g, w,
+                                        _ptr(out), _ptr(anchor), _stream_handle(stream)), "lca_decode_gqa")
 
     def device_error(self, stream=None) -> int:
         return int(self._lib.lca_get_device_error(self._h, _stream_handle(stream)))

@@ -15,7 +15,8 @@ LIB = os.path.join(HERE, "liblca.so")
 LIB_CHECKED = os.path.join(HERE, "liblca_checked.so")
 SOURCES = ["lca_capi.cu"]
 HEADERS = ["checks.cuh", "ptx.cuh", "tc_kernel.cuh", "pair_kernel.cuh", "simt_kernel.cuh", "combine_kernel.cuh",
-           "condense_kernel.cuh", "paged_kernel.cuh"]
+           "condense_kernel.cuh", "paged_kernel.cuh",
+           "gqa_kernel.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -15,6 +15,7 @@
 #include "checks.cuh"
 #include "combine_kernel.cuh"
 #include "condense_kernel.cuh"
+#include "gqa_kernel.cuh"
 #include "paged_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "simt_kernel.cuh"
@@ -591,6 +592,53 @@ lca_status paged_impl(lca_plan* p, const void* q_c, const void* q_r, const void*
   if (k == kTc) return run_tc(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
   return run_simt(p, q_c, q_r, c_pool, k_pool, 0, ge, nG_cap, out, anchor, s, whole, &pg);
 }
+
+// GQA LCA decode on the CUDA-core kernel: one CTA per (split, KV head,
+// sequence) over the r = H / H_kv query heads of the KV head.
+lca_status run_gqa(lca_plan* p, const void* q, const void* k, const void* v, int64_t L, int H_kv, int g,
+                   int64_t nG, float* out, int32_t* anchor, cudaStream_t stream) {
+  static std::atomic<uint64_t> configured[2] = {{0}, {0}};
+  const int r = p->H / H_kv;
+  const int ge = nG > 0 ? g : 1;
+  const int tile = ge * std::max(1, 64 / ge);
+  const int elem = (int)elem_size(p->dt);
+  const size_t smem = lca::gqa_smem_bytes(r, p->d_r, p->d_c, tile, elem);
+  constexpr size_t kMaxSmem = 227 * 1024;
+  if (smem > kMaxSmem) return LCA_ERR_UNSUPPORTED;
+  const int64_t units = (int64_t)p->B * H_kv;
+  int64_t n_split = std::max<int64_t>(1, ceil_div(4LL * p->num_sms, units));
+  n_split = std::min<int64_t>(n_split, p->ws_slots / p->B);
+  n_split = std::min<int64_t>(n_split, ceil_div(L, tile));
+  if (n_split < 1) return LCA_ERR_UNSUPPORTED;
+  int64_t split_len = ceil_div(ceil_div(L, n_split), ge) * ge;
+  n_split = ceil_div(L, split_len);
+  lca::GqaParams gp = {};
+  gp.q = q; gp.k = k; gp.v = v;
+  gp.B = p->B; gp.H = p->H; gp.H_kv = H_kv; gp.r = r; gp.d_k = p->d_r; gp.d_v = p->d_c;
+  gp.L = L; gp.g = ge; gp.nG = nG; gp.win0 = nG * ge; gp.split_len = split_len; gp.tile = tile;
+  gp.n_split = (int)n_split; gp.anchor = anchor; gp.part_o = p->part_o; gp.part_mz = p->part_mz;
+  gp.ws_slots = p->ws_slots; gp.err = p->err;
+  const int which = p->dt == LCA_F32 ? 0 : 1;
+  if (!device_flag_set(configured[which], p->device)) {
+    const cudaError_t e = p->dt == LCA_F32
+        ? cudaFuncSetAttribute(lca::lca_gqa_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem)
+        : cudaFuncSetAttribute(lca::lca_gqa_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kMaxSmem);
+    if (e != cudaSuccess) return LCA_ERR_CUDA;
+    device_flag_mark(configured[which], p->device);
+  }
+  dim3 grid((unsigned)n_split, (unsigned)H_kv, (unsigned)p->B);
+  if (p->dt == LCA_F32)
+    lca::lca_gqa_kernel<float><<<grid, lca::kGqaThreads, smem, stream>>>(gp);
+  else
+    lca::lca_gqa_kernel<__nv_bfloat16><<<grid, lca::kGqaThreads, smem, stream>>>(gp);
+  if (cudaGetLastError() != cudaSuccess) return LCA_ERR_CUDA;
+  if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
+  lca::CombineParams cp = {};
+  cp.part_o = p->part_o; cp.part_mz = p->part_mz; cp.out = out;
+  cp.B = p->B; cp.H = p->H; cp.d_c = p->d_c; cp.mode = 0; cp.n_split = (int)n_split;
+  return launch_combine(p, cp, stream, false);
+}
 }  // namespace
 
 extern "C" {
@@ -640,6 +688,11 @@ lca_status lca_plan_create(int B, int H, int d_c, int d_r, lca_dtype dt, int64_t
   const int64_t simt_slots = (int64_t)B * simt_target_splits(p);
   const int64_t tc_slots = p->tc_shape ? (int64_t)B + p->num_sms : 0;
   p->ws_slots = std::max(simt_slots, tc_slots);
+  // the GQA kernel's splits (about four CTAs per SM over B x H_kv), where the
+  // partials of that many slots take at most 64 MiB
+  const int64_t gqa_slots = (int64_t)B * ceil_div(4LL * p->num_sms, B);
+  if ((size_t)gqa_slots * H * d_c * sizeof(float) <= ((size_t)64 << 20))
+    p->ws_slots = std::max(p->ws_slots, gqa_slots);
   const size_t o_bytes = (size_t)p->ws_slots * H * d_c * sizeof(float);
   const size_t mz_bytes = (size_t)p->ws_slots * H * 2 * sizeof(float);
   const size_t meta_bytes = (size_t)lca::meta_ints(B, p->ws_slots) * sizeof(int);
@@ -873,6 +926,26 @@ lca_status lca_get_device_error(lca_plan* p, void* stream) {
 }
 
 int lca_get_device_error_site(const lca_plan* p) { return p ? p->last_site : 0; }
+
+lca_status lca_decode_gqa(lca_plan* p, const void* q, const void* k_cache, const void* v_cache, int64_t L,
+                          int n_kv_heads, int g, int w, float* out, int32_t* anchor, void* stream) {
+  if (!p || !q || !k_cache || !v_cache || !out) return LCA_ERR_INVALID_ARG;
+  if (L < 1 || L > p->max_L || g < 1 || w < 0 || n_kv_heads < 1 || p->H % n_kv_heads != 0)
+    return LCA_ERR_INVALID_ARG;
+  if (p->H / n_kv_heads > lca::kGqaMaxR || p->d_c > lca::kGqaMaxD || p->d_r > lca::kGqaMaxD)
+    return LCA_ERR_UNSUPPORTED;
+  const int64_t nG = lca_num_groups(L, g, w);
+  if (nG > 0 && !anchor) return LCA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
+  if (dev != p->device) return LCA_ERR_PLAN_MISMATCH;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (nG > 0 && !aligned16(anchor)))
+    return LCA_ERR_ALIGNMENT;
+  if ((uint64_t)p->B * (uint64_t)L * (uint64_t)n_kv_heads > (uint64_t)INT64_MAX / 1024) return LCA_ERR_UNSUPPORTED;
+  return run_gqa(p, q, k_cache, v_cache, L, n_kv_heads, g, nG, out, nG > 0 ? anchor : nullptr,
+                 static_cast<cudaStream_t>(stream));
+}
 
 lca_status lca_decode_paged(lca_plan* p, const void* q_c, const void* q_r, const void* c_pool,
                             const void* k_pool, int64_t num_pages, int page_size,

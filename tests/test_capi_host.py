@@ -62,6 +62,7 @@ def test_null_arguments_rejected_without_device(lib):
                                 None) == 1
     assert lib.lca_prefill_paged(None, None, None, None, None, 1, 64, None, 1, 0, 1, 0, None, None, 0,
                                  None) == 1
+    assert lib.lca_decode_gqa(None, None, None, None, 16, 1, 1, 0, None, None, None) == 1
 
 
 def test_plan_creation_fails_cleanly_without_gpu(lib):

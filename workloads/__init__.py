@@ -35,7 +35,8 @@ from dataclasses import dataclass, field, replace
 
 import numpy as np
 
-TENSOR_ID = {"q_c": 1, "q_r": 2, "c_kv": 3, "k_r": 4, "needle_pos": 5, "page_order": 6}
+TENSOR_ID = {"q_c": 1, "q_r": 2, "c_kv": 3, "k_r": 4, "needle_pos": 5, "page_order": 6,
+             "gqa_q": 7, "gqa_k": 8, "gqa_v": 9}
 NEEDLES_PER_SEQ = 64
 
 
@@ -246,3 +247,31 @@ def paged_layout(x: Inputs, seq_lens, page_size: int, seed: int = 0, spare_pages
             c_pool[r0:r0 + t1 - t0] = x.c_kv[b, t0:t1]
             k_pool[r0:r0 + t1 - t0] = x.k_r[b, t0:t1]
     return PagedCache(c_pool, k_pool, table, seq_lens, page_size)
+
+
+@dataclass
+class GqaInputs:
+    q: np.ndarray       # [B, H, d_k]
+    k: np.ndarray       # [B, L, H_kv, d_k]
+    v: np.ndarray       # [B, L, H_kv, d_v]
+    dtype: str
+
+
+def generate_gqa(B: int, H: int, H_kv: int, d_k: int, d_v: int, L: int, dtype: str = "bf16",
+                 seed: int = 0) -> GqaInputs:
+    """A grouped-query-attention decode batch: per sequence b, q = N(0,1)/sqrt(d_k)
+    [H, d_k], keys and values N(0,1) [L, H_kv, d] (rng tensors "gqa_q", "gqa_k",
+    "gqa_v"), rounded to bfloat16 when dtype is bf16.  Shapes follow
+    Distill-Qwen-7B-style GQA (28 query heads over 4 KV heads of 128)."""
+    np_dt = np.float32 if dtype == "f32" else np.uint16
+    q = np.empty((B, H, d_k), np_dt)
+    k = np.empty((B, L, H_kv, d_k), np_dt)
+    v = np.empty((B, L, H_kv, d_v), np_dt)
+    for b in range(B):
+        for name, arr, shape, scale in (("gqa_q", q, (H, d_k), 1.0 / math.sqrt(d_k)),
+                                        ("gqa_k", k, (L, H_kv, d_k), 1.0), ("gqa_v", v, (L, H_kv, d_v), 1.0)):
+            x = _rng(seed, name, b).standard_normal(shape, dtype=np.float32)
+            if scale != 1.0:
+                x *= np.float32(scale)
+            arr[b] = f32_to_bf16_bits(x) if dtype == "bf16" else x
+    return GqaInputs(q, k, v, dtype)
