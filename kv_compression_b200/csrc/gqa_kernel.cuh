@@ -8,23 +8,30 @@
 // cache the key carries the position (RoPE) and the value the content, so for
 // each query head and each group G_j of the section-2 segmentation:
 //   s_t = q . k_t,  w_t = softmax_{t in G_j}(s_t),  a_j = lowest-index argmax,
-//   condensed entry: key k_{a_j} (logit s_{a_j} = max_{G_j} s), value sum_t w_t v_t;
+//   condensed entry: key k_{a_j} (logit s_{a_j} = m_j = max_{G_j} s), value sum_t w_t v_t;
 // window tokens stand for themselves, and attention runs over
 // [condensed || window].  As an online softmax over tokens: a grouped token
-// weighs e^{S_j - M} w_t = e^{s_t - M} / den_j (S_j = m_j), a window token
-// e^{s_t - M}; O = sum_t P_t v_t.
+// weighs e^{m_j - M} w_t = e^{s_t - M} / den_j (den_j = sum_{G_j} e^{s_t - m_j}),
+// a window token e^{s_t - M}; the group adds e^{m_j - M} to Z; O = sum_t P_t v_t.
 //
 // One CTA per (context split, KV head, sequence) serves the r = H / H_kv query
 // heads that share the KV head, so each K and V row is read from HBM once per
-// step.  With r <= 16 heads the score block is r x tile, too thin a contraction
-// for the tensor cores; several CTAs per SM hide the load latency.  Per tile:
-//   load      the tile's K and V rows of this KV head into shared memory,
-//             16-byte vector loads (the cache is [B][L][H_kv][d], rows strided)
-//   scores    one warp per token, lanes over dims, r warp sums
-//   condense  one thread per (head, group): max, anchor, den, in-group weights
-//   max       one warp per head: the tile's largest entry, the rescale factor
-//   weights   one thread per (head, token); Z by one warp per head
-//   O         one thread per (head, value dim): O = O alpha + sum_t P_t v_t
+// step.  With r <= 16 heads the score block is r x 64, too thin a contraction
+// for the tensor cores.  Per 64-token tile:
+//   load      the next tile's K and V rows of this KV head stream into the other
+//             shared-memory buffer (cp.async, 16 bytes a copy) while this one is
+//             used; K rows are padded by 16 bytes so the score reads are
+//             conflict-free
+//   scores    one lane per token (warps 2 i and 2 i + 1 take the tile's two halves
+//             for heads i, i + 4, i + 8, i + 12): 16-byte row loads, the heads'
+//             q read as broadcast float4, no reduction
+//   condense  one thread per (head, token), the heads' 64 tokens in two
+//             consecutive warps, so a group of g <= 32 tokens is g neighbouring
+//             lanes: butterfly max and sum, ballot for the lowest-index argmax
+//             (a 64-token group joins its two warps through shared memory)
+//   max, Z    warp reductions per (head, half tile), combined by one thread per head
+//   O         one thread per (head, pair of value dims): O = O alpha + sum_t P_t v_t,
+//             four tokens' weights per float4 load
 // The split partial (M, Z, O) of each head is merged by the combine kernel.
 #pragma once
 #include <cuda_bf16.h>
@@ -36,9 +43,11 @@ namespace lca {
 
 constexpr int kGqaThreads = 256;
 constexpr int kGqaWarps = kGqaThreads / 32;
-constexpr int kGqaMaxR = 16;        // query heads per KV head
-constexpr int kGqaMaxD = 256;       // d_k and d_v
-constexpr int kGqaMaxOut = kGqaMaxR * kGqaMaxD / kGqaThreads;   // O values per thread
+constexpr int kGqaTile = 64;                                        // tokens per tile
+constexpr int kGqaMaxR = 16;                                        // query heads per KV head
+constexpr int kGqaMaxD = 256;                                       // d_k and d_v
+constexpr int kGqaMaxOut = kGqaMaxR * kGqaMaxD / 2 / kGqaThreads;   // O dim pairs per thread
+constexpr int kGqaItems = kGqaMaxR * kGqaTile / kGqaThreads;        // (head, token) items per thread
 
 struct GqaParams {
   const void* q;     // [B][H][d_k]
@@ -46,11 +55,10 @@ struct GqaParams {
   const void* v;     // [B][L][H_kv][d_v]
   int B, H, H_kv, r, d_k, d_v;
   int64_t L;
-  int g;             // group size (1 when nG == 0)
+  int g;             // group size, a power of two <= 64 (1 when nG == 0)
   int64_t nG;
   int64_t win0;      // first window token: n_G g
-  int64_t split_len; // tokens per split (a multiple of g)
-  int tile;          // tokens per tile (a multiple of g)
+  int64_t split_len; // tokens per split (a multiple of 64)
   int n_split;
   int32_t* anchor;   // [B][H][nG] or null when nG == 0
   float* part_o;     // [B * n_split][H][d_v]
@@ -59,51 +67,89 @@ struct GqaParams {
   int* err;
 };
 
+// Elements of one 16-byte copy, and a K row's stride in shared memory (16 bytes of padding).
+template <typename T>
+__host__ __device__ constexpr int gqa_vec() { return 16 / (int)sizeof(T); }
+template <typename T>
+__host__ __device__ inline int gqa_kstride(int d_k) { return d_k + gqa_vec<T>(); }
+
+// Shared memory (floats first): q [r][d_k] | s [r][64] | pw [r][64] | wpart, zpart
+// [r][2] | gstat [r][2][4] | M, Z, alpha [r] | then two buffers of K [64][kstride]
+// and V [64][d_v] elements.
+__host__ __device__ inline size_t gqa_float_bytes(int r, int d_k) {
+  const size_t f = (size_t)r * d_k + 2 * (size_t)r * kGqaTile + 4 * (size_t)r + 8 * (size_t)r + 3 * (size_t)r;
+  return (f * 4 + 15) / 16 * 16;
+}
+template <typename T>
+__host__ __device__ inline size_t gqa_smem_bytes(int r, int d_k, int d_v) {
+  return gqa_float_bytes(r, d_k) + 2 * (size_t)kGqaTile * (gqa_kstride<T>(d_k) + d_v) * sizeof(T);
+}
+
+__device__ __forceinline__ void gqa_cp_async16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void gqa_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void gqa_cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename T>
+__device__ __forceinline__ void gqa_unpack(const uint4& raw, float* f);
+template <>
+__device__ __forceinline__ void gqa_unpack<float>(const uint4& raw, float* f) {
+  f[0] = __uint_as_float(raw.x); f[1] = __uint_as_float(raw.y);
+  f[2] = __uint_as_float(raw.z); f[3] = __uint_as_float(raw.w);
+}
+template <>
+__device__ __forceinline__ void gqa_unpack<__nv_bfloat16>(const uint4& raw, float* f) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+// two consecutive elements (an even index: 4- or 8-byte aligned) as floats
+template <typename T>
+__device__ __forceinline__ void gqa_pair(const T* p, float& a, float& b);
+template <>
+__device__ __forceinline__ void gqa_pair<float>(const float* p, float& a, float& b) {
+  const float2 v = *reinterpret_cast<const float2*>(p);
+  a = v.x;
+  b = v.y;
+}
+template <>
+__device__ __forceinline__ void gqa_pair<__nv_bfloat16>(const __nv_bfloat16* p, float& a, float& b) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  a = __uint_as_float(u << 16);
+  b = __uint_as_float(u & 0xffff0000u);
+}
 template <typename T>
 __device__ __forceinline__ float gqa_elem(const T* p);
 template <>
 __device__ __forceinline__ float gqa_elem<float>(const float* p) { return *p; }
 template <>
-__device__ __forceinline__ float gqa_elem<__nv_bfloat16>(const __nv_bfloat16* p) {
-  return __bfloat162float(*p);
-}
-
-// Shared memory of one CTA (floats unless noted): q [r][d_k] | s [r][tile] |
-// pw [r][tile] | glog [r][tile] | M, Z, alpha [r] each | K tile [tile][d_k] T |
-// V tile [tile][d_v] T.
-__host__ __device__ inline size_t gqa_smem_bytes(int r, int d_k, int d_v, int tile, int elem) {
-  const size_t f = (size_t)r * d_k + 3 * (size_t)r * tile + 3 * (size_t)r;
-  const size_t fb = (f * 4 + 15) / 16 * 16;
-  return fb + (size_t)tile * (d_k + d_v) * elem;
-}
-
-__device__ __forceinline__ float gqa_warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ float gqa_warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
+__device__ __forceinline__ float gqa_elem<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 template <typename T>
-__global__ void __launch_bounds__(kGqaThreads) lca_gqa_kernel(const GqaParams p) {
+__global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams p) {
+  constexpr int kVec = gqa_vec<T>();
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int r = p.r, d_k = p.d_k, d_v = p.d_v, tile = p.tile;
+  const int r = p.r, d_k = p.d_k, d_v = p.d_v, g = p.g;
+  const int kstride = gqa_kstride<T>(d_k);
   extern __shared__ __align__(16) uint8_t gsm[];
   float* qs = reinterpret_cast<float*>(gsm);          // [r][d_k]
-  float* s = qs + r * d_k;                            // [r][tile]
-  float* pw = s + r * tile;                           // [r][tile]
-  float* glog = pw + r * tile;                        // [r][tile]
-  float* Ms = glog + r * tile;                        // [r]
-  float* Zs = Ms + r;                                 // [r]
-  float* As = Zs + r;                                 // [r]
-  const size_t fbytes = (((size_t)r * d_k + 3 * (size_t)r * tile + 3 * (size_t)r) * 4 + 15) / 16 * 16;
-  T* ks = reinterpret_cast<T*>(gsm + fbytes);         // [tile][d_k]
-  T* vs = ks + (size_t)tile * d_k;                    // [tile][d_v]
+  float* s = qs + r * d_k;                            // [r][64] scores
+  float* pw = s + r * kGqaTile;                       // [r][64] token weights
+  float* wpart = pw + r * kGqaTile;                   // [r][2] half-tile maxima
+  float* zpart = wpart + 2 * r;                       // [r][2] half-tile weight sums
+  float* gstat = zpart + 2 * r;                       // [r][2][4] half-group m, den, anchor (64-token groups)
+  float* Ms = gstat + 8 * r;
+  float* Zs = Ms + r;
+  float* As = Zs + r;
+  T* kbuf = reinterpret_cast<T*>(gsm + gqa_float_bytes(r, d_k));   // [2][64][kstride]
+  T* vbuf = kbuf + 2 * kGqaTile * kstride;                          // [2][64][d_v]
 
   const int h0 = kvh * r;
   const T* qg = static_cast<const T*>(p.q) + ((int64_t)b * p.H + h0) * d_k;
@@ -112,124 +158,200 @@ __global__ void __launch_bounds__(kGqaThreads) lca_gqa_kernel(const GqaParams p)
 
   const int64_t s0 = (int64_t)split * p.split_len;
   const int64_t s1 = (p.L < s0 + p.split_len) ? p.L : s0 + p.split_len;
-  const int64_t row_stride = (int64_t)p.H_kv;          // rows of one KV head are H_kv rows apart
-  const T* kg = static_cast<const T*>(p.k) + ((int64_t)b * p.L * row_stride + kvh) * d_k;
-  const T* vg = static_cast<const T*>(p.v) + ((int64_t)b * p.L * row_stride + kvh) * d_v;
-  constexpr int kVec = 16 / sizeof(T);                // elements per 16-byte load
+  const int64_t rs = p.H_kv;                           // a KV head's rows are H_kv rows apart
+  const T* kg = static_cast<const T*>(p.k) + ((int64_t)b * p.L * rs + kvh) * d_k;
+  const T* vg = static_cast<const T*>(p.v) + ((int64_t)b * p.L * rs + kvh) * d_v;
 
-  float o[kGqaMaxOut];
+  auto issue = [&](int64_t t0, int bf) {
+    const int n = (int)(s1 - t0 < kGqaTile ? s1 - t0 : kGqaTile);
+    T* kd = kbuf + bf * kGqaTile * kstride;
+    T* vd = vbuf + bf * kGqaTile * d_v;
+    const int kc = d_k / kVec, vc = d_v / kVec;
+    for (int i = tid; i < n * kc; i += kGqaThreads) {
+      const int tt = i / kc, c = i - tt * kc;
+      gqa_cp_async16(kd + tt * kstride + c * kVec, kg + (t0 + tt) * rs * d_k + c * kVec);
+    }
+    for (int i = tid; i < n * vc; i += kGqaThreads) {
+      const int tt = i / vc, c = i - tt * vc;
+      gqa_cp_async16(vd + tt * d_v + c * kVec, vg + (t0 + tt) * rs * d_v + c * kVec);
+    }
+    gqa_cp_commit();
+  };
+
+  float o[2 * kGqaMaxOut];
 #pragma unroll
-  for (int k = 0; k < kGqaMaxOut; ++k) o[k] = 0.f;
+  for (int k = 0; k < 2 * kGqaMaxOut; ++k) o[k] = 0.f;
+  if (s0 < s1) issue(s0, 0);
   __syncthreads();
 
-  for (int64_t t0 = s0; t0 < s1; t0 += tile) {
-    const int n = (int)((int64_t)tile < s1 - t0 ? (int64_t)tile : s1 - t0);
-    // ---- load the tile's K and V rows of this KV head
+  int bf = 0;
+  for (int64_t t0 = s0; t0 < s1; t0 += kGqaTile, bf ^= 1) {
+    const int n = (int)(s1 - t0 < kGqaTile ? s1 - t0 : kGqaTile);
+    if (t0 + kGqaTile < s1) {
+      issue(t0 + kGqaTile, bf ^ 1);
+      gqa_cp_wait<1>();
+    } else {
+      gqa_cp_wait<0>();
+    }
+    __syncthreads();
+    const T* kb = kbuf + bf * kGqaTile * kstride;
+    const T* vb = vbuf + bf * kGqaTile * d_v;
+
+    // ---- scores: lane = token of the warp's half tile, heads hg, hg + 4, ...
     {
-      const int kc = d_k / kVec, vc = d_v / kVec;
-      for (int i = tid; i < n * kc; i += kGqaThreads) {
-        const int tt = i / kc, c = i - tt * kc;
-        *reinterpret_cast<uint4*>(ks + (size_t)tt * d_k + c * kVec) =
-            __ldg(reinterpret_cast<const uint4*>(kg + (t0 + tt) * row_stride * d_k) + c);
-      }
-      for (int i = tid; i < n * vc; i += kGqaThreads) {
-        const int tt = i / vc, c = i - tt * vc;
-        *reinterpret_cast<uint4*>(vs + (size_t)tt * d_v + c * kVec) =
-            __ldg(reinterpret_cast<const uint4*>(vg + (t0 + tt) * row_stride * d_v) + c);
+      const int hg = warp >> 1;
+      const int tt = (warp & 1) * 32 + lane;
+      float acc[kGqaMaxR / 4];
+#pragma unroll
+      for (int i = 0; i < kGqaMaxR / 4; ++i) acc[i] = 0.f;
+      if (tt < n) {
+        const T* krow = kb + tt * kstride;
+        for (int c = 0; c < d_k; c += kVec) {
+          float kf[kVec];
+          gqa_unpack<T>(*reinterpret_cast<const uint4*>(krow + c), kf);
+#pragma unroll
+          for (int i = 0; i < kGqaMaxR / 4; ++i) {
+            const int h = hg + 4 * i;
+            if (h < r) {
+              const float4* qv = reinterpret_cast<const float4*>(qs + h * d_k + c);
+#pragma unroll
+              for (int e = 0; e < kVec / 4; ++e) {
+                const float4 q4 = qv[e];
+                acc[i] = fmaf(q4.x, kf[4 * e], acc[i]);
+                acc[i] = fmaf(q4.y, kf[4 * e + 1], acc[i]);
+                acc[i] = fmaf(q4.z, kf[4 * e + 2], acc[i]);
+                acc[i] = fmaf(q4.w, kf[4 * e + 3], acc[i]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kGqaMaxR / 4; ++i)
+          if (hg + 4 * i < r) s[(hg + 4 * i) * kGqaTile + tt] = acc[i];
       }
     }
     __syncthreads();
-    // ---- scores: one warp per token, lanes over dims, every head of the KV head
-    for (int tt = warp; tt < n; tt += kGqaWarps) {
-      float acc[kGqaMaxR];
+
+    // ---- condense and the tile's entries: thread per (head, token)
+    const bool tile_groups = t0 < p.win0;               // tile-uniform (g = 1 included)
+    float sv[kGqaItems], dn[kGqaItems];
+    bool gr[kGqaItems];
 #pragma unroll
-      for (int h = 0; h < kGqaMaxR; ++h) acc[h] = 0.f;
-      const T* krow = ks + (size_t)tt * d_k;
-      for (int d = lane; d < d_k; d += 32) {
-        const float kv = gqa_elem(krow + d);
-#pragma unroll
-        for (int h = 0; h < kGqaMaxR; ++h)
-          if (h < r) acc[h] = fmaf(qs[h * d_k + d], kv, acc[h]);
-      }
-#pragma unroll
-      for (int h = 0; h < kGqaMaxR; ++h) {
-        if (h < r) {
-          const float v = gqa_warp_sum(acc[h]);
-          if (lane == 0) s[h * tile + tt] = v;
+    for (int k = 0; k < kGqaItems; ++k) {
+      const int idx = tid + k * kGqaThreads;
+      const bool active = idx < r * kGqaTile;           // warp-uniform (r * 64 is a multiple of 32)
+      const int h = idx >> 6, tt = idx & (kGqaTile - 1);
+      const int64_t t = t0 + tt;
+      const bool valid = active && tt < n;
+      sv[k] = valid ? s[h * kGqaTile + tt] : -INFINITY;
+      gr[k] = valid && t < p.win0;
+      dn[k] = 1.f;
+      float ent = gr[k] ? -INFINITY : sv[k];             // a window token is its own entry
+      if (tile_groups) {
+        // groups are aligned to g and the window starts on a group boundary, so a
+        // group's lanes agree on gr; an invalid lane is never in a valid group
+        const int W = g < 32 ? g : 32;
+        float m = sv[k];
+        for (int off = 1; off < W; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const int base = lane & ~(W - 1);
+        const uint32_t gmask = W == 32 ? 0xffffffffu : (((1u << W) - 1u) << base);
+        const uint32_t ties = __ballot_sync(0xffffffffu, sv[k] == m) & gmask;
+        int a = __ffs(ties) - 1 - base;                  // lowest index among the maxima
+        float den = gr[k] ? expf(sv[k] - m) : 0.f;
+        for (int off = 1; off < W; off <<= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+        if (g > 32) {
+          // a 64-token group: the head's two warps meet in shared memory (warp half 0 first,
+          // so both form the same bits and a tie keeps half 0's anchor)
+          const int half = tt >> 5;
+          if (active && lane == 0) {
+            float* gs = gstat + (h * 2 + half) * 4;
+            gs[0] = m; gs[1] = den; gs[2] = __int_as_float(a + 32 * half);
+          }
+          __syncthreads();
+          if (active) {
+            const float* g0 = gstat + h * 8;
+            const float m0 = g0[0], m1 = g0[4];
+            const float mm = fmaxf(m0, m1);
+            const float f0 = m0 == -INFINITY ? 0.f : expf(m0 - mm), f1 = m1 == -INFINITY ? 0.f : expf(m1 - mm);
+            const float den2 = g0[1] * f0 + g0[5] * f1;
+            a = m1 > m0 ? __float_as_int(g0[6]) : __float_as_int(g0[2]);
+            den = den2;
+            m = mm;
+          }
+          __syncthreads();
+        }
+        dn[k] = den;
+        if (gr[k]) {
+          const bool leader = (tt & (g - 1)) == 0;
+          if (leader) {
+            ent = m;                                     // the condensed logit s_{a_j} = m_j
+            if (LCA_CHECK(p.err, t / g < p.nG && a >= 0 && a < g, 0xC21))
+              p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + t / g] = (int32_t)(t + a);
+          }
         }
       }
+      // the tile's largest entry per (head, half tile)
+      float mx = ent;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      if (active && lane == 0) wpart[h * 2 + (tt >> 5)] = mx;
     }
     __syncthreads();
-    // ---- condense: one thread per (head, group start); the group's logit is its max
-    for (int i = tid; i < r * n; i += kGqaThreads) {
-      const int h = i / n, tt = i - h * n;
-      const int64_t t = t0 + tt;
-      if (t < p.win0 && (t % p.g) == 0 && LCA_CHECK(p.err, tt + p.g <= tile, 0xC21)) {
-        const float* sh = s + h * tile;
-        float m = sh[tt];
-        int amax = tt;
-        for (int u = tt + 1; u < tt + p.g; ++u)
-          if (sh[u] > m) { m = sh[u]; amax = u; }   // strict: the lowest index keeps a tie
-        float den = 0.f;
-        for (int u = tt; u < tt + p.g; ++u) den += expf(sh[u] - m);
-        const float inv = 1.f / den;
-        for (int u = tt; u < tt + p.g; ++u) pw[h * tile + u] = expf(sh[u] - m) * inv;   // w_t
-        glog[h * tile + tt] = m;
-        if (LCA_CHECK(p.err, t / p.g < p.nG, 0xC22))
-          p.anchor[((int64_t)b * p.H + h0 + h) * p.nG + t / p.g] = (int32_t)(t0 + amax);
-      }
+    if (tid < r) {
+      const float Mn = fmaxf(Ms[tid], fmaxf(wpart[2 * tid], wpart[2 * tid + 1]));
+      As[tid] = expf(Ms[tid] - Mn);                      // 0 on the first tile (M = -inf)
+      Ms[tid] = Mn;
     }
     __syncthreads();
-    // ---- the tile's largest entry per head (one warp per head) and the rescale factor
-    for (int h = warp; h < r; h += kGqaWarps) {
-      float mx = -INFINITY;
-      for (int tt = lane; tt < n; tt += 32) {
-        const int64_t t = t0 + tt;
-        if (t < p.win0) {
-          if ((t % p.g) == 0) mx = fmaxf(mx, glog[h * tile + tt]);
-        } else {
-          mx = fmaxf(mx, s[h * tile + tt]);
-        }
+    // ---- per-token weights and Z
+#pragma unroll
+    for (int k = 0; k < kGqaItems; ++k) {
+      const int idx = tid + k * kGqaThreads;
+      const bool active = idx < r * kGqaTile;
+      const int h = idx >> 6, tt = idx & (kGqaTile - 1);
+      float wgt = 0.f;
+      if (active && sv[k] != -INFINITY) {
+        wgt = expf(sv[k] - Ms[h]);
+        if (gr[k]) wgt /= dn[k];
       }
-      mx = gqa_warp_max(mx);
-      if (lane == 0) {
-        const float Mn = fmaxf(Ms[h], mx);
-        As[h] = expf(Ms[h] - Mn);    // 0 on the first tile (M = -inf)
-        Ms[h] = Mn;
-      }
+      if (active) pw[h * kGqaTile + tt] = wgt;
+      float z = wgt;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+      if (active && lane == 0) zpart[h * 2 + (tt >> 5)] = z;
     }
     __syncthreads();
-    // ---- per-token weights
-    for (int i = tid; i < r * n; i += kGqaThreads) {
-      const int h = i / n, tt = i - h * n;
-      const int64_t t = t0 + tt;
-      float wgt;
-      if (t < p.win0) {
-        const int gs = tt - (int)(t % p.g);           // the group's start within the tile
-        wgt = expf(glog[h * tile + gs] - Ms[h]) * pw[h * tile + tt];
-      } else {
-        wgt = expf(s[h * tile + tt] - Ms[h]);
-      }
-      pw[h * tile + tt] = wgt;
-    }
-    __syncthreads();
-    // ---- Z: one warp per head
-    for (int h = warp; h < r; h += kGqaWarps) {
-      float z = 0.f;
-      for (int tt = lane; tt < n; tt += 32) z += pw[h * tile + tt];
-      z = gqa_warp_sum(z);
-      if (lane == 0) Zs[h] = Zs[h] * As[h] + z;
-    }
-    // ---- O = O alpha + sum_t P_t v_t, one thread per (head, value dim)
+    if (tid < r) Zs[tid] = Zs[tid] * As[tid] + (zpart[2 * tid] + zpart[2 * tid + 1]);
+    // ---- O = O alpha + sum_t P_t v_t, one thread per (head, pair of value dims)
+    const int n4 = n & ~3;
 #pragma unroll
     for (int k = 0; k < kGqaMaxOut; ++k) {
       const int idx = tid + k * kGqaThreads;
-      if (idx < r * d_v) {
-        const int h = idx / d_v, d = idx - h * d_v;
-        float acc = o[k] * As[h];
-        const float* ph = pw + h * tile;
-        for (int tt = 0; tt < n; ++tt) acc = fmaf(ph[tt], gqa_elem(vs + (size_t)tt * d_v + d), acc);
-        o[k] = acc;
+      if (idx < r * (d_v / 2)) {
+        const int h = idx / (d_v / 2), d = 2 * (idx - h * (d_v / 2));
+        const float a = As[h];
+        float acc0 = o[2 * k] * a, acc1 = o[2 * k + 1] * a;
+        const float4* ph = reinterpret_cast<const float4*>(pw + h * kGqaTile);
+        for (int t4 = 0; t4 < n4; t4 += 4) {
+          const float4 w4 = ph[t4 >> 2];
+          const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v0, v1;
+            gqa_pair<T>(vb + (t4 + e) * d_v + d, v0, v1);
+            acc0 = fmaf(wv[e], v0, acc0);
+            acc1 = fmaf(wv[e], v1, acc1);
+          }
+        }
+        for (int tt = n4; tt < n; ++tt) {   // rows past n are never read
+          const float wt = pw[h * kGqaTile + tt];
+          float v0, v1;
+          gqa_pair<T>(vb + tt * d_v + d, v0, v1);
+          acc0 = fmaf(wt, v0, acc0);
+          acc1 = fmaf(wt, v1, acc1);
+        }
+        o[2 * k] = acc0;
+        o[2 * k + 1] = acc1;
       }
     }
     __syncthreads();
@@ -240,9 +362,9 @@ __global__ void __launch_bounds__(kGqaThreads) lca_gqa_kernel(const GqaParams p)
 #pragma unroll
   for (int k = 0; k < kGqaMaxOut; ++k) {
     const int idx = tid + k * kGqaThreads;
-    if (idx < r * d_v) {
-      const int h = idx / d_v, d = idx - h * d_v;
-      p.part_o[(slot * p.H + h0 + h) * (int64_t)d_v + d] = o[k];
+    if (idx < r * (d_v / 2)) {
+      const int h = idx / (d_v / 2), d = 2 * (idx - h * (d_v / 2));
+      *reinterpret_cast<float2*>(p.part_o + (slot * p.H + h0 + h) * (int64_t)d_v + d) = make_float2(o[2 * k], o[2 * k + 1]);
     }
   }
   if (tid < r) {

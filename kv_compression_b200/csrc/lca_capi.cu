@@ -600,24 +600,10 @@ lca_status run_gqa(lca_plan* p, const void* q, const void* k, const void* v, int
   static std::atomic<uint64_t> configured[2] = {{0}, {0}};
   const int r = p->H / H_kv;
   const int ge = nG > 0 ? g : 1;
-  const int tile = ge * std::max(1, 64 / ge);
-  const int elem = (int)elem_size(p->dt);
-  const size_t smem = lca::gqa_smem_bytes(r, p->d_r, p->d_c, tile, elem);
+  const size_t smem = p->dt == LCA_F32 ? lca::gqa_smem_bytes<float>(r, p->d_r, p->d_c)
+                                       : lca::gqa_smem_bytes<__nv_bfloat16>(r, p->d_r, p->d_c);
   constexpr size_t kMaxSmem = 227 * 1024;
   if (smem > kMaxSmem) return LCA_ERR_UNSUPPORTED;
-  const int64_t units = (int64_t)p->B * H_kv;
-  int64_t n_split = std::max<int64_t>(1, ceil_div(4LL * p->num_sms, units));
-  n_split = std::min<int64_t>(n_split, p->ws_slots / p->B);
-  n_split = std::min<int64_t>(n_split, ceil_div(L, tile));
-  if (n_split < 1) return LCA_ERR_UNSUPPORTED;
-  int64_t split_len = ceil_div(ceil_div(L, n_split), ge) * ge;
-  n_split = ceil_div(L, split_len);
-  lca::GqaParams gp = {};
-  gp.q = q; gp.k = k; gp.v = v;
-  gp.B = p->B; gp.H = p->H; gp.H_kv = H_kv; gp.r = r; gp.d_k = p->d_r; gp.d_v = p->d_c;
-  gp.L = L; gp.g = ge; gp.nG = nG; gp.win0 = nG * ge; gp.split_len = split_len; gp.tile = tile;
-  gp.n_split = (int)n_split; gp.anchor = anchor; gp.part_o = p->part_o; gp.part_mz = p->part_mz;
-  gp.ws_slots = p->ws_slots; gp.err = p->err;
   const int which = p->dt == LCA_F32 ? 0 : 1;
   if (!device_flag_set(configured[which], p->device)) {
     const cudaError_t e = p->dt == LCA_F32
@@ -627,6 +613,27 @@ lca_status run_gqa(lca_plan* p, const void* q, const void* k, const void* v, int
     if (e != cudaSuccess) return LCA_ERR_CUDA;
     device_flag_mark(configured[which], p->device);
   }
+  // Splits: as many CTAs as are resident at once (one wave, so no tail wave
+  // runs half empty), at least one per (sequence, KV head).
+  int per_sm = 0;
+  const cudaError_t oe = p->dt == LCA_F32
+      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lca::lca_gqa_kernel<float>, lca::kGqaThreads, smem)
+      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lca::lca_gqa_kernel<__nv_bfloat16>,
+                                                      lca::kGqaThreads, smem);
+  if (oe != cudaSuccess || per_sm < 1) { cudaGetLastError(); per_sm = 1; }
+  const int64_t units = (int64_t)p->B * H_kv;
+  int64_t n_split = std::max<int64_t>(1, ((int64_t)per_sm * p->num_sms) / units);
+  n_split = std::min<int64_t>(n_split, p->ws_slots / p->B);
+  n_split = std::min<int64_t>(n_split, ceil_div(L, lca::kGqaTile));
+  if (n_split < 1) return LCA_ERR_UNSUPPORTED;
+  const int64_t split_len = ceil_div(ceil_div(L, n_split), lca::kGqaTile) * lca::kGqaTile;
+  n_split = ceil_div(L, split_len);
+  lca::GqaParams gp = {};
+  gp.q = q; gp.k = k; gp.v = v;
+  gp.B = p->B; gp.H = p->H; gp.H_kv = H_kv; gp.r = r; gp.d_k = p->d_r; gp.d_v = p->d_c;
+  gp.L = L; gp.g = ge; gp.nG = nG; gp.win0 = nG * ge; gp.split_len = split_len;
+  gp.n_split = (int)n_split; gp.anchor = anchor; gp.part_o = p->part_o; gp.part_mz = p->part_mz;
+  gp.ws_slots = p->ws_slots; gp.err = p->err;
   dim3 grid((unsigned)n_split, (unsigned)H_kv, (unsigned)p->B);
   if (p->dt == LCA_F32)
     lca::lca_gqa_kernel<float><<<grid, lca::kGqaThreads, smem, stream>>>(gp);
@@ -935,6 +942,7 @@ lca_status lca_decode_gqa(lca_plan* p, const void* q, const void* k_cache, const
   if (p->H / n_kv_heads > lca::kGqaMaxR || p->d_c > lca::kGqaMaxD || p->d_r > lca::kGqaMaxD)
     return LCA_ERR_UNSUPPORTED;
   const int64_t nG = lca_num_groups(L, g, w);
+  if (nG > 0 && !(is_pow2(g) && g <= lca::kGqaTile)) return LCA_ERR_UNSUPPORTED;
   if (nG > 0 && !anchor) return LCA_ERR_INVALID_ARG;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return LCA_ERR_CUDA;
