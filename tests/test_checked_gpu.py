@@ -16,6 +16,7 @@ from gpu_helpers import (BF16_TOL, F32_TOL, DeviceInputs, compare, oracle_dense,
                          rel_err, run_dense, run_lca, to_device)
 from kv_compression_b200 import build as kbuild  # noqa: E402
 from kv_compression_b200.shard import slice_bounds  # noqa: E402
+from oracle import oracle as orc  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 
@@ -97,4 +98,49 @@ def test_checked_build_fp32_and_stored_and_slices(checked_lib):
     torch.cuda.synchronize()
     assert plan.device_error() == kvc.LCA_OK
     ref = oracle_lca(x, wl.g, wl.w)
+    assert rel_err(out.cpu().numpy().astype(np.float64), ref.out) <= BF16_TOL
+
+
+@pytest.mark.parametrize("H", [128, 16, 4])
+def test_checked_build_paged_and_prefill(H, checked_lib):
+    """The paged decode (ragged lengths, NaN rows outside the sequences) and a
+    prefill chunk on the range-checked build: no check fires, oracle parity."""
+    dt = "f32" if H == 4 else "bf16"
+    kw = dict(d_c=64, d_r=16) if dt == "f32" else {}
+    lengths = [700, 65, 1, 300]
+    wl = workloads.small("chk_paged", B=4, H=H, L=700, g=8, w=40, dtype=dt, seed=9, **kw)
+    x = workloads.generate(wl)
+    cache = workloads.paged_layout(x, lengths, 64, seed=9)
+    plan = _plan(wl, checked_lib)
+    stride = kvc.num_groups(wl.L, 8, 40)
+    out = torch.empty(wl.B, H, wl.d_c, device="cuda")
+    anc = torch.empty(wl.B, H, stride, dtype=torch.int32, device="cuda")
+    c_pool, k_pool = to_device(cache.c_pool), to_device(cache.k_pool)
+    table = torch.from_numpy(cache.block_table).cuda()
+    plan.decode_paged(to_device(x.q_c), to_device(x.q_r), c_pool, k_pool, 64, table,
+                      torch.from_numpy(cache.seq_lens).cuda(), 8, 40, out, anc)
+    torch.cuda.synchronize()
+    assert plan.device_error() == kvc.LCA_OK
+    ref = orc.lca_paged(x.q_c, x.q_r, cache.c_pool, cache.k_pool, cache.block_table, cache.seq_lens, 64, 8, 40)
+    tol = F32_TOL if dt == "f32" else BF16_TOL
+    assert rel_err(out.cpu().numpy().astype(np.float64), ref.out) <= tol
+    # a prefill chunk: the 4 queries at positions 200 .. 203 of sequence 0
+    plan.prefill_paged(to_device(x.q_c), to_device(x.q_r), c_pool, k_pool, 64, table[0].contiguous(), 200, 8, 40,
+                       out, anc)
+    torch.cuda.synchronize()
+    assert plan.device_error() == kvc.LCA_OK
+    pre = orc.lca_prefill(x.q_c, x.q_r, cache.c_pool, cache.k_pool, cache.block_table[0], 200, 64, 8, 40)
+    assert rel_err(out.cpu().numpy().astype(np.float64), pre.out) <= tol
+
+
+def test_checked_build_gqa(checked_lib):
+    x = workloads.generate_gqa(2, 28, 4, 128, 128, 900, "bf16", 3)
+    plan = kvc.Plan(2, 28, 128, 128, "bf16", 900, lib_path=checked_lib)
+    nG = kvc.num_groups(900, 16, 100)
+    out = torch.empty(2, 28, 128, device="cuda")
+    anc = torch.empty(2, 28, nG, dtype=torch.int32, device="cuda")
+    plan.decode_gqa(to_device(x.q), to_device(x.k), to_device(x.v), 900, 4, 16, 100, out, anc)
+    torch.cuda.synchronize()
+    assert plan.device_error() == kvc.LCA_OK
+    ref = orc.lca_gqa(x.q, x.k, x.v, 16, 100)
     assert rel_err(out.cpu().numpy().astype(np.float64), ref.out) <= BF16_TOL
