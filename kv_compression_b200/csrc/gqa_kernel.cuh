@@ -32,12 +32,16 @@
 //   max, Z    warp reductions per (head, half tile), combined by one thread per head
 //   O         one thread per (head, pair of value dims): O = O alpha + sum_t P_t v_t,
 //             four tokens' weights per float4 load
+// The number of heads a lane or thread serves, SLOTS = ceil(r / 4), is a template
+// parameter, so no work is issued for head slots beyond r; the dot products and O
+// run on packed fp32 pairs (two multiply-adds per instruction).
 // The split partial (M, Z, O) of each head is merged by the combine kernel.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
 
 #include "checks.cuh"
+#include "ptx.cuh"
 
 namespace lca {
 
@@ -46,8 +50,6 @@ constexpr int kGqaWarps = kGqaThreads / 32;
 constexpr int kGqaTile = 64;                                        // tokens per tile
 constexpr int kGqaMaxR = 16;                                        // query heads per KV head
 constexpr int kGqaMaxD = 256;                                       // d_k and d_v
-constexpr int kGqaMaxOut = kGqaMaxR * kGqaMaxD / 2 / kGqaThreads;   // O dim pairs per thread
-constexpr int kGqaItems = kGqaMaxR * kGqaTile / kGqaThreads;        // (head, token) items per thread
 
 struct GqaParams {
   const void* q;     // [B][H][d_k]
@@ -131,8 +133,9 @@ __device__ __forceinline__ float gqa_elem<float>(const float* p) { return *p; }
 template <>
 __device__ __forceinline__ float gqa_elem<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-template <typename T>
+template <typename T, int SLOTS>
 __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams p) {
+  static_assert(SLOTS >= 1 && 4 * SLOTS <= kGqaMaxR, "head slots");
   constexpr int kVec = gqa_vec<T>();
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -162,25 +165,39 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
   const T* kg = static_cast<const T*>(p.k) + ((int64_t)b * p.L * rs + kvh) * d_k;
   const T* vg = static_cast<const T*>(p.v) + ((int64_t)b * p.L * rs + kvh) * d_v;
 
+  // this thread's first (row, chunk) of the K and V copies; later ones step by
+  // 256 chunks (the divisions are done once)
+  const int kc = d_k / kVec, vc = d_v / kVec;
+  const int k_row0 = tid / kc, k_c0 = tid - k_row0 * kc;
+  const int v_row0 = tid / vc, v_c0 = tid - v_row0 * vc;
+  const int k_rstep = kGqaThreads / kc, k_cstep = kGqaThreads - k_rstep * kc;
+  const int v_rstep = kGqaThreads / vc, v_cstep = kGqaThreads - v_rstep * vc;
   auto issue = [&](int64_t t0, int bf) {
     const int n = (int)(s1 - t0 < kGqaTile ? s1 - t0 : kGqaTile);
     T* kd = kbuf + bf * kGqaTile * kstride;
     T* vd = vbuf + bf * kGqaTile * d_v;
-    const int kc = d_k / kVec, vc = d_v / kVec;
-    for (int i = tid; i < n * kc; i += kGqaThreads) {
-      const int tt = i / kc, c = i - tt * kc;
-      gqa_cp_async16(kd + tt * kstride + c * kVec, kg + (t0 + tt) * rs * d_k + c * kVec);
+    const T* ks = kg + t0 * rs * d_k;
+    const T* vs = vg + t0 * rs * d_v;
+    for (int tt = k_row0, c = k_c0; tt < n;) {
+      gqa_cp_async16(kd + tt * kstride + c * kVec, ks + (int64_t)tt * rs * d_k + c * kVec);
+      tt += k_rstep;
+      c += k_cstep;
+      if (c >= kc) { c -= kc; ++tt; }
     }
-    for (int i = tid; i < n * vc; i += kGqaThreads) {
-      const int tt = i / vc, c = i - tt * vc;
-      gqa_cp_async16(vd + tt * d_v + c * kVec, vg + (t0 + tt) * rs * d_v + c * kVec);
+    for (int tt = v_row0, c = v_c0; tt < n;) {
+      gqa_cp_async16(vd + tt * d_v + c * kVec, vs + (int64_t)tt * rs * d_v + c * kVec);
+      tt += v_rstep;
+      c += v_cstep;
+      if (c >= vc) { c -= vc; ++tt; }
     }
     gqa_cp_commit();
   };
 
-  float o[2 * kGqaMaxOut];
+  // O dim pairs per thread: r * d_v / 2 pairs over 256 threads, at most SLOTS * d_v / 128
+  constexpr int kOutSlots = SLOTS * kGqaMaxD / 128;
+  float o[2 * kOutSlots];
 #pragma unroll
-  for (int k = 0; k < 2 * kGqaMaxOut; ++k) o[k] = 0.f;
+  for (int k = 0; k < 2 * kOutSlots; ++k) o[k] = 0.f;
   if (s0 < s1) issue(s0, 0);
   __syncthreads();
 
@@ -201,43 +218,49 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
     {
       const int hg = warp >> 1;
       const int tt = (warp & 1) * 32 + lane;
-      float acc[kGqaMaxR / 4];
+      uint64_t acc[SLOTS];   // packed (even dims, odd dims) partial sums
 #pragma unroll
-      for (int i = 0; i < kGqaMaxR / 4; ++i) acc[i] = 0.f;
+      for (int i = 0; i < SLOTS; ++i) acc[i] = ptx::f32x2(0.f, 0.f);
       if (tt < n) {
         const T* krow = kb + tt * kstride;
         for (int c = 0; c < d_k; c += kVec) {
           float kf[kVec];
           gqa_unpack<T>(*reinterpret_cast<const uint4*>(krow + c), kf);
+          uint64_t k2[kVec / 2];
 #pragma unroll
-          for (int i = 0; i < kGqaMaxR / 4; ++i) {
+          for (int e = 0; e < kVec / 2; ++e) k2[e] = ptx::f32x2(kf[2 * e], kf[2 * e + 1]);
+#pragma unroll
+          for (int i = 0; i < SLOTS; ++i) {
             const int h = hg + 4 * i;
             if (h < r) {
               const float4* qv = reinterpret_cast<const float4*>(qs + h * d_k + c);
 #pragma unroll
               for (int e = 0; e < kVec / 4; ++e) {
                 const float4 q4 = qv[e];
-                acc[i] = fmaf(q4.x, kf[4 * e], acc[i]);
-                acc[i] = fmaf(q4.y, kf[4 * e + 1], acc[i]);
-                acc[i] = fmaf(q4.z, kf[4 * e + 2], acc[i]);
-                acc[i] = fmaf(q4.w, kf[4 * e + 3], acc[i]);
+                acc[i] = ptx::fma_f32x2(ptx::f32x2(q4.x, q4.y), k2[2 * e], acc[i]);
+                acc[i] = ptx::fma_f32x2(ptx::f32x2(q4.z, q4.w), k2[2 * e + 1], acc[i]);
               }
             }
           }
         }
 #pragma unroll
-        for (int i = 0; i < kGqaMaxR / 4; ++i)
-          if (hg + 4 * i < r) s[(hg + 4 * i) * kGqaTile + tt] = acc[i];
+        for (int i = 0; i < SLOTS; ++i) {
+          if (hg + 4 * i < r) {
+            float a0, a1;
+            ptx::f32x2_split(acc[i], a0, a1);
+            s[(hg + 4 * i) * kGqaTile + tt] = a0 + a1;
+          }
+        }
       }
     }
     __syncthreads();
 
     // ---- condense and the tile's entries: thread per (head, token)
     const bool tile_groups = t0 < p.win0;               // tile-uniform (g = 1 included)
-    float sv[kGqaItems], dn[kGqaItems];
-    bool gr[kGqaItems];
+    float sv[SLOTS], dn[SLOTS];
+    bool gr[SLOTS];
 #pragma unroll
-    for (int k = 0; k < kGqaItems; ++k) {
+    for (int k = 0; k < SLOTS; ++k) {
       const int idx = tid + k * kGqaThreads;
       const bool active = idx < r * kGqaTile;           // warp-uniform (r * 64 is a multiple of 32)
       const int h = idx >> 6, tt = idx & (kGqaTile - 1);
@@ -305,7 +328,7 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
     __syncthreads();
     // ---- per-token weights and Z
 #pragma unroll
-    for (int k = 0; k < kGqaItems; ++k) {
+    for (int k = 0; k < SLOTS; ++k) {
       const int idx = tid + k * kGqaThreads;
       const bool active = idx < r * kGqaTile;
       const int h = idx >> 6, tt = idx & (kGqaTile - 1);
@@ -325,12 +348,12 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
     // ---- O = O alpha + sum_t P_t v_t, one thread per (head, pair of value dims)
     const int n4 = n & ~3;
 #pragma unroll
-    for (int k = 0; k < kGqaMaxOut; ++k) {
+    for (int k = 0; k < kOutSlots; ++k) {
       const int idx = tid + k * kGqaThreads;
       if (idx < r * (d_v / 2)) {
         const int h = idx / (d_v / 2), d = 2 * (idx - h * (d_v / 2));
         const float a = As[h];
-        float acc0 = o[2 * k] * a, acc1 = o[2 * k + 1] * a;
+        uint64_t acc = ptx::f32x2(o[2 * k] * a, o[2 * k + 1] * a);
         const float4* ph = reinterpret_cast<const float4*>(pw + h * kGqaTile);
         for (int t4 = 0; t4 < n4; t4 += 4) {
           const float4 w4 = ph[t4 >> 2];
@@ -339,19 +362,16 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
           for (int e = 0; e < 4; ++e) {
             float v0, v1;
             gqa_pair<T>(vb + (t4 + e) * d_v + d, v0, v1);
-            acc0 = fmaf(wv[e], v0, acc0);
-            acc1 = fmaf(wv[e], v1, acc1);
+            acc = ptx::fma_f32x2(ptx::f32x2(wv[e], wv[e]), ptx::f32x2(v0, v1), acc);
           }
         }
         for (int tt = n4; tt < n; ++tt) {   // rows past n are never read
           const float wt = pw[h * kGqaTile + tt];
           float v0, v1;
           gqa_pair<T>(vb + tt * d_v + d, v0, v1);
-          acc0 = fmaf(wt, v0, acc0);
-          acc1 = fmaf(wt, v1, acc1);
+          acc = ptx::fma_f32x2(ptx::f32x2(wt, wt), ptx::f32x2(v0, v1), acc);
         }
-        o[2 * k] = acc0;
-        o[2 * k + 1] = acc1;
+        ptx::f32x2_split(acc, o[2 * k], o[2 * k + 1]);
       }
     }
     __syncthreads();
@@ -360,7 +380,7 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
   const int64_t slot = (int64_t)b * p.n_split + split;
   if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xC23)) return;
 #pragma unroll
-  for (int k = 0; k < kGqaMaxOut; ++k) {
+  for (int k = 0; k < kOutSlots; ++k) {
     const int idx = tid + k * kGqaThreads;
     if (idx < r * (d_v / 2)) {
       const int h = idx / (d_v / 2), d = 2 * (idx - h * (d_v / 2));

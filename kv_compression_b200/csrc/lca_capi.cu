@@ -595,32 +595,56 @@ lca_status paged_impl(lca_plan* p, const void* q_c, const void* q_r, const void*
 
 // GQA LCA decode on the CUDA-core kernel: one CTA per (split, KV head,
 // sequence) over the r = H / H_kv query heads of the KV head.
+template <typename T, int SLOTS>
+cudaError_t gqa_setup(int device, size_t smem, int* per_sm) {
+  static std::atomic<uint64_t> configured{0};
+  constexpr size_t kMaxSmem = 227 * 1024;
+  if (!device_flag_set(configured, device)) {
+    const cudaError_t e = cudaFuncSetAttribute(lca::lca_gqa_kernel<T, SLOTS>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
+    if (e != cudaSuccess) return e;
+    device_flag_mark(configured, device);
+  }
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, lca::lca_gqa_kernel<T, SLOTS>, lca::kGqaThreads,
+                                                    smem) != cudaSuccess || *per_sm < 1) {
+    cudaGetLastError();
+    *per_sm = 1;
+  }
+  return cudaSuccess;
+}
+
+template <typename T, int SLOTS>
+void gqa_launch(const lca::GqaParams& gp, dim3 grid, size_t smem, cudaStream_t stream) {
+  lca::lca_gqa_kernel<T, SLOTS><<<grid, lca::kGqaThreads, smem, stream>>>(gp);
+}
+
+// GQA LCA decode on the CUDA-core kernel: one CTA per (split, KV head,
+// sequence) over the r = H / H_kv query heads of the KV head; the kernel is
+// instantiated for ceil(r / 4) head slots.
 lca_status run_gqa(lca_plan* p, const void* q, const void* k, const void* v, int64_t L, int H_kv, int g,
                    int64_t nG, float* out, int32_t* anchor, cudaStream_t stream) {
-  static std::atomic<uint64_t> configured[2] = {{0}, {0}};
   const int r = p->H / H_kv;
+  const int slots = (r + 3) / 4;
   const int ge = nG > 0 ? g : 1;
-  const size_t smem = p->dt == LCA_F32 ? lca::gqa_smem_bytes<float>(r, p->d_r, p->d_c)
-                                       : lca::gqa_smem_bytes<__nv_bfloat16>(r, p->d_r, p->d_c);
-  constexpr size_t kMaxSmem = 227 * 1024;
-  if (smem > kMaxSmem) return LCA_ERR_UNSUPPORTED;
-  const int which = p->dt == LCA_F32 ? 0 : 1;
-  if (!device_flag_set(configured[which], p->device)) {
-    const cudaError_t e = p->dt == LCA_F32
-        ? cudaFuncSetAttribute(lca::lca_gqa_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem)
-        : cudaFuncSetAttribute(lca::lca_gqa_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kMaxSmem);
-    if (e != cudaSuccess) return LCA_ERR_CUDA;
-    device_flag_mark(configured[which], p->device);
-  }
+  const bool f32 = p->dt == LCA_F32;
+  const size_t smem = f32 ? lca::gqa_smem_bytes<float>(r, p->d_r, p->d_c)
+                          : lca::gqa_smem_bytes<__nv_bfloat16>(r, p->d_r, p->d_c);
+  if (smem > 227 * 1024) return LCA_ERR_UNSUPPORTED;
   // Splits: as many CTAs as are resident at once (one wave, so no tail wave
   // runs half empty), at least one per (sequence, KV head).
-  int per_sm = 0;
-  const cudaError_t oe = p->dt == LCA_F32
-      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lca::lca_gqa_kernel<float>, lca::kGqaThreads, smem)
-      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lca::lca_gqa_kernel<__nv_bfloat16>,
-                                                      lca::kGqaThreads, smem);
-  if (oe != cudaSuccess || per_sm < 1) { cudaGetLastError(); per_sm = 1; }
+  int per_sm = 1;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (slots * 2 + (f32 ? 0 : 1)) {
+    case 2: e = gqa_setup<float, 1>(p->device, smem, &per_sm); break;
+    case 3: e = gqa_setup<__nv_bfloat16, 1>(p->device, smem, &per_sm); break;
+    case 4: e = gqa_setup<float, 2>(p->device, smem, &per_sm); break;
+    case 5: e = gqa_setup<__nv_bfloat16, 2>(p->device, smem, &per_sm); break;
+    case 6: e = gqa_setup<float, 3>(p->device, smem, &per_sm); break;
+    case 7: e = gqa_setup<__nv_bfloat16, 3>(p->device, smem, &per_sm); break;
+    case 8: e = gqa_setup<float, 4>(p->device, smem, &per_sm); break;
+    case 9: e = gqa_setup<__nv_bfloat16, 4>(p->device, smem, &per_sm); break;
+  }
+  if (e != cudaSuccess) return LCA_ERR_CUDA;
   const int64_t units = (int64_t)p->B * H_kv;
   int64_t n_split = std::max<int64_t>(1, ((int64_t)per_sm * p->num_sms) / units);
   n_split = std::min<int64_t>(n_split, p->ws_slots / p->B);
@@ -635,10 +659,16 @@ lca_status run_gqa(lca_plan* p, const void* q, const void* k, const void* v, int
   gp.n_split = (int)n_split; gp.anchor = anchor; gp.part_o = p->part_o; gp.part_mz = p->part_mz;
   gp.ws_slots = p->ws_slots; gp.err = p->err;
   dim3 grid((unsigned)n_split, (unsigned)H_kv, (unsigned)p->B);
-  if (p->dt == LCA_F32)
-    lca::lca_gqa_kernel<float><<<grid, lca::kGqaThreads, smem, stream>>>(gp);
-  else
-    lca::lca_gqa_kernel<__nv_bfloat16><<<grid, lca::kGqaThreads, smem, stream>>>(gp);
+  switch (slots * 2 + (f32 ? 0 : 1)) {
+    case 2: gqa_launch<float, 1>(gp, grid, smem, stream); break;
+    case 3: gqa_launch<__nv_bfloat16, 1>(gp, grid, smem, stream); break;
+    case 4: gqa_launch<float, 2>(gp, grid, smem, stream); break;
+    case 5: gqa_launch<__nv_bfloat16, 2>(gp, grid, smem, stream); break;
+    case 6: gqa_launch<float, 3>(gp, grid, smem, stream); break;
+    case 7: gqa_launch<__nv_bfloat16, 3>(gp, grid, smem, stream); break;
+    case 8: gqa_launch<float, 4>(gp, grid, smem, stream); break;
+    case 9: gqa_launch<__nv_bfloat16, 4>(gp, grid, smem, stream); break;
+  }
   if (cudaGetLastError() != cudaSuccess) return LCA_ERR_CUDA;
   if (p->timing_event && cudaEventRecord(p->timing_event, stream) != cudaSuccess) return LCA_ERR_CUDA;
   lca::CombineParams cp = {};
