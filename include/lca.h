@@ -303,7 +303,8 @@ int lca_plan_kernel(lca_plan *plan, int64_t L, int g, int w);
  *            only when n_G = 0)
  * Runs a CUDA-core kernel with fp32 accumulation (one CTA per context split, KV
  * head and sequence, serving the KV head's query heads).  Needs
- * H / n_kv_heads <= 16 and d_k, d_v <= 256 (LCA_ERR_UNSUPPORTED otherwise).
+ * H / n_kv_heads <= 16, d_k <= 256, d_v a power of two in [32, 256], and g a
+ * power of two <= 64 when there are groups (LCA_ERR_UNSUPPORTED otherwise).
  * Errors: LCA_ERR_INVALID_ARG (null pointers, L outside [1, max_L], g < 1, w < 0,
  * n_kv_heads < 1 or not dividing H, NULL anchor with groups), LCA_ERR_ALIGNMENT
  * (q, caches, out or anchor not 16-byte aligned), LCA_ERR_PLAN_MISMATCH,

@@ -30,8 +30,9 @@
 //             lanes: butterfly max and sum, ballot for the lowest-index argmax
 //             (a 64-token group joins its two warps through shared memory)
 //   max, Z    warp reductions per (head, half tile), combined by one thread per head
-//   O         one thread per (head, pair of value dims): O = O alpha + sum_t P_t v_t,
-//             four tokens' weights per float4 load
+//   O         one thread per (slice of the tile's tokens, pair of value dims), for all
+//             r heads: each V element is read from shared memory once and used r
+//             times; the slices' partial sums are added once, at the end
 // The number of heads a lane or thread serves, SLOTS = ceil(r / 4), is a template
 // parameter, so no work is issued for head slots beyond r; the dot products and O
 // run on packed fp32 pairs (two multiply-adds per instruction).
@@ -84,7 +85,11 @@ __host__ __device__ inline size_t gqa_float_bytes(int r, int d_k) {
 }
 template <typename T>
 __host__ __device__ inline size_t gqa_smem_bytes(int r, int d_k, int d_v) {
-  return gqa_float_bytes(r, d_k) + 2 * (size_t)kGqaTile * (gqa_kstride<T>(d_k) + d_v) * sizeof(T);
+  // the tile buffers, which at the end also hold the token slices' partial O
+  // (512 r floats: (256 / (d_v / 2)) slices x r heads x d_v)
+  const size_t tiles = 2 * (size_t)kGqaTile * (gqa_kstride<T>(d_k) + d_v) * sizeof(T);
+  const size_t red = 512 * (size_t)r * sizeof(float);
+  return gqa_float_bytes(r, d_k) + (tiles > red ? tiles : red);
 }
 
 __device__ __forceinline__ void gqa_cp_async16(void* smem_dst, const void* gmem_src) {
@@ -193,11 +198,15 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
     gqa_cp_commit();
   };
 
-  // O dim pairs per thread: r * d_v / 2 pairs over 256 threads, at most SLOTS * d_v / 128
-  constexpr int kOutSlots = SLOTS * kGqaMaxD / 128;
-  float o[2 * kOutSlots];
+  // O: thread = (token slice tg, value-dim pair dp), all r heads; d_v / 2 is a power
+  // of two in [16, 128], so there are 256 / (d_v / 2) slices of d_v / 8 tokens
+  const int npairs = d_v / 2;
+  const int lg_np = __ffs(npairs) - 1;
+  const int dp = tid & (npairs - 1), tg = tid >> lg_np;
+  const int tpg = npairs >> 2;                        // tokens per slice, a multiple of 4
+  float o0[4 * SLOTS], o1[4 * SLOTS];
 #pragma unroll
-  for (int k = 0; k < 2 * kOutSlots; ++k) o[k] = 0.f;
+  for (int h = 0; h < 4 * SLOTS; ++h) { o0[h] = 0.f; o1[h] = 0.f; }
   if (s0 < s1) issue(s0, 0);
   __syncthreads();
 
@@ -345,33 +354,42 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
     }
     __syncthreads();
     if (tid < r) Zs[tid] = Zs[tid] * As[tid] + (zpart[2 * tid] + zpart[2 * tid + 1]);
-    // ---- O = O alpha + sum_t P_t v_t, one thread per (head, pair of value dims)
-    const int n4 = n & ~3;
+    // ---- O = O alpha + sum_t P_t v_t over this thread's token slice, every head
+    {
 #pragma unroll
-    for (int k = 0; k < kOutSlots; ++k) {
-      const int idx = tid + k * kGqaThreads;
-      if (idx < r * (d_v / 2)) {
-        const int h = idx / (d_v / 2), d = 2 * (idx - h * (d_v / 2));
-        const float a = As[h];
-        uint64_t acc = ptx::f32x2(o[2 * k] * a, o[2 * k + 1] * a);
-        const float4* ph = reinterpret_cast<const float4*>(pw + h * kGqaTile);
-        for (int t4 = 0; t4 < n4; t4 += 4) {
-          const float4 w4 = ph[t4 >> 2];
-          const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      for (int h = 0; h < 4 * SLOTS; ++h)
+        if (h < r) { o0[h] *= As[h]; o1[h] *= As[h]; }
+      const int ta = tg * tpg;
+      const int tb = ta + tpg < n ? ta + tpg : n;     // rows past n are never read
+      int tt = ta;
+      for (; tt + 4 <= tb; tt += 4) {
+        float v0[4], v1[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float v0, v1;
-            gqa_pair<T>(vb + (t4 + e) * d_v + d, v0, v1);
-            acc = ptx::fma_f32x2(ptx::f32x2(wv[e], wv[e]), ptx::f32x2(v0, v1), acc);
+        for (int e = 0; e < 4; ++e) gqa_pair<T>(vb + (tt + e) * d_v + 2 * dp, v0[e], v1[e]);
+#pragma unroll
+        for (int h = 0; h < 4 * SLOTS; ++h) {
+          if (h < r) {
+            const float4 w4 = *reinterpret_cast<const float4*>(pw + h * kGqaTile + tt);
+            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o0[h] = fmaf(wv[e], v0[e], o0[h]);
+              o1[h] = fmaf(wv[e], v1[e], o1[h]);
+            }
           }
         }
-        for (int tt = n4; tt < n; ++tt) {   // rows past n are never read
-          const float wt = pw[h * kGqaTile + tt];
-          float v0, v1;
-          gqa_pair<T>(vb + tt * d_v + d, v0, v1);
-          acc = ptx::fma_f32x2(ptx::f32x2(wt, wt), ptx::f32x2(v0, v1), acc);
+      }
+      for (; tt < tb; ++tt) {
+        float v0, v1;
+        gqa_pair<T>(vb + tt * d_v + 2 * dp, v0, v1);
+#pragma unroll
+        for (int h = 0; h < 4 * SLOTS; ++h) {
+          if (h < r) {
+            const float wt = pw[h * kGqaTile + tt];
+            o0[h] = fmaf(wt, v0, o0[h]);
+            o1[h] = fmaf(wt, v1, o1[h]);
+          }
         }
-        ptx::f32x2_split(acc, o[2 * k], o[2 * k + 1]);
       }
     }
     __syncthreads();
@@ -379,12 +397,27 @@ __global__ void __launch_bounds__(kGqaThreads, 3) lca_gqa_kernel(const GqaParams
 
   const int64_t slot = (int64_t)b * p.n_split + split;
   if (!LCA_CHECK(p.err, slot < p.ws_slots, 0xC23)) return;
+  // the token slices' partial sums meet in shared memory (the tile buffers are
+  // free now) and are added in slice order
+  {
+    float* red = reinterpret_cast<float*>(kbuf);      // [slice][r][d_v]
 #pragma unroll
-  for (int k = 0; k < kOutSlots; ++k) {
-    const int idx = tid + k * kGqaThreads;
-    if (idx < r * (d_v / 2)) {
-      const int h = idx / (d_v / 2), d = 2 * (idx - h * (d_v / 2));
-      *reinterpret_cast<float2*>(p.part_o + (slot * p.H + h0 + h) * (int64_t)d_v + d) = make_float2(o[2 * k], o[2 * k + 1]);
+    for (int h = 0; h < 4 * SLOTS; ++h) {
+      if (h < r) {
+        red[(tg * r + h) * d_v + 2 * dp] = o0[h];
+        red[(tg * r + h) * d_v + 2 * dp + 1] = o1[h];
+      }
+    }
+    __syncthreads();
+    const int n_slices = kGqaThreads >> lg_np;
+    for (int i = tid; i < r * npairs; i += kGqaThreads) {
+      const int h = i >> lg_np, d = 2 * (i & (npairs - 1));
+      float a0 = 0.f, a1 = 0.f;
+      for (int sl = 0; sl < n_slices; ++sl) {
+        a0 += red[(sl * r + h) * d_v + d];
+        a1 += red[(sl * r + h) * d_v + d + 1];
+      }
+      *reinterpret_cast<float2*>(p.part_o + (slot * p.H + h0 + h) * (int64_t)d_v + d) = make_float2(a0, a1);
     }
   }
   if (tid < r) {

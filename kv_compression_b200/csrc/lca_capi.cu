@@ -969,7 +969,8 @@ lca_status lca_decode_gqa(lca_plan* p, const void* q, const void* k_cache, const
   if (!p || !q || !k_cache || !v_cache || !out) return LCA_ERR_INVALID_ARG;
   if (L < 1 || L > p->max_L || g < 1 || w < 0 || n_kv_heads < 1 || p->H % n_kv_heads != 0)
     return LCA_ERR_INVALID_ARG;
-  if (p->H / n_kv_heads > lca::kGqaMaxR || p->d_c > lca::kGqaMaxD || p->d_r > lca::kGqaMaxD)
+  if (p->H / n_kv_heads > lca::kGqaMaxR || p->d_c > lca::kGqaMaxD || p->d_r > lca::kGqaMaxD ||
+      !is_pow2(p->d_c) || p->d_c < 32)
     return LCA_ERR_UNSUPPORTED;
   const int64_t nG = lca_num_groups(L, g, w);
   if (nG > 0 && !(is_pow2(g) && g <= lca::kGqaTile)) return LCA_ERR_UNSUPPORTED;
