@@ -772,6 +772,12 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       auto tile_math = [&](auto fast_tag) {
         constexpr bool kFast = decltype(fast_tag)::value;
         float s[kHalfT];
+        // this thread's tokens before the sequence end, with the bias, and grouped,
+        // as counts (32-bit compares against each token's constant offset; unused,
+        // so not formed, when the whole tile is condensed)
+        const int n_in = (int)(sL - tok0 < 0 ? 0 : (sL - tok0 > kHalfT ? kHalfT : sL - tok0));
+        const int n_bias = (int)(p.bias_rows - tok0 < 0 ? 0 : (p.bias_rows - tok0 > kHalfT ? kHalfT : p.bias_rows - tok0));
+        const int n_grp = (int)(swin0 - tok0 < 0 ? 0 : (swin0 - tok0 > kHalfT ? kHalfT : swin0 - tok0));
         // Some of this thread's groups are condensed: the window starts at a
         // multiple of g, which may fall inside the thread's 32 tokens, so the
         // choice is made per group (grp[]).  For g = 64 a group is the whole
@@ -779,13 +785,13 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         const bool half_groups = kFast || ((g > 1) && (tok0 < swin0));
         bool grp[NGT];
 #pragma unroll
-        for (int gi = 0; gi < NGT; ++gi) grp[gi] = kFast || (half_groups && (tok0 + gi * GW < swin0));
+        for (int gi = 0; gi < NGT; ++gi) grp[gi] = kFast || (half_groups && gi * GW < n_grp);
 
         float f[NGT], Sg[NGT], deng[NGT], own_den[NGT], ent = -INFINITY;
         if constexpr (!kFast && g == 1) {
 #pragma unroll
           for (int t = 0; t < kHalfT; ++t)
-            if (tok0 + t < swin0 && LCA_CHECK(p.err, tok0 + t < snG, 0xE05))
+            if (t < n_grp && LCA_CHECK(p.err, tok0 + t < snG, 0xE05))
               anc[tok0 + t] = (int32_t)(p.pos0 + tok0 + t);
         }
         if (half_groups) {
@@ -841,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
 #pragma unroll
                 for (int t = 0; t < GW; ++t) {
                   s[gi * GW + t] = x[gi * GW + t] + sr[gi * GW + t];
-                  if (tok0 + gi * GW + t < sL) ent = fmaxf(ent, s[gi * GW + t]);
+                  if (gi * GW + t < n_in) ent = fmaxf(ent, s[gi * GW + t]);
                 }
               }
             }
@@ -849,8 +855,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         } else {   // window tokens (and g = 1): the entry is the token itself
 #pragma unroll
           for (int t = 0; t < kHalfT; ++t) {
-            s[t] = x[t] + sr[t] + (tok0 + t < p.bias_rows ? p.bias : 0.f);
-            if (tok0 + t < sL) ent = fmaxf(ent, s[t]);
+            s[t] = x[t] + sr[t] + (t < n_bias ? p.bias : 0.f);
+            if (t < n_in) ent = fmaxf(ent, s[t]);
           }
         }
 
@@ -903,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
               if (grp[t / GW]) {
                 v = s[t] * f[t / GW];
               } else {
-                v = tok0 + t < sL ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
+                v = t < n_in ? ex2(fmaf(s[t], kLog2e, mb)) : 0.f;
                 Z += v;
               }
               pv[e2] = v;
