@@ -700,9 +700,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     float M = -INFINITY, Z = 0.f;
     int64_t cseq = seq0, ctile = tile0, ctps = tps0;
     // the current sequence's length, groups and first window token
-    // (32-bit in the paged kernel: the registers are short there)
-    using SeqInt = std::conditional_t<kPaged, int32_t, int64_t>;
-    SeqInt sL = 0, snG = 0, swin0 = 0;
+    // (32-bit: token positions fit, anchors are int32 and B L rows are bounded by
+    // the TMA coordinates; the registers are short here)
+    int32_t sL = 0, snG = 0, swin0 = 0;
     int64_t s_of = -1;
     int seg = 0;
     int64_t i = 0;
@@ -718,9 +718,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           swin0 = snG * g;
         }
       } else {
-        sL = p.L;
-        snG = p.nG;
-        swin0 = p.win0;
+        sL = (int32_t)p.L;
+        snG = (int32_t)p.nG;
+        swin0 = (int32_t)p.win0;
       }
       const int buf = (int)(i & 1);
       if (!warp_wait(&bb.s_full[buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x800)) break;
@@ -761,7 +761,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         if (!load_qr(nb, seg)) break;
       }
 
-      const int64_t tok0 = tile * kT + kHalfT * k;
+      const int32_t tile0 = (int32_t)tile * kT;         // first token of the tile
+      const int32_t tok0 = tile0 + kHalfT * k;
       int32_t* anc = p.anchor + ((int64_t)b * p.H + h) * p.anchor_stride;
       const bool first = i == 0 || tile == 0;
       float alpha = 1.f;
@@ -835,9 +836,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           if (g <= kHalfT || k == 0) {
 #pragma unroll
             for (int gi = 0; gi < NGT; ++gi) {
-              const int64_t jg = (tile * kT + (g <= kHalfT ? kHalfT * k + gi * GW : 0)) / g;
+              const int32_t jg = (tile0 + (g <= kHalfT ? kHalfT * k + gi * GW : 0)) / g;
               if (grp[gi] && LCA_CHECK(p.err, jg >= 0 && jg < snG && ag[gi] >= 0 && ag[gi] < kT, 0xE04))
-                anc[jg] = (int32_t)(p.pos0 + tile * kT + ag[gi]);
+                anc[jg] = (int32_t)p.pos0 + tile0 + ag[gi];
             }
           }
           if constexpr (!kFast) {
@@ -918,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
           }
         }
       };
-      const bool fast = g > 1 && (tile + 1) * kT <= swin0;   // warp-uniform
+      const bool fast = g > 1 && tile0 + kT <= swin0;   // warp-uniform
       if (fast) tile_math(std::true_type{});
       else tile_math(std::false_type{});
       if (*abort_flag) break;
