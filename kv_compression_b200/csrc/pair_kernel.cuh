@@ -219,12 +219,15 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
   return bounded_wait_slow(bar, parity, abort, p, where, honour_abort);
 }
 
+// A wait of a whole warp: every lane probes the same phase (one shared-memory
+// request for the warp, no divergent branch and no broadcast of a verdict),
+// and each lane acquires the phase itself.  A lane that finds the phase
+// incomplete takes the bounded loop; the warp reconverges at its next
+// warp-wide instruction.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const PairParams& p, int where) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, abort, p, where, true);
-  __syncwarp();
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return bounded_wait_slow(bar, parity, abort, p, where, true);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -238,14 +241,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Pairwise (tree) maximum over N compile-time-indexed values: depth log2 N
-// instead of a chain of N - 1 dependent operations.
+// Maximum of s[0..N), the lowest index attaining it and sr at that index, as
+// a pairwise tree: depth log2 N instead of a chain of N dependent selects.  A
+// node keeps its left (lower-index) half unless the right half's maximum is
+// strictly greater, so each subtree returns its lowest-index maximum.
 template <int N>
-__device__ __forceinline__ float tree_max(const float* v) {
+__device__ __forceinline__ void tree_argmax(const float* s, const float* sr, int base, float& m, int& a,
+                                            float& sra) {
   if constexpr (N == 1) {
-    return v[0];
+    m = s[0];
+    a = base;
+    sra = sr[0];
   } else {
-    return fmaxf(tree_max<N / 2>(v), tree_max<N / 2>(v + N / 2));
+    float m0, m1, r0, r1;
+    int a0, a1;
+    tree_argmax<N / 2>(s, sr, base, m0, a0, r0);
+    tree_argmax<N / 2>(s + N / 2, sr + N / 2, base + N / 2, m1, a1, r1);
+    const bool right = m1 > m0;
+    m = right ? m1 : m0;
+    a = right ? a1 : a0;
+    sra = right ? r1 : r0;
   }
 }
 
@@ -269,16 +284,7 @@ __device__ __forceinline__ void group_stats(const float* x, const float* sr, flo
 #pragma unroll
     for (int t = 0; t < N; t += 2)
       ptx::f32x2_split(ptx::add_f32x2(ptx::f32x2(x[t], x[t + 1]), ptx::f32x2(sr[t], sr[t + 1])), s[t], s[t + 1]);
-    m = tree_max<N>(s);
-    // scanning down, the last hit is the lowest index attaining the maximum
-    a = 0;
-    sra = sr[0];
-#pragma unroll
-    for (int t = N - 1; t >= 0; --t) {
-      const bool hit = s[t] == m;
-      a = hit ? t : a;
-      sra = hit ? sr[t] : sra;
-    }
+    tree_argmax<N>(s, sr, 0, m, a, sra);
     const float mb = -m * kLog2e;
     const uint64_t l2e = ptx::f32x2(kLog2e, kLog2e), mb2 = ptx::f32x2(mb, mb);
     uint64_t nacc = ptx::f32x2(0.f, 0.f), dacc = ptx::f32x2(0.f, 0.f);

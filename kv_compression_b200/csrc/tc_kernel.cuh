@@ -189,16 +189,17 @@ __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.  The
-// warp reconverges here even when the caller ignores the verdict, so the
-// other lanes wait at this barrier rather than at the next aligned tcgen05
-// instruction.
+// A wait of a whole warp: every lane probes the same phase once inline (one
+// shared-memory request for the warp, no divergent branch); a lane that finds
+// it incomplete takes the sleeping bounded loop.  The warp reconverges here
+// even when the caller ignores the verdict, so no lane waits at the next
+// aligned tcgen05 instruction instead.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const TcParams& p, int where) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, abort, p, where, true);
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const bool ok = bounded_wait(bar, parity, abort, p, where, true);
   __syncwarp();
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  return ok;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
