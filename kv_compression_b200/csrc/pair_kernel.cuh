@@ -105,7 +105,7 @@ constexpr int kOffRecv = kOffP + 2 * kPBytes;
 constexpr int kOffAlpha = kOffRecv + kRecvBytes;           // [2][128] float: the rescale factor per head
 constexpr int kOffFlag = kOffAlpha + 2 * kHeads * 4;       // int [2]: peer rows need a rescale
 constexpr int kOffBar = kOffFlag + 16;
-constexpr int kNumBars = 53;
+constexpr int kNumBars = 57;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -173,6 +173,7 @@ struct Bars {
   uint64_t* sr_empty;    // the softmax warps have read sr
   uint64_t* recv_full;   // [4] quarter q of the peer's partial scores landed (transaction bytes)
   uint64_t* recv_free;   // [4] the peer's quarter q has read the partial scores sent to it
+  uint64_t* recv_used;   // [4] this CTA's softmax warp of quarter q has read the received partials
   uint64_t* p_local;     // [2] the own rows of P buffer b are written (one barrier per buffer: a
                          // single one could run two phases ahead of the O issuer's wait)
   uint64_t* p_remote;    // [2 x 4] quarter q of the peer's rows of P buffer b landed (transaction bytes)
@@ -344,7 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.resc_done = bb.resc_go + 1;
   bb.part_done = bb.resc_done + 1;
   bb.drain = bb.part_done + 1;
-  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 ==
+  bb.recv_used = bb.drain + 2;
+  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 + 4 ==
                     kNumBars,
                 "barrier count");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -413,7 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     ptx::mbar_init(bb.sr_empty, 4);               // the 4 softmax warps
     for (int q = 0; q < 4; ++q) {
       ptx::mbar_init(&bb.recv_full[q], 1);        // armed with its transaction bytes
-      ptx::mbar_init(&bb.recv_free[q], 1);        // the peer's softmax warp of quarter q
+      ptx::mbar_init(&bb.recv_free[q], 1);        // the peer's shipper warp of quarter q
+      ptx::mbar_init(&bb.recv_used[q], 1);        // this CTA's softmax warp of quarter q
       ptx::mbar_init(&bb.p_remote[q], 1);         // armed with its transaction bytes
       ptx::mbar_init(&bb.p_remote[4 + q], 1);
     }
@@ -675,7 +678,6 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     const int h = h0 + m;
     const uint32_t lanes = (uint32_t)(32 * q + 16 * r) << 16;
     const uint32_t lanes_peer = (uint32_t)(32 * q + 16 * peer) << 16;
-    const uint32_t peer_recv_free = ptx::mapa(ptx::smem_u32(&bb.recv_free[q]), peer);
     const uint32_t peer_p_remote0 = ptx::mapa(ptx::smem_u32(&bb.p_remote[q]), peer);
     const uint32_t peer_p_remote1 = ptx::mapa(ptx::smem_u32(&bb.p_remote[4 + q]), peer);
     const int row0 = 32 * q + 16 * r;            // this warp's 16 P rows (2 KB) and factors
@@ -756,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         // this quarter's buffer takes the next tile's partials: armed before the
         // peer may send them
         if (i + 1 < n_tiles) ptx::mbar_arrive_expect_tx(&bb.recv_full[q], kRecvQBytes);
-        ptx::mbar_arrive_remote(peer_recv_free);
+        // the received partials are read: the quarter's shipper tells the peer
+        ptx::mbar_arrive(&bb.recv_used[q]);
       }
       // the next sequence's q_r, for the sr MMA of the tile after this one
       if (last_of_part(i, tile, ctps) && i + 1 < n_tiles) {
@@ -1038,9 +1041,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   } else if (warp >= 7) {
     // ===================================================== shipper (peer heads of quarter q)
     // Thread (hi, k): peer head m = 32 q + 16 peer + hi, tokens 32 k .. of a tile.
-    // Iteration i: send the partial scores of tile i + 1 to the peer; then, one
-    // tile behind, do what O of tile i - 1 asked of these heads' O rows: the
-    // rescale (rare), and at the end of a sequence part the write-out.
+    // Iteration i: tell the peer that this CTA's softmax has read the partials
+    // of tile i, and send it those of tile i + 1; then, one tile behind, do what
+    // O of tile i - 1 asked of these heads' O rows: the rescale (rare), and at
+    // the end of a sequence part the write-out.
     const int q = warp & 3;
     const int hi = lane & 15, k = lane >> 4;
     const int m = 32 * q + 16 * peer + hi;
@@ -1048,9 +1052,20 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     const uint32_t lanes = (uint32_t)(32 * q + 16 * peer) << 16;
     const uint32_t peer_row = ptx::mapa(ptx::smem_u32(recv + olp * kT), peer);
     const uint32_t peer_recv_full = ptx::mapa(ptx::smem_u32(&bb.recv_full[q]), peer);
+    const uint32_t peer_recv_free = ptx::mapa(ptx::smem_u32(&bb.recv_free[q]), peer);
     int n_resc = 0, n_part = 0;
+    // This CTA's softmax warp of quarter q has read the partials of tile t: the
+    // peer may overwrite them.  The release at cluster scope is taken here, off
+    // the softmax warp's path; it covers the softmax's reads, which its
+    // CTA-scope release on recv_used ordered before this warp's acquire.
+    auto forward = [&](int64_t t) -> bool {
+      if (!warp_wait(&bb.recv_used[q], (uint32_t)t & 1, abort_flag, p, 0x905)) return false;
+      if (lane == 0) ptx::mbar_arrive_remote(peer_recv_free);
+      return true;
+    };
     auto ship = [&](int64_t t) -> bool {
       const int buf = (int)(t & 1);
+      if (t >= 1 && !forward(t - 1)) return false;
       if (!warp_wait(&bb.sc_full[buf], (uint32_t)(t >> 1) & 1, abort_flag, p, 0x900)) return false;
       ptx::tc_fence_after();
       float v[32];
@@ -1127,7 +1142,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     if (ok && i == n_tiles && n_tiles > 0) {
       behind(n_tiles - 1, bseq, btile, btps);
       // the peer's release of the last partial scores has landed here before this CTA exits
-      if (lane == 0)
+      if (forward(n_tiles - 1) && lane == 0)
         bounded_wait(&bb.recv_free[q], (uint32_t)(n_tiles - 1) & 1, abort_flag, p, 0x9F0, true);
     }
   }
