@@ -103,9 +103,9 @@ constexpr int kOffKr = kOffC + kNS * kStage;
 constexpr int kOffP = kOffKr + kNKr * kKrBytes;            // [2] P tiles
 constexpr int kOffRecv = kOffP + 2 * kPBytes;
 constexpr int kOffAlpha = kOffRecv + kRecvBytes;           // [2][128] float: the rescale factor per head
-constexpr int kOffFlag = kOffAlpha + 2 * kHeads * 4;       // int [2]: peer rows need a rescale
+constexpr int kOffFlag = kOffAlpha + 2 * kHeads * 4;       // int [4]: peer rows need a rescale
 constexpr int kOffBar = kOffFlag + 16;
-constexpr int kNumBars = 57;
+constexpr int kNumBars = 59;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -178,8 +178,8 @@ struct Bars {
                          // single one could run two phases ahead of the O issuer's wait)
   uint64_t* p_remote;    // [2 x 4] quarter q of the peer's rows of P buffer b landed (transaction bytes)
   uint64_t* p_free;      // [2 x 2] index 2 c + b: O of CTA c done with P buffer b (and every O before)
-  uint64_t* lanes_ready; // the shippers finished what precedes O of a tile (the tile before's rows)
-  uint64_t* dec;         // [2] the O issuer's decision for a tile (flag: rescale the peer rows)
+  uint64_t* part_written; // the shippers wrote out their rows of a sequence part (one phase per part)
+  uint64_t* dec;         // [4] the O issuer's decision for a tile (flag: rescale the peer rows)
   uint64_t* resc_go;     // every O issued before a rescale request is done
   uint64_t* resc_done;   // the shippers rescaled the peer rows as asked
   uint64_t* part_done;   // the last O of a sequence part is done (one phase per part)
@@ -339,14 +339,14 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.p_local = bb.recv_free + 4;
   bb.p_remote = bb.p_local + 2;
   bb.p_free = bb.p_remote + 8;
-  bb.lanes_ready = bb.p_free + 4;
-  bb.dec = bb.lanes_ready + 1;
-  bb.resc_go = bb.dec + 2;
+  bb.part_written = bb.p_free + 4;
+  bb.dec = bb.part_written + 1;
+  bb.resc_go = bb.dec + 4;
   bb.resc_done = bb.resc_go + 1;
   bb.part_done = bb.resc_done + 1;
   bb.drain = bb.part_done + 1;
   bb.recv_used = bb.drain + 2;
-  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 + 4 ==
+  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 + 4 + 2 ==
                     kNumBars,
                 "barrier count");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -409,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       ptx::mbar_init(&bb.sc_full[i], 1);
       ptx::mbar_init(&bb.sc_empty[i], 8);         // 4 softmax + 4 shipper warps
       ptx::mbar_init(&bb.dec[i], 1);
+      ptx::mbar_init(&bb.dec[2 + i], 1);
       ptx::mbar_init(&bb.drain[i], 1);
     }
     for (int i = 0; i < 4; ++i) ptx::mbar_init(&bb.p_free[i], 1);   // one O commit (multicast)
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     }
     ptx::mbar_init(&bb.p_local[0], 4);            // the 4 softmax warps
     ptx::mbar_init(&bb.p_local[1], 4);
-    ptx::mbar_init(bb.lanes_ready, 4);            // the 4 shipper warps
+    ptx::mbar_init(bb.part_written, 4);           // the 4 shipper warps
     ptx::mbar_init(bb.resc_go, 1);
     ptx::mbar_init(bb.resc_done, 4);
     ptx::mbar_init(bb.part_done, 1);
@@ -609,16 +610,20 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   } else if (warp == 2 && lane == 0) {
     // ===================================================== O MMA issuer
     // Tile j once P buffer j & 1 is complete (own rows, the peer's rows and
-    // factors) and the shippers are done with the tile before: if a peer
-    // factor is not 1, the shippers rescale those heads' O rows first (rare).
-    // Then O[128 x 256] += P[128 x 64] . C_KV[tile, dims_r] (A K-major from
-    // the P buffer, B MN-major from the tile's stage), four K steps of 16
-    // tokens; a sequence part starts afresh.  The release of the P buffer is
-    // signalled in both CTAs (each writes into the other's).
+    // factors), and, when a sequence part ended with the tile before, once the
+    // shippers have written out their rows of it.  The decision for tile j
+    // goes to the shippers on one of four barriers (they run at most three
+    // tiles behind: O of tile j needs the peer's partials of tile j, which
+    // the peer sends once this CTA's shippers have finished tile j - 3): if a
+    // peer factor is not 1, the shippers rescale those heads' O rows first
+    // (rare).  Then O[128 x 256] += P[128 x 64] . C_KV[tile, dims_r] (A
+    // K-major from the P buffer, B MN-major from the tile's stage), four K
+    // steps of 16 tokens; a sequence part starts afresh.  The release of the
+    // P buffer is signalled in both CTAs (each writes into the other's).
     constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(kHeads, kDim, 0, 1);   // A K-major, B MN-major
     const uint64_t d_p = ptx::smem_desc(ptx::smem_u32(smem + kOffP), 16, 1024, ptx::kSwizzle128B);
     const uint64_t d_cb = ptx::smem_desc(ptx::smem_u32(smem + kOffC), kCAtom, 1024, ptx::kSwizzle128B);
-    int n_resc = 0;
+    int n_resc = 0, n_pw = 0;
     int64_t oseq = seq0, otile = tile0, otps = tps0;
     for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile, otps)) {
       const int buf = (int)(j & 1);
@@ -631,7 +636,12 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       // them only after this CTA's O of tile j is done
       if (j + 2 < n_tiles)
         for (int q = 0; q < 4; ++q) ptx::mbar_arrive_expect_tx(&bb.p_remote[4 * buf + q], kPQBytes);
-      if (!bounded_wait(bb.lanes_ready, (uint32_t)j & 1, abort_flag, p, 0x702, true)) break;
+      // a part ended with the tile before: the shippers have written out their
+      // rows of it before this tile's O starts the next part over them
+      if (j > 0 && otile == 0) {
+        if (!bounded_wait(bb.part_written, (uint32_t)n_pw & 1, abort_flag, p, 0x702, true)) break;
+        ++n_pw;
+      }
       bool resc = false;
       if (j > 0 && otile > 0) {
         const float* al = alpha_s + kHeads * buf;
@@ -646,8 +656,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         }
       }
       if (resc) ptx::mma_commit(bb.resc_go);       // lands once every O issued so far is done
-      dec_flag[j & 1] = resc ? 1 : 0;
-      ptx::mbar_arrive(&bb.dec[j & 1]);
+      dec_flag[j & 3] = resc ? 1 : 0;
+      ptx::mbar_arrive(&bb.dec[j & 3]);
       if (resc) {
         if (!bounded_wait(bb.resc_done, (uint32_t)n_resc & 1, abort_flag, p, 0x703, true)) break;
         ++n_resc;
@@ -1084,8 +1094,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     };
     // what O of tile j needed of these heads' rows, done after O of tile j
     auto behind = [&](int64_t j, int64_t b, int64_t tile, int64_t tps) -> bool {
-      if (!warp_wait(&bb.dec[j & 1], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x902)) return false;
-      if (dec_flag[j & 1]) {
+      if (!warp_wait(&bb.dec[j & 3], (uint32_t)(j >> 2) & 1, abort_flag, p, 0x902)) return false;
+      if (dec_flag[j & 3]) {
         // every O before tile j is done (one phase per request, seen in order)
         const float a = alpha_s[kHeads * (j & 1) + m];
         if (!warp_wait(bb.resc_go, (uint32_t)n_resc & 1, abort_flag, p, 0x903)) return false;
@@ -1124,6 +1134,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
             *reinterpret_cast<float4*>(dst + 64 * cc + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
         }
         ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bb.part_written);
       }
       return true;
     };
@@ -1136,8 +1148,6 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         if (!(ok = behind(i - 1, bseq, btile, btps))) break;
         step(bseq, btile, btps);
       }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bb.lanes_ready);
     }
     if (ok && i == n_tiles && n_tiles > 0) {
       behind(n_tiles - 1, bseq, btile, btps);
