@@ -716,6 +716,41 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       return true;
     };
     float M = -INFINITY, Z = 0.f;
+    // A sequence part's partial (this head's O row over this CTA's dims, and
+    // (M, Z)) is written out one tile later, just before that tile's P: the
+    // next tile then starts without waiting for the part's last O, which may
+    // wait for a rescale by the shippers, who reach it only once this warp
+    // has started the next tile.  O of the next tile, which starts the next
+    // part over these rows, needs that tile's P, so it comes after.
+    bool pend = false;
+    int pend_buf = 0;
+    uint32_t pend_par = 0;
+    int64_t pend_slot = 0;
+    float pend_M = 0.f, pend_Z = 0.f;
+    auto write_part = [&]() -> bool {
+      const bool slot_ok = LCA_CHECK(p.err, pend_slot < p.ws_slots, 0xE06);
+      // the part's last O is done once its P buffer is released
+      if (!warp_wait(&bb.p_free[2 * r + pend_buf], pend_par, abort_flag, p, 0x806)) return false;
+      ptx::tc_fence_after();
+      float* dst = p.part_o + (pend_slot * p.H + h) * (int64_t)kDC + kDim * r + 32 * k;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float o[32];
+        ptx::tmem_ld16x2_32(tmem + lanes + kColO + 64u * cc, o);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; t += 4)
+          if (slot_ok)
+            *reinterpret_cast<float4*>(dst + 64 * cc + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
+      }
+      ptx::tc_fence_before();
+      if (k == 0 && slot_ok) {
+        p.part_mz[(pend_slot * p.H + h) * 2 + 0] = pend_M;
+        p.part_mz[(pend_slot * p.H + h) * 2 + 1] = pend_Z;
+      }
+      pend = false;
+      return true;
+    };
     int64_t cseq = seq0, ctile = tile0, ctps = tps0;
     // the current sequence's length, groups and first window token
     // (32-bit: token positions fit, anchors are int32 and B L rows are bounded by
@@ -963,6 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
       }
+      if (pend && !write_part()) break;
       // A paged sequence's last tile: its stage rows past the last token hold
       // whatever the pool has there.  Their weights are 0, but 0 x NaN is not,
       // so the four softmax warps clear those rows before O reads the stage
@@ -1011,35 +1047,18 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ptx::mbar_arrive(&bb.p_local[buf]);
       }
 
-      if (last_of_part(i, tile, ctps)) {
-        // the partial of the range's part of sequence b: this head's O row over
-        // this CTA's dims, and (owner) its (M, Z).  O of tile i is done when
-        // buffer i & 1 is released (this warp saw its previous release above).
-        const int64_t slot = b + c;
-        const bool slot_ok = LCA_CHECK(p.err, slot < p.ws_slots, 0xE06);
-        if (!warp_wait(&bb.p_free[2 * r + buf], (uint32_t)(i >> 1) & 1, abort_flag, p, 0x806)) break;
-        ptx::tc_fence_after();
-        float* dst = p.part_o + (slot * p.H + h) * (int64_t)kDC + kDim * r + 32 * k;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float o[32];
-          ptx::tmem_ld16x2_32(tmem + lanes + kColO + 64u * cc, o);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 32; t += 4)
-            if (slot_ok)
-              *reinterpret_cast<float4*>(dst + 64 * cc + t) = make_float4(o[t], o[t + 1], o[t + 2], o[t + 3]);
-        }
-        ptx::tc_fence_before();
-        const float zh = Z + __shfl_xor_sync(0xffffffffu, Z, 16);
-        if (k == 0 && slot_ok) {
-          p.part_mz[(slot * p.H + h) * 2 + 0] = M;
-          p.part_mz[(slot * p.H + h) * 2 + 1] = zh;
-        }
+      if (last_of_part(i, tile, ctps)) {   // written out before the next tile's P
+        pend = true;
+        pend_buf = buf;
+        pend_par = (uint32_t)(i >> 1) & 1;
+        pend_slot = b + c;
+        pend_M = M;
+        pend_Z = Z + __shfl_xor_sync(0xffffffffu, Z, 16);
         M = -INFINITY;
         Z = 0.f;
       }
     }
+    if (pend && i == n_tiles) write_part();
     if (lane == 0 && copy_pending) ptx::bulk_wait_group_read0();
     // The peer O issuer's releases of the last two P buffers (multicast into
     // this CTA's shared memory) have landed before this CTA exits.

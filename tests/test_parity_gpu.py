@@ -124,6 +124,38 @@ def test_pair_kernel_rescale():
         compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
 
 
+def test_pair_rescales_and_part_ends_back_to_back():
+    """Short sequences (five tiles, the last partial) whose scores rise past the
+    rescale threshold in every tile: the O issuer's rescale decisions come tile
+    after tile, and with few clusters a sequence part ends every few tiles of
+    a range, so the shippers' write-outs, the decisions and the rescales follow
+    each other closely.  Repeated at several cluster counts, for g = 16 and 64."""
+    from workloads import bf16_bits_to_f32, f32_to_bf16_bits
+    for g, w, seed in ((16, 40, 31), (64, 44, 32)):
+        wl = workloads.small("t", B=6, H=128, L=300, g=g, w=w, seed=seed)
+        x = workloads.generate(wl)
+        c = bf16_bits_to_f32(x.c_kv).copy()
+        k = bf16_bits_to_f32(x.k_r).copy()
+        for b in range(wl.B):
+            qdir = np.concatenate([bf16_bits_to_f32(x.q_c[b]), bf16_bits_to_f32(x.q_r[b])], axis=1)
+            u = qdir.mean(axis=0)
+            u /= np.linalg.norm(u)
+            for n, t in enumerate((20, 84, 148, 212, 276)):     # one rise in each tile
+                row = (12.0 * (n + 1) * np.sqrt(576.0) * u).astype(np.float32)
+                c[b, t] = row[:512]
+                k[b, t] = row[512:]
+        x.c_kv = f32_to_bf16_bits(c)
+        x.k_r = f32_to_bf16_bits(k)
+        d = DeviceInputs(x)
+        ref = oracle_lca(x, wl.g, wl.w)
+        for n in (2, 4, 10, 148):
+            plan = make_plan(wl, {kvc.OPT_NUM_CTAS: n})
+            assert plan.kernel(wl.L, wl.g, wl.w) == "tcgen05_pair"
+            for _ in range(3):
+                out, anc = run_lca(plan, d, wl.g, wl.w)
+                compare(out, anc, ref, BF16_TOL, exact_anchors=False, x=x, g=wl.g)
+
+
 def test_pair_ranges_spanning_sequences():
     """Few clusters: every tile range of the two-CTA kernel crosses sequence
     boundaries (query reloads, partials in several slots)."""
