@@ -90,7 +90,8 @@ constexpr int kRecvBytes = kOwn * kT * 4;   // partial scores from the peer, 16 
 // quarter waits only for its rows and each barrier takes a quarter of the
 // transaction updates.
 constexpr int kRecvQBytes = kRecvBytes / 4;               // 16 heads x 64 tokens x 4 B
-constexpr int kPQBytes = 16 * kT * 2 + 16 * 4;            // 16 rows of P + their 16 factors
+constexpr int kFacChunk = 20;                             // 16 factors, a flag word, 3 words of padding
+constexpr int kPQBytes = 16 * kT * 2 + kFacChunk * 4;     // 16 rows of P + their factors and flag
 constexpr int kThreads = 32 * 11;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -102,8 +103,11 @@ constexpr int kOffC = kOffQc + kAtoms * kQcAtom;
 constexpr int kOffKr = kOffC + kNS * kStage;
 constexpr int kOffP = kOffKr + kNKr * kKrBytes;            // [2] P tiles
 constexpr int kOffRecv = kOffP + 2 * kPBytes;
-constexpr int kOffAlpha = kOffRecv + kRecvBytes;           // [2][128] float: the rescale factor per head
-constexpr int kOffFlag = kOffAlpha + 2 * kHeads * 4;       // int [4]: peer rows need a rescale
+// [2 buffers][4 quarters][2 CTAs] chunks of kFacChunk floats: the rescale
+// factors of a quarter's 16 rows of one CTA, then a flag word (1 when one of
+// them is not 1), copied to the peer with the rows of P
+constexpr int kOffAlpha = kOffRecv + kRecvBytes;
+constexpr int kOffFlag = kOffAlpha + 2 * 4 * 2 * kFacChunk * 4;   // int [4]: peer rows need a rescale
 constexpr int kOffBar = kOffFlag + 16;
 constexpr int kNumBars = 59;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -353,7 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* dec_flag = reinterpret_cast<volatile int*>(smem + kOffFlag);
   float* recv = reinterpret_cast<float*>(smem + kOffRecv);
-  float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);   // [2][128]
+  float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
+  // the chunk of (P buffer, lane quarter, CTA)
+  auto fac_chunk = [&](int buf, int q, int rank) -> int { return ((buf * 4 + q) * 2 + rank) * kFacChunk; };
 
   const int64_t cl = blockIdx.x >> 1;
   const int hb = (int)(cl % p.n_hb);
@@ -643,17 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         ++n_pw;
       }
       bool resc = false;
-      if (j > 0 && otile > 0) {
-        const float* al = alpha_s + kHeads * buf;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4* a4 = reinterpret_cast<const float4*>(al + 32 * q + 16 * peer);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 a = a4[v];
-            resc = resc || a.x != 1.f || a.y != 1.f || a.z != 1.f || a.w != 1.f;
-          }
-        }
+      if (j > 0 && otile > 0) {   // a factor of the peer's rows is not 1: one flag per quarter
+        const volatile float* al = alpha_s;
+        resc = (__float_as_int(al[fac_chunk(buf, 0, peer) + 16]) | __float_as_int(al[fac_chunk(buf, 1, peer) + 16]) |
+                __float_as_int(al[fac_chunk(buf, 2, peer) + 16]) | __float_as_int(al[fac_chunk(buf, 3, peer) + 16])) != 0;
       }
       if (resc) ptx::mma_commit(bb.resc_go);       // lands once every O issued so far is done
       dec_flag[j & 3] = resc ? 1 : 0;
@@ -978,7 +977,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       else tile_math(std::false_type{});
       if (*abort_flag) break;
 
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      const bool any_resc = __any_sync(0xffffffffu, alpha != 1.f);
+      if (any_resc) {
         // this head's O row must be complete (O of tile i - 1) before it is
         // scaled here; this warp saw buffer (i - 1) & 1's earlier release when
         // it wrote P of tile i - 1
@@ -1028,7 +1028,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
         for (int j = 0; j < 4; ++j)
           *reinterpret_cast<uint4*>(row + 16 * ((4 * k + j) ^ (m & 7))) =
               make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        if (k == 0) alpha_s[kHeads * buf + m] = alpha;
+        if (k == 0) alpha_s[fac_chunk(buf, q, r) + hi] = alpha;
+        if (lane == 0) alpha_s[fac_chunk(buf, q, r) + 16] = __int_as_float(any_resc ? 1 : 0);
       }
       ptx::fence_proxy_async_smem();                 // visible to the MMA's and the copy's reads
       __syncwarp();
@@ -1039,9 +1040,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       if (lane == 0) {
         const uint32_t bar = buf ? peer_p_remote1 : peer_p_remote0;
         const uint8_t* rows = smem + kOffP + buf * kPBytes + row0 * 128;
-        const float* fac = alpha_s + kHeads * buf + row0;
+        const float* fac = alpha_s + fac_chunk(buf, q, r);
         ptx::bulk_copy_to_peer(ptx::mapa(ptx::smem_u32(rows), peer), rows, 16 * 128, bar);
-        ptx::bulk_copy_to_peer(ptx::mapa(ptx::smem_u32(fac), peer), fac, 16 * 4, bar);
+        ptx::bulk_copy_to_peer(ptx::mapa(ptx::smem_u32(fac), peer), fac, kFacChunk * 4, bar);
         ptx::bulk_commit_group();
         copy_pending = true;
         ptx::mbar_arrive(&bb.p_local[buf]);
@@ -1116,7 +1117,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       if (!warp_wait(&bb.dec[j & 3], (uint32_t)(j >> 2) & 1, abort_flag, p, 0x902)) return false;
       if (dec_flag[j & 3]) {
         // every O before tile j is done (one phase per request, seen in order)
-        const float a = alpha_s[kHeads * (j & 1) + m];
+        const float a = alpha_s[fac_chunk((int)(j & 1), q, peer) + hi];
         if (!warp_wait(bb.resc_go, (uint32_t)n_resc & 1, abort_flag, p, 0x903)) return false;
         ++n_resc;
         ptx::tc_fence_after();
