@@ -109,7 +109,7 @@ constexpr int kOffRecv = kOffP + 2 * kPBytes;
 constexpr int kOffAlpha = kOffRecv + kRecvBytes;
 constexpr int kOffFlag = kOffAlpha + 2 * 4 * 2 * kFacChunk * 4;   // int [4]: peer rows need a rescale
 constexpr int kOffBar = kOffFlag + 16;
-constexpr int kNumBars = 59;
+constexpr int kNumBars = 53;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
@@ -180,7 +180,7 @@ struct Bars {
   uint64_t* recv_used;   // [4] this CTA's softmax warp of quarter q has read the received partials
   uint64_t* p_local;     // [2] the own rows of P buffer b are written (one barrier per buffer: a
                          // single one could run two phases ahead of the O issuer's wait)
-  uint64_t* p_remote;    // [2 x 4] quarter q of the peer's rows of P buffer b landed (transaction bytes)
+  uint64_t* p_remote;    // [2] the peer's rows of P buffer b landed, all four quarters (transaction bytes)
   uint64_t* p_free;      // [2 x 2] index 2 c + b: O of CTA c done with P buffer b (and every O before)
   uint64_t* part_written; // the shippers wrote out their rows of a sequence part (one phase per part)
   uint64_t* dec;         // [4] the O issuer's decision for a tile (flag: rescale the peer rows)
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.recv_free = bb.recv_full + 4;
   bb.p_local = bb.recv_free + 4;
   bb.p_remote = bb.p_local + 2;
-  bb.p_free = bb.p_remote + 8;
+  bb.p_free = bb.p_remote + 2;
   bb.part_written = bb.p_free + 4;
   bb.dec = bb.part_written + 1;
   bb.resc_go = bb.dec + 4;
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
   bb.part_done = bb.resc_done + 1;
   bb.drain = bb.part_done + 1;
   bb.recv_used = bb.drain + 2;
-  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 8 + 4 + 1 + 2 + 1 + 1 + 1 + 2 + 4 + 2 ==
+  static_assert(2 * kNS + 2 * kNKr + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 4 + 4 + 2 + 2 + 4 + 1 + 2 + 1 + 1 + 1 + 2 + 4 + 2 ==
                     kNumBars,
                 "barrier count");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
@@ -424,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
       ptx::mbar_init(&bb.recv_full[q], 1);        // armed with its transaction bytes
       ptx::mbar_init(&bb.recv_free[q], 1);        // the peer's shipper warp of quarter q
       ptx::mbar_init(&bb.recv_used[q], 1);        // this CTA's softmax warp of quarter q
-      ptx::mbar_init(&bb.p_remote[q], 1);         // armed with its transaction bytes
-      ptx::mbar_init(&bb.p_remote[4 + q], 1);
     }
+    ptx::mbar_init(&bb.p_remote[0], 1);           // armed with the four quarters' transaction bytes
+    ptx::mbar_init(&bb.p_remote[1], 1);
     ptx::mbar_init(&bb.p_local[0], 4);            // the 4 softmax warps
     ptx::mbar_init(&bb.p_local[1], 4);
     ptx::mbar_init(bb.part_written, 4);           // the 4 shipper warps
@@ -436,10 +436,10 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     *abort_flag = 0;
     ptx::fence_mbarrier_init();
     // the first phases of the barriers the peer completes with transaction bytes
+    ptx::mbar_arrive_expect_tx(&bb.p_remote[0], 4 * kPQBytes);
+    ptx::mbar_arrive_expect_tx(&bb.p_remote[1], 4 * kPQBytes);
     for (int q = 0; q < 4; ++q) {
       ptx::mbar_arrive_expect_tx(&bb.recv_full[q], kRecvQBytes);
-      ptx::mbar_arrive_expect_tx(&bb.p_remote[q], kPQBytes);
-      ptx::mbar_arrive_expect_tx(&bb.p_remote[4 + q], kPQBytes);
     }
   }
   if (warp == 1) {
@@ -634,14 +634,11 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     for (int64_t j = 0; j < n_tiles; ++j, step(oseq, otile, otps)) {
       const int buf = (int)(j & 1);
       if (!bounded_wait(&bb.p_local[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x700, true)) break;
-      bool ok = true;
-      for (int q = 0; q < 4 && ok; ++q)
-        ok = bounded_wait(&bb.p_remote[4 * buf + q], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x701, true);
-      if (!ok) break;
+      if (!bounded_wait(&bb.p_remote[buf], (uint32_t)(j >> 1) & 1, abort_flag, p, 0x701, true)) break;
       // this buffer takes the peer's rows of tile j + 2 next; the peer writes
       // them only after this CTA's O of tile j is done
       if (j + 2 < n_tiles)
-        for (int q = 0; q < 4; ++q) ptx::mbar_arrive_expect_tx(&bb.p_remote[4 * buf + q], kPQBytes);
+        ptx::mbar_arrive_expect_tx(&bb.p_remote[buf], 4 * kPQBytes);
       // a part ended with the tile before: the shippers have written out their
       // rows of it before this tile's O starts the next part over them
       if (j > 0 && otile == 0) {
@@ -687,8 +684,8 @@ __global__ void __launch_bounds__(kThreads, 1) lca_pair_kernel(const __grid_cons
     const int h = h0 + m;
     const uint32_t lanes = (uint32_t)(32 * q + 16 * r) << 16;
     const uint32_t lanes_peer = (uint32_t)(32 * q + 16 * peer) << 16;
-    const uint32_t peer_p_remote0 = ptx::mapa(ptx::smem_u32(&bb.p_remote[q]), peer);
-    const uint32_t peer_p_remote1 = ptx::mapa(ptx::smem_u32(&bb.p_remote[4 + q]), peer);
+    const uint32_t peer_p_remote0 = ptx::mapa(ptx::smem_u32(&bb.p_remote[0]), peer);
+    const uint32_t peer_p_remote1 = ptx::mapa(ptx::smem_u32(&bb.p_remote[1]), peer);
     const int row0 = 32 * q + 16 * r;            // this warp's 16 P rows (2 KB) and factors
     bool copy_pending = false;
     // q_r of sequence `seq` (segment s) into TMEM buffer s & 1, both lane
