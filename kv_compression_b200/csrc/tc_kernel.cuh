@@ -169,13 +169,14 @@ __device__ __forceinline__ void record_timeout(volatile int* abort, const TcPara
   if (atomicOr(p.err, kErrTimeout) == 0) atomicExch(p.err + 1, where);
 }
 
-// Bounded wait.  Returns false when the CTA's abort flag is set (if honoured)
-// or when the bound runs out (then the flag and the error word are set).
-// The thread sleeps in hardware between probes (up to 1 us each, woken when
-// the phase completes), so waiting threads take no issue slots from the
-// softmax warps on their sub-partition.
-__device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          const TcParams& p, int where, bool honour_abort) {
+// Bounded wait, the loop after a first probe that found the phase incomplete.
+// Returns false when the CTA's abort flag is set (if honoured) or when the
+// bound runs out (then the flag and the error word are set).  The thread
+// sleeps in hardware between probes (up to 1 us each, woken when the phase
+// completes), so waiting threads take no issue slots from the softmax warps on
+// their sub-partition.
+__device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               const TcParams& p, int where, bool honour_abort) {
   constexpr uint32_t kSleepNs = 1000;
   if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
@@ -189,6 +190,15 @@ __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait: the first probe plain and inline, because most waits find the
+// phase complete and a first probe with a suspend-time hint (or a call) cost
+// the hand-off time.
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             const TcParams& p, int where, bool honour_abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return bounded_wait_slow(bar, parity, abort, p, where, honour_abort);
+}
+
 // A wait of a whole warp: every lane probes the same phase once inline (one
 // shared-memory request for the warp, no divergent branch); a lane that finds
 // it incomplete takes the sleeping bounded loop.  The warp reconverges here
@@ -197,7 +207,7 @@ __device__ __noinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           const TcParams& p, int where) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
-  const bool ok = bounded_wait(bar, parity, abort, p, where, true);
+  const bool ok = bounded_wait_slow(bar, parity, abort, p, where, true);
   __syncwarp();
   return ok;
 }
