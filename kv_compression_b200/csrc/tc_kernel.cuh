@@ -172,12 +172,12 @@ __device__ __forceinline__ void record_timeout(volatile int* abort, const TcPara
 // Bounded wait, the loop after a first probe that found the phase incomplete.
 // Returns false when the CTA's abort flag is set (if honoured) or when the
 // bound runs out (then the flag and the error word are set).  The thread
-// sleeps in hardware between probes (up to 1 us each, woken when the phase
-// completes), so waiting threads take no issue slots from the softmax warps on
-// their sub-partition.
+// sleeps in hardware between probes (up to 100 ns each, woken when the phase
+// completes), so waiting threads take few issue slots from the softmax warps
+// on their sub-partition; a longer hint (1 us) measured 1% slower.
 __device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                const TcParams& p, int where, bool honour_abort) {
-  constexpr uint32_t kSleepNs = 1000;
+  constexpr uint32_t kSleepNs = 100;
   if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t spin = 1;; ++spin) {
