@@ -31,9 +31,10 @@
 //              (bulk shared-to-distributed-shared copies) into the peer's, so
 //              O of a tile starts as soon as both halves have landed.  M rises
 //              only when an entry exceeds it by more than 2^8; the owner
-//              rescales its O rows, and the factor travels with P so that the
-//              O MMA issuer of the other CTA has its receiving warps rescale
-//              that CTA's copy of the rows first (rare).
+//              rescales its O rows, and the factors (with one flag per lane
+//              quarter) travel with P so that the O MMA issuer of the other
+//              CTA has its shipper warps rescale that CTA's copy of the rows
+//              first (rare).
 // Each CTA writes its dims of every head's partial O, the owner CTA the
 // head's (M, Z); the combine kernel merges the ranges of a sequence.
 //
@@ -46,11 +47,13 @@
 //
 // Roles (352 threads): warp 0 lane 0 issues TMA loads; warp 1 allocates TMEM
 // and its lane 0 issues the score MMAs; warp 2 lane 0 issues the O MMAs and
-// decides, from the peer's factors, whether a tile needs the peer rows
-// rescaled; warps 3-6 run the softmax of the own heads of lane quarter
-// (warp % 4) and load each sequence's q_r into TMEM; warps 7-10 ship the
-// partial scores of the peer heads of their quarter a tile ahead and, one tile
-// behind, rescale (on request) and write out those heads' O rows.
+// decides, from the peer's per-quarter flags, whether a tile needs the peer
+// rows rescaled; warps 3-6 run the softmax of the own heads of lane quarter
+// (warp % 4) and load each sequence's q_r into TMEM; warps 7-10 tell the peer
+// when their quarter's softmax has read the received partials (the
+// cluster-scope release, kept off the softmax warps), ship the partial scores
+// of the peer heads of their quarter a tile ahead and, one tile behind,
+// rescale (on request) and write out those heads' O rows.
 // Completion of O is only ever waited on barriers whose every phase the
 // waiter observes in order (a parity wait on a barrier two phases ahead would
 // pass early).  Waits suspend in hardware (mbarrier.try_wait) and are bounded;
