@@ -191,9 +191,11 @@ lca_status launch_combine(const lca_plan* p, const lca::CombineParams& cp_in, cu
     cp.n_slots = (int64_t)cp.n_split * p->B;
     cp.err = p->err;
   }
+  cp.vec = (p->d_c % lca::kCombineVec == 0) && (reinterpret_cast<uintptr_t>(cp.part_o) % 16 == 0) &&
+           (reinterpret_cast<uintptr_t>(cp.out) % 16 == 0) ? 1 : 0;
+  constexpr int kDimsPerBlock = lca::kCombineThreads * lca::kCombineVec;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p->H, (unsigned)p->B,
-                     (unsigned)((p->d_c + lca::kCombineThreads - 1) / lca::kCombineThreads));
+  cfg.gridDim = dim3((unsigned)p->H, (unsigned)p->B, (unsigned)((p->d_c + kDimsPerBlock - 1) / kDimsPerBlock));
   cfg.blockDim = dim3(lca::kCombineThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
